@@ -1,0 +1,416 @@
+"""Benchmark of the MISA token indexer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload chunk_128k] [--h 8]
+
+One step = the whole indexer over one long-context prefill chunk: pool the
+131072 keys into 1024 blocks, route every (query, head) against them and keep
+the top-8 heads, score the causal prefix of all 8192 queries with their routed
+heads (fused ReLU * w head-sum on the tensor cores, in 1024-query sub-chunks),
+and select the top-2048 tokens per query.  Inputs are seeded synthetic arrays
+of the chunk's shape (clustered keys, head-specific query mixtures), resident in
+HBM when the timed region starts.  L2 is flushed (a 256 MiB write) before every
+timed step; all times are CUDA events on the launching stream.
+
+N > 1 (torchrun, one process per GPU): every rank indexes its own chunk
+(independent problems, no data-path collective), timing is the max over ranks
+and `value` is the whole-job milliseconds per chunk (max step time / N).
+
+--impl reference times the CPU oracle (the fp64 restatement of the method) on a
+bounded sample of the same workload and extrapolates to the chunk.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from long_context_sparse_block_b200 import workloads as W  # noqa: E402
+
+METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor peak"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        loaded = [x for x in sm if mx and x > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+_SHARED = {}
+
+
+def _oracle_worker(rows):
+    """One single-threaded oracle over query rows (route + score + top-k each)."""
+    import oracle
+    wl, h = _SHARED["wl"], _SHARED["h"]
+    Kd, kbar, inp = _SHARED["Kd"], _SHARED["kbar"], _SHARED["inp"]
+    Qd_rows = oracle.bf16_to_f64(inp["Q"][rows])
+    wd = inp["w"][rows].astype(np.float64)
+    t0 = time.perf_counter()
+    for i, t in enumerate(rows):
+        pos = wl.q_pos0 + int(t)
+        r, hd = oracle.route(Qd_rows[i:i + 1], wd[i:i + 1], kbar, pos, wl.n_k, wl.B, h)
+        lg = oracle.score(Qd_rows[i:i + 1], wd[i:i + 1], hd, Kd, pos)
+        oracle.topk(lg, pos, wl.n_k, wl.k)
+    return time.perf_counter() - t0, len(rows)
+
+
+def cpu_baseline(wl: W.Workload, h: int, inp: dict, budget_s: float = 15.0) -> dict:
+    """Times the oracle as it stands (route + score + top-k per query; keys pooled
+    once) on a seeded sample of query rows, one single-threaded oracle process per
+    core, and extrapolates to milliseconds per chunk.  Must run before any CUDA
+    call: the worker processes are forked."""
+    import oracle
+    oracle.build()
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    workers = max(1, min(cores, 32))
+    Kd = oracle.bf16_to_f64(inp["K"])
+    _SHARED.update(wl=wl, h=h, inp=inp, Kd=Kd, kbar=oracle.pool_keys(Kd, wl.B))
+    rng = np.random.default_rng(12345)
+    cal_t, _ = _oracle_worker([wl.n_q - 1])
+    per_worker = max(1, min(64, int(budget_s / max(cal_t, 1e-3))))
+    n_rows = min(wl.n_q, per_worker * workers)
+    rows = np.sort(rng.choice(wl.n_q, size=n_rows, replace=False))
+    parts = [rows[i::workers].tolist() for i in range(workers)]
+    t0 = time.perf_counter()
+    with mp.get_context("fork").Pool(workers) as pool:
+        res = pool.map(_oracle_worker, [p for p in parts if p])
+    wall = time.perf_counter() - t0
+    per_query = sum(t for t, _ in res) / sum(n for _, n in res)   # single-thread s/query
+    ms_chunk = per_query * wl.n_q / workers * 1e3
+    return {"value": round(ms_chunk, 1), "unit": "ms", "cores": workers, "kind": "oracle",
+            "sample": f"{n_rows} of {wl.n_q} query rows of {wl.name} (route + score + top-k "
+                      f"each), {workers} single-threaded oracle processes, {wall:.1f} s wall; "
+                      f"extrapolated to the whole chunk",
+            "per_query_s": round(per_query, 4)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args, rank, world, local_rank, inp):
+    import torch
+    import torch.distributed as dist
+
+    from long_context_sparse_block_b200 import _lib
+    from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
+
+    torch.cuda.set_device(local_rank)
+    wl = W.WORKLOADS[args.workload]
+    h = args.h or wl.h
+    if world > 1:
+        rng = np.random.default_rng(1000 + rank)
+        perm = rng.permutation(wl.n_q)
+        inp["Q"], inp["w"] = inp["Q"][perm].copy(), inp["w"][perm].copy()
+
+    def d16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+    Q, K, w = d16(inp["Q"]), d16(inp["K"]), torch.from_numpy(inp["w"]).cuda()
+    shape = IndexerShape(wl.n_q, wl.q_pos0, wl.n_k, wl.H, wl.d, wl.B, h, wl.k,
+                         sub_chunk=args.sub_chunk)
+    ix = MisaIndexer(shape)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    # per-stage events: wrap the library calls of one step
+    stage_events = []
+
+    def step(record):
+        ev = []
+        s = shape
+        e0 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        _lib.misa_pool_keys(K, s.B, kbar_hl=ix.kbar_hl, want_kbar=False)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e1.record(stream)
+        _lib.misa_route_heads(Q, w, ix.kbar_hl, s.q_pos0, s.n_k, s.B, s.h, heads=ix.heads)
+        e2 = torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+        ev += [("pool", e0, e1), ("route", e1, e2)]
+        prev = e2
+        for c0 in range(0, s.n_q, ix.sub):
+            c1 = min(s.n_q, c0 + ix.sub)
+            lg = ix.logits[:c1 - c0]
+            _lib.misa_score_tokens(Q[c0:c1], w[c0:c1], ix.heads[c0:c1], K, s.q_pos0 + c0,
+                                   logits=lg, h=s.h)
+            ea = torch.cuda.Event(enable_timing=True)
+            ea.record(stream)
+            _lib.misa_topk(lg, s.q_pos0 + c0, s.n_k, s.k, idx=ix.sel[c0:c1])
+            eb = torch.cuda.Event(enable_timing=True)
+            eb.record(stream)
+            ev += [("score", prev, ea), ("topk", ea, eb)]
+            prev = eb
+        if record:
+            stage_events.append(ev)
+        return e0, prev
+
+    launches_per_step = 2 + 2 * math.ceil(wl.n_q / ix.sub)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(False)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+    spans = []
+    for _ in range(args.steps):
+        flush.zero_()
+        spans.append(step(True))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop() if rank == 0 else None
+    assert _lib.misa_last_device_status() == 0, "device status"
+    step_ms = [a.elapsed_time(b) for a, b in spans]
+    stage_ms = {}
+    for ev in stage_events:
+        for name, a, b in ev:
+            stage_ms[name] = stage_ms.get(name, 0.0) + a.elapsed_time(b)
+    stage_ms = {k: v / args.steps for k, v in stage_ms.items()}
+    ms = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end through the public API from pinned host buffers
+    Qh = torch.from_numpy(inp["Q"].view(np.int16)).pin_memory()
+    Kh = torch.from_numpy(inp["K"].view(np.int16)).pin_memory()
+    wh = torch.from_numpy(inp["w"]).pin_memory()
+    idx_h = torch.empty(ix.final.shape, dtype=torch.int32).pin_memory()
+    e2e_ms = []
+    for i in range(0 if args.no_e2e else args.warmup + args.steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Q.copy_(Qh, non_blocking=True)
+        K.copy_(Kh, non_blocking=True)
+        w.copy_(wh, non_blocking=True)
+        out = ix.run(Q, K, w)
+        idx_h.copy_(out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = statistics.mean(e2e_ms) if e2e_ms else float("nan")
+    if world > 1:
+        t = torch.tensor([e2e], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = float(t.item())
+    if rank != 0:
+        return None
+
+    peaks = _peaks()
+    pairs = wl.causal_pairs()
+    score_flops = 2.0 * h * wl.d * pairs
+    score_ms = stage_ms["score"]
+    tflops = score_flops / (score_ms * 1e-3) / 1e12
+    topk_gbs = 4.0 * pairs / (stage_ms["topk"] * 1e-3) / 1e9
+    pool_gbs = (wl.n_k * wl.d * 2 + 2 * wl.M * wl.d * 2) / (stage_ms["pool"] * 1e-3) / 1e9
+    rt = wl.n_q * wl.H * 2 * wl.d * sum(min((p + 1) // wl.B, wl.n_k // wl.B)
+                                        for p in wl.positions().tolist())
+    route_tflops = 2 * rt / (stage_ms["route"] * 1e-3) / 1e12  # hi and lo contractions
+    h2d = inp["Q"].nbytes + inp["K"].nbytes + inp["w"].nbytes
+    d2h = idx_h.numel() * 4
+    out = {
+        "metric": METRIC,
+        "value": round(ms / world, 4),
+        "unit": "ms",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": (f"{wl.name}: {wl.n_q} queries at {wl.q_pos0}..{wl.q_pos0 + wl.n_q - 1} "
+                         f"x {wl.n_k} keys, H_I={wl.H}, d={wl.d}, B={wl.B}, h={h}, k={wl.k}"),
+            "query_sub_chunk": ix.sub,
+            "l2": "flushed by a 256 MiB write before every timed step",
+            "parallelism": f"independent chunks per rank x{world}",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "score_tokens (tcgen05, fused ReLU*w head-sum epilogue)",
+            "achieved": round(tflops, 1),
+            "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s",
+            "frac": round(tflops / peaks["bf16_tflops"], 4),
+            "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
+            "traffic": None,
+            "algorithmic": f"2*h*d*pairs = {score_flops:.4g} flop per step, {pairs} causal pairs",
+        },
+        "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "stage_rates": {
+            "score_tflops": round(tflops, 1),
+            "route_tflops_hi_lo": round(route_tflops, 1),
+            "topk_logit_gbs": round(topk_gbs, 1),
+            "pool_gbs": round(pool_gbs, 1),
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+            "pairs_per_s": round(pairs / (ms * 1e-3), 1),
+        },
+        "e2e": {"value": round(e2e / world, 4), "unit": "ms", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    return out
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    wl = W.WORKLOADS[args.workload]
+    h = args.h or wl.h
+    t0 = time.perf_counter()
+    cb = cpu_baseline(wl, h, W.generate(wl), budget_s=args.cpu_budget)
+    return {"metric": METRIC, "value": cb["value"], "unit": "ms", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["value"],
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{wl.name}", "h": h},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "ms", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "wall_s": round(time.perf_counter() - t0, 1)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="chunk_128k")
+    ap.add_argument("--h", type=int, default=0)
+    ap.add_argument("--sub-chunk", type=int, default=1024)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    # the oracle's process pool is spawned before any CUDA work
+    wl = W.WORKLOADS[args.workload]
+    inp = W.generate(wl)  # each rank indexes its own chunk (same shape)
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(wl, args.h or wl.h, inp, budget_s=args.cpu_budget)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank, inp)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if out is not None:
+        if cb is not None:
+            out["cpu_baseline"] = cb
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

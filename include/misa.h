@@ -1,0 +1,146 @@
+/*
+ * misa.h — C ABI of the MISA token indexer library (libmisa.so, sm_100a).
+ *
+ * MISA ("MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
+ * Inference") replaces the DeepSeek-Sparse-Attention lightning indexer.  Per
+ * query it (1) mean-pools the shared index keys into M = ceil(L/B) block keys,
+ * (2-3) routes: scores every indexer head against the pooled keys and keeps the
+ * top-h heads, (4) lets only those heads score the causal prefix token by token,
+ * and (5) keeps the top-k tokens.  The hierarchical variant (MISA-dagger) keeps a
+ * larger routed candidate set and re-scores it with all heads.  (Technical
+ * summary, Metodologia steps 1-2 and Variante Hierarquica; abstract.)
+ *
+ * Shapes and layouts (all row-major, all pointers are DEVICE pointers owned by
+ * the caller unless stated otherwise):
+ *   Q       [n_q, H, d]  bf16 (uint16 codes)  index queries, H = H_I heads
+ *   K       [n_k, d]     bf16 codes, or FP8 E4M3 codes with k_scale [n_k] fp32
+ *                        (value = e4m3(code) * k_scale[s])
+ *   w       [n_q, H]     fp32 per-query head weights
+ *   kbar    [M, d]       fp32 pooled block keys
+ *   kbar_hl [2, M, d]    bf16: hi = bf16(kbar), lo = bf16(kbar - hi)
+ *   heads   [n_q, h]     int32 routed heads, ascending head index
+ *   logits  [n_q, ld]    fp32
+ *   idx     [n_q, k]     int32 token indices, ascending, padded with -1
+ * Query t sits at position pos(t) = q_pos0 + t and sees keys 0..pos(t); every
+ * call requires q_pos0 >= 0 and q_pos0 + n_q <= n_k.  d must be 32, 64 or 128.
+ *
+ * Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ * stream), validates its arguments before launching anything and returns a
+ * misa_status.  Argument errors launch nothing.  Device-side faults detected by
+ * the kernels' own checks (a bounded wait that ran out, a value outside its
+ * contract) are recorded in a per-device status word read by
+ * misa_last_device_status().  No entry point allocates device memory.
+ */
+#ifndef MISA_H_
+#define MISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum misa_status {
+    MISA_OK = 0,
+    MISA_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, size out of range */
+    MISA_ERR_UNSUPPORTED = -2,  /* a shape the kernels do not implement (d, H, h) */
+    MISA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
+    MISA_ERR_TIMEOUT = -4,      /* a kernel's bounded wait ran out (device status) */
+    MISA_ERR_WORKSPACE = -5,    /* workspace pointer/size too small */
+    MISA_ERR_DEVICE = -6        /* a kernel detected an input outside its contract */
+} misa_status;
+
+typedef enum misa_kdtype {
+    MISA_K_BF16 = 0,
+    MISA_K_FP8E4M3 = 1
+} misa_kdtype;
+
+/*
+ * Stage 1 — block mean-pooling of the index keys (Metodologia step 1: keys split
+ * into M = ceil(n_k/B) blocks, each summarised by its mean key).
+ *   kbar[m, :] = (1/n_m) * sum_{s = mB}^{mB+n_m-1} K[s, :],  n_m = min(B, n_k - mB)
+ * Sums in fp32.  Writes kbar (nullable) and kbar_hl (nullable; hi/lo bf16 split
+ * used by misa_route_heads).  K: 16-byte aligned; k_scale required iff
+ * kdtype == MISA_K_FP8E4M3.  1 <= B <= 4096.
+ */
+int misa_pool_keys(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d, int B,
+                   float* kbar, uint16_t* kbar_hl, void* stream);
+
+/*
+ * Stages 2-3 — router and top-h (Metodologia step 1: per-head affinities
+ * against the pooled keys, aggregated into one importance per head; keep the
+ * top-h heads).  The aggregate is
+ *   r[t, j] = w[t, j] * sum_{m in C(t)} ReLU(q[t, j] . kbar_m),
+ *   C(t) = { m : (m+1)B - 1 <= pos(t), m < floor(n_k/B) }  (complete causal blocks)
+ * with kbar_m = hi_m + lo_m read from kbar_hl ([2, M, d], M = ceil(n_k/B)).
+ * heads[t, :] = the h heads of largest r, ties to the lower index, written in
+ * ascending head order.  r_out (nullable) receives r.  H must divide 128
+ * (H in {1,2,4,...,128}); 1 <= h <= H.  Q and kbar_hl 16-byte aligned.
+ */
+int misa_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl, int n_q,
+                     int64_t q_pos0, int64_t n_k, int H, int d, int B, int h, int32_t* heads,
+                     float* r_out, void* stream);
+
+/*
+ * Stage 4 — routed token scoring (Metodologia step 2: only the h routed heads
+ * score the prefix token by token).
+ *   logits[t, s] = sum_{i < h} w[t, j_i] * ReLU(q[t, j_i] . k_s),  j_i = heads[t, i],
+ * for s <= pos(t).  heads == NULL scores with all H heads (h must equal H): the
+ * dense DSA lightning indexer (Declaracao do Problema).  For FP8 keys the
+ * product uses the decoded code and the per-token scale multiplies the dot
+ * product before the ReLU.  Entries s > pos(t) are not part of the result:
+ * those in a 128-key tile that also holds causal keys are written -inf, the
+ * rest are left untouched.  h must be a power of two <= 128; ld >= n_k.
+ * Q, K, logits 16-byte aligned.
+ */
+int misa_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
+                      const float* k_scale, int kdtype, int n_q, int64_t q_pos0, int64_t n_k,
+                      int H, int d, int h, float* logits, int64_t ld, void* stream);
+
+/*
+ * Stage 5 — top-k token selection (technical summary, Metodologia step 2: the
+ * final top-k tokens come from the reduced scores).  For each row t, among
+ * logits[t, 0..min(pos(t), n_k-1)] keep the k largest, ties to the lower token
+ * index (-0.0 equals +0.0), and write their indices ascending into idx[t, :],
+ * padded with -1 when fewer than k tokens are visible.  Rows must hold no NaN.
+ * logits 16-byte aligned with ld a multiple of 4.  0 <= k <= 16384.
+ * ws/ws_bytes: workspace, size from misa_workspace_size("topk", ...) (may be 0).
+ */
+int misa_topk(const float* logits, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k, int k,
+              int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * MISA-dagger fine stage (Variante Hierarquica: the original all-head indexer
+ * re-scores the k' routed candidates and the final top-k comes from them).
+ *   full[t, i] = sum_{j < H} w[t, j] * ReLU(q[t, j] . k_{c}),  c = cand[t, i]
+ * Entries c outside 0..pos(t) (including the -1 padding) are ignored.  The k
+ * candidates of largest full score, ties to the lower token index, are written
+ * ascending to idx[t, :], -1 padded.  full_logits (nullable, [n_q, kp]) receives
+ * full, -inf where ignored.  Candidates must be distinct.  H <= 128 and a
+ * multiple of 16; 1 <= kp <= 16384; 0 <= k <= kp.
+ * ws/ws_bytes: workspace, size from misa_workspace_size("rerank", ...).
+ */
+int misa_rerank(const uint16_t* Q, const float* w, const void* K, const float* k_scale, int kdtype,
+                const int32_t* cand, int kp, int n_q, int64_t q_pos0, int64_t n_k, int H, int d,
+                int k, int32_t* idx, float* full_logits, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes needed by op "topk" or "rerank" for the given sizes (0 if none). */
+size_t misa_workspace_size(const char* op, int n_q, int64_t n_k, int k, int kp);
+
+/* Static text for a misa_status value. */
+const char* misa_status_string(int status);
+
+/* Synchronises `stream`, returns and clears the device status word of the
+ * current device (MISA_OK, MISA_ERR_TIMEOUT or MISA_ERR_DEVICE). */
+int misa_last_device_status(void* stream);
+
+/* Sets the time budget of every bounded device-side wait, in nanoseconds
+ * (default 2e9; 0 restores the default).  Diagnostic knob: a tiny value makes
+ * kernels give up and report MISA_ERR_TIMEOUT instead of waiting. */
+int misa_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MISA_H_ */

@@ -1,0 +1,192 @@
+"""ctypes binding of libmisa.so — argument marshalling only.
+
+Every function here checks tensor devices/dtypes/shapes, allocates outputs with
+torch when the caller gives none, and calls the C entry point of the same name
+on the current torch CUDA stream.  No step of the indexer runs in Python; when
+the library is missing the import fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmisa.so")
+
+MISA_OK = 0
+MISA_ERR_INVALID_ARG = -1
+MISA_ERR_UNSUPPORTED = -2
+MISA_ERR_CUDA = -3
+MISA_ERR_TIMEOUT = -4
+MISA_ERR_WORKSPACE = -5
+MISA_ERR_DEVICE = -6
+MISA_K_BF16 = 0
+MISA_K_FP8E4M3 = 1
+
+
+class MisaError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn} -> {status} ({text})")
+        self.status = status
+
+
+_vp, _i64, _int, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+_SIGS = {
+    "misa_pool_keys": (_int, [_vp, _vp, _int, _i64, _int, _int, _vp, _vp, _vp]),
+    "misa_route_heads": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _int, _int, _int, _int, _vp, _vp,
+                                _vp]),
+    "misa_score_tokens": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _int, _int, _int,
+                                 _vp, _i64, _vp]),
+    "misa_topk": (_int, [_vp, _i64, _int, _i64, _i64, _int, _vp, _vp, _sz, _vp]),
+    "misa_rerank": (_int, [_vp, _vp, _vp, _vp, _int, _vp, _int, _int, _i64, _i64, _int, _int, _int,
+                           _vp, _vp, _vp, _sz, _vp]),
+    "misa_workspace_size": (_sz, [ctypes.c_char_p, _int, _i64, _int, _int]),
+    "misa_status_string": (ctypes.c_char_p, [_int]),
+    "misa_last_device_status": (_int, [_vp]),
+    "misa_set_wait_limit_ns": (_int, [ctypes.c_uint64]),
+}
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m long_context_sparse_block_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = load_library()
+
+
+def _check(fn: str, status: int):
+    if status != MISA_OK:
+        raise MisaError(fn, status, _lib.misa_status_string(status).decode())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t, dtypes=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+_BF16_CODES = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def _kdtype(K):
+    return MISA_K_FP8E4M3 if K.dtype in (torch.uint8, torch.float8_e4m3fn) else MISA_K_BF16
+
+
+# ---------------------------------------------------------------- stage calls
+
+def misa_pool_keys(K, B: int, k_scale=None, kbar=None, kbar_hl=None, want_kbar: bool = True):
+    """K [n_k, d] bf16 codes (or e4m3 codes + k_scale) -> (kbar [M,d] f32, kbar_hl [2,M,d])."""
+    n_k, d = K.shape
+    M = -(-n_k // B)
+    if kbar is None and want_kbar:
+        kbar = torch.empty((M, d), dtype=torch.float32, device=K.device)
+    if kbar_hl is None:
+        kbar_hl = torch.empty((2, M, d), dtype=torch.int16, device=K.device)
+    st = _lib.misa_pool_keys(_ptr(K, name="K"), _ptr(k_scale, (torch.float32,), "k_scale"),
+                             _kdtype(K), n_k, d, B, _ptr(kbar, (torch.float32,), "kbar"),
+                             _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), _stream())
+    _check("misa_pool_keys", st)
+    return kbar, kbar_hl
+
+
+def misa_route_heads(Q, w, kbar_hl, q_pos0: int, n_k: int, B: int, h: int, heads=None,
+                     want_r: bool = False):
+    """Q [n_q,H,d], w [n_q,H] f32, kbar_hl [2,M,d] -> (heads [n_q,h] int32, r [n_q,H] or None)."""
+    n_q, H, d = Q.shape
+    if heads is None:
+        heads = torch.empty((n_q, h), dtype=torch.int32, device=Q.device)
+    r = torch.empty((n_q, H), dtype=torch.float32, device=Q.device) if want_r else None
+    st = _lib.misa_route_heads(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                               _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), n_q, q_pos0, n_k, H, d, B, h,
+                               _ptr(heads, (torch.int32,), "heads"), _ptr(r, (torch.float32,), "r"),
+                               _stream())
+    _check("misa_route_heads", st)
+    return heads, r
+
+
+def misa_score_tokens(Q, w, heads, K, q_pos0: int, k_scale=None, logits=None, h: int | None = None):
+    """Fused routed logits [n_q, ld] f32 (heads None: all H heads, the dense indexer)."""
+    n_q, H, d = Q.shape
+    n_k = K.shape[0]
+    if h is None:
+        h = heads.shape[1] if heads is not None else H
+    if logits is None:
+        logits = torch.empty((n_q, n_k), dtype=torch.float32, device=Q.device)
+    ld = logits.stride(0) if logits.dim() == 2 else n_k
+    st = _lib.misa_score_tokens(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                                _ptr(heads, (torch.int32,), "heads"), _ptr(K, name="K"),
+                                _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K), n_q, q_pos0,
+                                n_k, H, d, h, ctypes.c_void_p(logits.data_ptr()), ld, _stream())
+    _check("misa_score_tokens", st)
+    return logits
+
+
+def misa_topk(logits, q_pos0: int, n_k: int, k: int, idx=None, n_q: int | None = None):
+    """Top-k token indices [n_q, k] int32 (ascending, -1 padded) of fp32 logits rows."""
+    if n_q is None:
+        n_q = logits.shape[0]
+    if idx is None:
+        idx = torch.empty((n_q, k), dtype=torch.int32, device=logits.device)
+    st = _lib.misa_topk(ctypes.c_void_p(logits.data_ptr()), logits.stride(0), n_q, q_pos0, n_k, k,
+                        _ptr(idx, (torch.int32,), "idx"), None, 0, _stream())
+    _check("misa_topk", st)
+    return idx
+
+
+def misa_workspace_size(op: str, n_q: int, n_k: int, k: int, kp: int) -> int:
+    return int(_lib.misa_workspace_size(op.encode(), n_q, n_k, k, kp))
+
+
+def misa_rerank(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, want_full: bool = False,
+                idx=None, ws=None):
+    """MISA-dagger: all-head rescoring of candidates [n_q, kp] -> idx [n_q, k] (and full scores)."""
+    n_q, H, d = Q.shape
+    n_k = K.shape[0]
+    kp = cand.shape[1]
+    if idx is None:
+        idx = torch.empty((n_q, k), dtype=torch.int32, device=Q.device)
+    full = torch.empty((n_q, kp), dtype=torch.float32, device=Q.device) if want_full else None
+    ws_bytes = 0
+    if full is None:
+        ws_bytes = misa_workspace_size("rerank", n_q, n_k, k, kp)
+        if ws is None or ws.numel() * ws.element_size() < ws_bytes:
+            ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=Q.device)
+    st = _lib.misa_rerank(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"), _ptr(K, name="K"),
+                          _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K),
+                          _ptr(cand, (torch.int32,), "cand"), kp, n_q, q_pos0, n_k, H, d, k,
+                          _ptr(idx, (torch.int32,), "idx"), _ptr(full, (torch.float32,), "full"),
+                          _ptr(ws, name="ws") if full is None else None, ws_bytes, _stream())
+    _check("misa_rerank", st)
+    return (idx, full) if want_full else idx
+
+
+def misa_last_device_status() -> int:
+    return int(_lib.misa_last_device_status(_stream()))
+
+
+def misa_set_wait_limit_ns(ns: int) -> None:
+    _check("misa_set_wait_limit_ns", _lib.misa_set_wait_limit_ns(ns))
+
+
+def misa_status_string(status: int) -> str:
+    return _lib.misa_status_string(status).decode()

@@ -1,0 +1,247 @@
+// C ABI of libmisa (declared in include/misa.h): argument validation, the
+// per-device status word, the bounded-wait budget, TMA descriptor encoding and
+// the stage launches.  Nothing here allocates device memory.
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "misa.h"
+
+namespace misa {
+
+namespace {
+
+__device__ int g_device_status;  // one per device that loads the library
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_status_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+std::atomic<unsigned long long> g_wait_ns{2000000000ull};
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+int* status_ptr() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool make_ctl(DevCtl& ctl) {
+  ctl.status = status_ptr();
+  ctl.wait_ns = g_wait_ns.load();
+  return ctl.status != nullptr;
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                              CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                              CUtensorMapFloatOOBfill);
+EncodeFn g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool good_d(int d) { return d == 32 || d == 64 || d == 128; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MISA_OK : MISA_ERR_CUDA; }
+
+}  // namespace
+
+int sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sm_count[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+CUresult encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                           const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                           CUtensorMapSwizzle swz) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return CUDA_ERROR_NOT_FOUND;
+      g_encode = reinterpret_cast<EncodeFn>(fn);
+    }
+  }
+  cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+                  reinterpret_cast<const cuuint64_t*>(dims),
+                  reinterpret_cast<const cuuint64_t*>(strides_bytes),
+                  reinterpret_cast<const cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace misa
+
+using namespace misa;
+
+extern "C" {
+
+int misa_pool_keys(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d, int B,
+                   float* kbar, uint16_t* kbar_hl, void* stream) {
+  if (!K || !aligned16(K) || n_k < 1 || !good_d(d) || B < 1 || B > 4096) return MISA_ERR_INVALID_ARG;
+  if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
+  if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
+  if (!kbar && !kbar_hl) return MISA_ERR_INVALID_ARG;
+  if ((kbar && !aligned4(kbar)) || (kbar_hl && (reinterpret_cast<uintptr_t>(kbar_hl) & 1u)))
+    return MISA_ERR_INVALID_ARG;
+  if ((n_k + B - 1) / B > 0x7fffffff) return MISA_ERR_INVALID_ARG;
+  return cuda_status(launch_pool_keys(K, k_scale, kdtype == MISA_K_FP8E4M3, n_k, d, B, kbar, kbar_hl,
+                                      as_stream(stream)));
+}
+
+int misa_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl, int n_q,
+                     int64_t q_pos0, int64_t n_k, int H, int d, int B, int h, int32_t* heads,
+                     float* r_out, void* stream) {
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !kbar_hl || !aligned16(kbar_hl) || !heads ||
+      !aligned4(heads))
+    return MISA_ERR_INVALID_ARG;
+  if (r_out && !aligned4(r_out)) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || B < 1 || h < 1 || h > H)
+    return MISA_ERR_INVALID_ARG;
+  if (!good_d(d) || !pow2(H) || H > 128) return MISA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(n_q) * H > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
+  if (n_q == 0) return MISA_OK;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  return cuda_status(launch_route_heads(Q, w, kbar_hl, n_q, q_pos0, n_k, H, d, B, h, heads, r_out,
+                                        ctl, as_stream(stream)));
+}
+
+int misa_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
+                      const float* k_scale, int kdtype, int n_q, int64_t q_pos0, int64_t n_k, int H,
+                      int d, int h, float* logits, int64_t ld, void* stream) {
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !K || !aligned16(K) || !logits ||
+      !aligned4(logits))
+    return MISA_ERR_INVALID_ARG;
+  if (heads && !aligned4(heads)) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || H < 1 || h < 1 || h > H ||
+      ld < n_k)
+    return MISA_ERR_INVALID_ARG;
+  if (!heads && h != H) return MISA_ERR_INVALID_ARG;
+  if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
+  if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
+  if (!good_d(d) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
+  if (kdtype == MISA_K_FP8E4M3) return MISA_ERR_UNSUPPORTED;
+  if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
+  if (n_q == 0) return MISA_OK;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  return cuda_status(launch_score_tokens(Q, w, heads, K, k_scale, kdtype == MISA_K_FP8E4M3, n_q,
+                                         q_pos0, n_k, H, d, h, logits, ld, ctl, as_stream(stream)));
+}
+
+int misa_topk(const float* logits, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k, int k,
+              int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!logits || !aligned4(logits) || (k > 0 && (!idx || !aligned4(idx)))) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || k < 0 || k > 16384)
+    return MISA_ERR_INVALID_ARG;
+  if (ld < std::min<int64_t>(n_k, q_pos0 + n_q)) return MISA_ERR_INVALID_ARG;
+  if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
+  if (n_q == 0 || k == 0) return MISA_OK;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  return cuda_status(
+      launch_topk(logits, ld, n_q, q_pos0, n_k, 0, nullptr, k, idx, ctl, as_stream(stream)));
+}
+
+int misa_rerank(const uint16_t* Q, const float* w, const void* K, const float* k_scale, int kdtype,
+                const int32_t* cand, int kp, int n_q, int64_t q_pos0, int64_t n_k, int H, int d,
+                int k, int32_t* idx, float* full_logits, void* ws, size_t ws_bytes, void* stream) {
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !K || !aligned16(K) || !cand ||
+      !aligned4(cand) || (k > 0 && (!idx || !aligned4(idx))))
+    return MISA_ERR_INVALID_ARG;
+  if (full_logits && !aligned4(full_logits)) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || kp < 1 || kp > 16384 || k < 0 ||
+      k > kp || H < 1)
+    return MISA_ERR_INVALID_ARG;
+  if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
+  if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
+  if (!good_d(d) || H > 128) return MISA_ERR_UNSUPPORTED;
+  if (n_q == 0) return MISA_OK;
+  float* full = full_logits;
+  if (!full) {
+    const size_t need = misa_workspace_size("rerank", n_q, n_k, k, kp);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return MISA_ERR_WORKSPACE;
+    full = static_cast<float*>(ws);
+  }
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  const cudaStream_t s = as_stream(stream);
+  cudaError_t e = launch_rerank_scores(Q, w, K, k_scale, kdtype == MISA_K_FP8E4M3, cand, kp, n_q,
+                                       q_pos0, n_k, H, d, full, kp, ctl, s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  if (k == 0) return MISA_OK;
+  return cuda_status(launch_topk(full, kp, n_q, q_pos0, n_k, kp, cand, k, idx, ctl, s));
+}
+
+size_t misa_workspace_size(const char* op, int n_q, int64_t n_k, int k, int kp) {
+  (void)n_k;
+  (void)k;
+  if (!op || n_q <= 0) return 0;
+  if (std::strcmp(op, "rerank") == 0 && kp > 0)
+    return static_cast<size_t>(n_q) * static_cast<size_t>(kp) * sizeof(float);
+  return 0;
+}
+
+const char* misa_status_string(int status) {
+  switch (status) {
+    case MISA_OK: return "ok";
+    case MISA_ERR_INVALID_ARG: return "invalid argument";
+    case MISA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MISA_ERR_CUDA: return "CUDA error";
+    case MISA_ERR_TIMEOUT: return "device wait timed out";
+    case MISA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MISA_ERR_DEVICE: return "device detected an input outside its contract";
+  }
+  return "unknown status";
+}
+
+int misa_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MISA_ERR_CUDA;
+  int* p = status_ptr();
+  if (!p) return MISA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MISA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return MISA_ERR_CUDA;
+  switch (v) {
+    case DEV_OK: return MISA_OK;
+    case DEV_TIMEOUT: return MISA_ERR_TIMEOUT;
+    default: return MISA_ERR_DEVICE;
+  }
+}
+
+int misa_set_wait_limit_ns(uint64_t ns) {
+  g_wait_ns.store(ns ? ns : 2000000000ull);
+  return MISA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Launchers the C ABI layer (api.cu) calls; each lives beside its kernel.
+// Arguments are validated by the caller; launchers only pick configurations.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace misa {
+
+int sm_count();  // of the current device
+
+cudaError_t launch_pool_keys(const void* K, const float* k_scale, bool fp8, int64_t n_k, int d,
+                             int B, float* kbar, uint16_t* kbar_hl, cudaStream_t s);
+
+cudaError_t launch_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
+                               int n_q, int64_t q_pos0, int64_t n_k, int H, int d, int B, int h,
+                               int32_t* heads, float* r_out, const DevCtl& ctl, cudaStream_t s);
+
+cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads,
+                                const void* K, const float* k_scale, bool fp8, int n_q,
+                                int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
+                                int64_t ld, const DevCtl& ctl, cudaStream_t s);
+
+// Top-k over rows.  Token mode (cand == nullptr): row t is logits[t*ld ..] with
+// min(pos(t)+1, n_k) visible entries; writes token indices.  Candidate mode:
+// row t is vals[t*ld .. t*ld+row_len); -inf entries are absent; writes
+// cand[t*row_len + i] for the selected positions i.
+cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k,
+                        int row_len, const int32_t* cand, int k, int32_t* idx,
+                        const DevCtl& ctl, cudaStream_t s);
+
+// All-head scores of candidate keys: full[t*ldf + i] (-inf where ignored).
+cudaError_t launch_rerank_scores(const uint16_t* Q, const float* w, const void* K,
+                                 const float* k_scale, bool fp8, const int32_t* cand, int kp,
+                                 int n_q, int64_t q_pos0, int64_t n_k, int H, int d, float* full,
+                                 int64_t ldf, const DevCtl& ctl, cudaStream_t s);
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once).
+CUresult encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank,
+                           const void* base, const uint64_t* dims, const uint64_t* strides_bytes,
+                           const uint32_t* box, CUtensorMapSwizzle swz);
+
+}  // namespace misa

@@ -1,0 +1,141 @@
+// Stage 1 — block mean-pooling of the shared index keys.
+//
+// kbar[m, :] = (1/n_m) * sum of K rows mB .. mB+n_m-1, n_m = min(B, n_k - mB)
+// ("MISA" technical summary, Metodologia step 1: the prefix is split into
+// M = ceil(L/B) blocks summarised by mean-pooled index keys).
+//
+// HBM-bound stream: one CTA per block, 16-byte loads along d, fp32 partial sums
+// per (row phase, column group), combined in shared memory.  Also writes the
+// hi/lo bf16 split of kbar that the router's tensor-core contraction reads.
+#include "internal.h"
+
+namespace misa {
+namespace {
+
+constexpr int kPoolThreads = 256;
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(kPoolThreads)
+pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scale, int64_t n_k,
+                 int B, int64_t M, float* __restrict__ kbar, uint16_t* __restrict__ kbar_hl) {
+  // elements per 16-byte unit and units per row
+  constexpr int EPU = FP8 ? 16 : 8;
+  constexpr int UPR = D / EPU;                 // column groups
+  constexpr int PHASES = kPoolThreads / UPR;   // rows handled in parallel
+  static_assert(kPoolThreads % UPR == 0, "column groups must tile the block");
+  __shared__ float part[PHASES][D];
+
+  const int64_t m = blockIdx.x;
+  const int64_t first = m * B;
+  const int n_m = static_cast<int>(n_k - first < B ? n_k - first : static_cast<int64_t>(B));
+  const int u = threadIdx.x % UPR;
+  const int ph = threadIdx.x / UPR;
+  constexpr int ROW_BYTES = D * (FP8 ? 1 : 2);
+
+  float acc[EPU];
+#pragma unroll
+  for (int e = 0; e < EPU; ++e) acc[e] = 0.0f;
+
+  const uint8_t* base = K + first * ROW_BYTES + u * 16;
+  int r = ph;
+  // two rows in flight per iteration
+  for (; r + PHASES < n_m; r += 2 * PHASES) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(r) * ROW_BYTES));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(r + PHASES) * ROW_BYTES));
+    const uint4 ab[2] = {a, b};
+    float sc[2] = {1.0f, 1.0f};
+    if (FP8) {
+      sc[0] = __ldg(k_scale + first + r);
+      sc[1] = __ldg(k_scale + first + r + PHASES);
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t* wv = reinterpret_cast<const uint32_t*>(&ab[q]);
+      if (FP8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t bf2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[i >> 1] >> ((i & 1) * 16)));
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bf2));
+          acc[2 * i] += f.x * sc[q];
+          acc[2 * i + 1] += f.y * sc[q];
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[i]));
+          acc[2 * i] += f.x;
+          acc[2 * i + 1] += f.y;
+        }
+      }
+    }
+  }
+  for (; r < n_m; r += PHASES) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(r) * ROW_BYTES));
+    const uint32_t* wv = reinterpret_cast<const uint32_t*>(&a);
+    if (FP8) {
+      const float sc = __ldg(k_scale + first + r);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t bf2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[i >> 1] >> ((i & 1) * 16)));
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bf2));
+        acc[2 * i] += f.x * sc;
+        acc[2 * i + 1] += f.y * sc;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[i]));
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPU; ++e) part[ph][u * EPU + e] = acc[e];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += kPoolThreads) {
+    float s = 0.0f;
+#pragma unroll 8
+    for (int p = 0; p < PHASES; ++p) s += part[p][c];
+    const float mean = s / static_cast<float>(n_m);
+    if (kbar) kbar[m * D + c] = mean;
+    if (kbar_hl) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(mean - __bfloat162float(hi));
+      kbar_hl[m * D + c] = __bfloat16_as_ushort(hi);
+      kbar_hl[(M + m) * D + c] = __bfloat16_as_ushort(lo);
+    }
+  }
+}
+
+template <int D, bool FP8>
+cudaError_t launch(const void* K, const float* k_scale, int64_t n_k, int B, float* kbar,
+                   uint16_t* kbar_hl, cudaStream_t s) {
+  const int64_t M = (n_k + B - 1) / B;
+  if (M == 0) return cudaSuccess;
+  pool_keys_kernel<D, FP8><<<static_cast<unsigned>(M), kPoolThreads, 0, s>>>(
+      static_cast<const uint8_t*>(K), k_scale, n_k, B, M, kbar, kbar_hl);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pool_keys(const void* K, const float* k_scale, bool fp8, int64_t n_k, int d,
+                             int B, float* kbar, uint16_t* kbar_hl, cudaStream_t s) {
+  if (fp8) {
+    switch (d) {
+      case 32: return launch<32, true>(K, k_scale, n_k, B, kbar, kbar_hl, s);
+      case 64: return launch<64, true>(K, k_scale, n_k, B, kbar, kbar_hl, s);
+      case 128: return launch<128, true>(K, k_scale, n_k, B, kbar, kbar_hl, s);
+    }
+  } else {
+    switch (d) {
+      case 32: return launch<32, false>(K, k_scale, n_k, B, kbar, kbar_hl, s);
+      case 64: return launch<64, false>(K, k_scale, n_k, B, kbar, kbar_hl, s);
+      case 128: return launch<128, false>(K, k_scale, n_k, B, kbar, kbar_hl, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace misa

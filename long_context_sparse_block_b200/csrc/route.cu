@@ -1,0 +1,377 @@
+// Stages 2-3 — block-pooled router and top-h head selection.
+//
+//   r[t, j] = w[t, j] * sum_{m in C(t)} ReLU(q[t, j] . kbar_m)
+//   heads[t] = the h heads of largest r (ties: lower head index), ascending
+//
+// ("MISA" technical summary, Metodologia step 1: per-head affinities against
+// the mean-pooled block keys are aggregated into one importance per head and
+// the top-h heads are kept; C(t) = the complete blocks whose last key is at or
+// before pos(t).)
+//
+// A dense contraction on the tensor cores: A = 128 consecutive (query, head)
+// rows of Q (128/H queries), B = a 128-block tile of the pooled keys, twice —
+// once for hi = bf16(kbar) and once for lo = bf16(kbar - hi) — accumulated into
+// the same fp32 TMEM tile, so the pooled keys carry ~16 significant bits.  TMEM
+// lane = (query, head), column = block: each epilogue thread sums ReLU over its
+// own row's causal columns, then the 4 epilogue warps exchange r through shared
+// memory and one warp per query runs the top-h as h rounds of a warp argmax.
+//
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
+// issuer, warps 2-5 epilogue.  Row tiles are distributed round-robin over a
+// persistent grid.
+#include "internal.h"
+
+namespace misa {
+namespace {
+
+constexpr int kRows = 128;    // MMA M: (query, head) rows per tile
+constexpr int kBlkN = 128;    // MMA N: pooled blocks per tile
+constexpr int kRouteThreads = 192;
+constexpr int kRouteStages = 2;
+constexpr uint64_t kDrainNs = 2000000;
+
+template <int D>
+struct RouteLayout {
+  static constexpr int ROWB = D >= 64 ? 128 : 64;
+  static constexpr int KCH = D * 2 / ROWB;
+  static constexpr int A_CHUNK = kRows * ROWB;
+  static constexpr int A_BYTES = kRows * D * 2;
+  static constexpr int B_CHUNK = kBlkN * ROWB;
+  static constexpr int B_HALF = kBlkN * D * 2;           // hi or lo tile
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + A_BYTES;
+  static constexpr int OFF_R = OFF_B + kRouteStages * 2 * B_HALF;
+  static constexpr int OFF_BAR = OFF_R + kRows * 4;
+  static constexpr int NBAR = 2 * kRouteStages + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+};
+
+struct RouteParams {
+  const float* w;
+  int32_t* heads;
+  float* r_out;
+  int n_q;
+  int64_t q_pos0;
+  int64_t n_k;
+  int H;
+  int B;
+  int h;
+  int row_tiles;
+  DevCtl ctl;
+};
+
+__device__ __forceinline__ int64_t causal_blocks(const RouteParams& p, int64_t pos) {
+  return min((pos + 1) / p.B, p.n_k / p.B);
+}
+
+// Number of 128-block N tiles a row tile needs (its last query has the most).
+__device__ __forceinline__ int ntiles_of(const RouteParams& p, int rt) {
+  const int QT = kRows / p.H;
+  const int t_last = min((rt + 1) * QT, p.n_q) - 1;
+  const int64_t nc = causal_blocks(p, p.q_pos0 + t_last);
+  return static_cast<int>((nc + kBlkN - 1) / kBlkN);
+}
+
+// warp-uniform argmax by (r desc, head asc)
+__device__ __forceinline__ void better(float& br, int& bj, float r, int j) {
+  if (r > br || (r == br && j < bj)) {
+    br = r;
+    bj = j;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kRouteThreads, 1)
+route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
+                   const __grid_constant__ CUtensorMap kbmap, const RouteParams p) {
+  using L = RouteLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sA = smem_u32(smem + L::OFF_A);
+  const uint32_t sB = smem_u32(smem + L::OFF_B);
+  float* r_s = reinterpret_cast<float*>(smem + L::OFF_R);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int FULL = 0, EMPTY = kRouteStages, AFULL = 2 * kRouteStages, AEMPTY = AFULL + 1,
+            ACCFULL = AFULL + 2, ACCEMPTY = AFULL + 4, ESYNC = AFULL + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRouteStages; ++i) {
+      mbar_init(bar(FULL + i), 1);
+      mbar_init(bar(EMPTY + i), 1);
+    }
+    mbar_init(bar(AFULL), 1);
+    mbar_init(bar(AEMPTY), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(ACCFULL + i), 1);
+      mbar_init(bar(ACCEMPTY + i), 4);
+    }
+    mbar_init(bar(ESYNC), 4);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&kbmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0, tcount = 0;
+    bool ok = true;
+    for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x) {
+      const int nN = ntiles_of(p, rt);
+      if (nN == 0) continue;
+      if (lane == 0) {
+        ok = mbar_wait(bar(AEMPTY), (tcount & 1) ^ 1, abort_flag, p.ctl);
+        if (ok) {
+          mbar_arrive_expect_tx(bar(AFULL), L::A_BYTES);
+          for (int c = 0; c < L::KCH; ++c)
+            tma_load_2d(sA + c * L::A_CHUNK, &qmap, bar(AFULL), c * (L::ROWB / 2), rt * kRows);
+        }
+        for (int nb = 0; nb < nN && ok; ++nb) {
+          ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(FULL + stage), 2 * L::B_HALF);
+          const uint32_t dst = sB + stage * 2 * L::B_HALF;
+          for (int half = 0; half < 2; ++half)
+            for (int c = 0; c < L::KCH; ++c)
+              tma_load_3d(dst + half * L::B_HALF + c * L::B_CHUNK, &kbmap, bar(FULL + stage),
+                          c * (L::ROWB / 2), nb * kBlkN, half);
+          if (++stage == kRouteStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      stage = __shfl_sync(0xffffffffu, stage, 0);
+      phase = __shfl_sync(0xffffffffu, phase, 0);
+      ++tcount;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, accph = 0, tcount = 0;
+    bool ok = true;
+    constexpr uint32_t idesc = umma_idesc_bf16_f32(kRows, kBlkN);
+    for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x) {
+      const int nN = ntiles_of(p, rt);
+      if (nN == 0) continue;
+      if (lane == 0) {
+        ok = mbar_wait(bar(AFULL), tcount & 1, abort_flag, p.ctl);
+        for (int nb = 0; nb < nN && ok; ++nb) {
+          ok = mbar_wait(bar(FULL + stage), phase, abort_flag, p.ctl) &&
+               mbar_wait(bar(ACCEMPTY + acc), accph ^ 1, abort_flag, p.ctl);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBlkN);
+          const uint32_t bstage = sB + stage * 2 * L::B_HALF;
+          for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int c = (kk * 32) / L::ROWB, within = (kk * 32) % L::ROWB;
+              const uint64_t ad = umma_desc_kmajor(sA + c * L::A_CHUNK + within, L::ROWB);
+              const uint64_t bd =
+                  umma_desc_kmajor(bstage + half * L::B_HALF + c * L::B_CHUNK + within, L::ROWB);
+              tc_mma_bf16(d_tmem, ad, bd, idesc, (half > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(bar(EMPTY + stage));
+          tc_commit(bar(ACCFULL + acc));
+          if (++stage == kRouteStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+          if (++acc == 2) {
+            acc = 0;
+            accph ^= 1;
+          }
+        }
+        if (ok) tc_commit(bar(AEMPTY));
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      stage = __shfl_sync(0xffffffffu, stage, 0);
+      phase = __shfl_sync(0xffffffffu, phase, 0);
+      acc = __shfl_sync(0xffffffffu, acc, 0);
+      accph = __shfl_sync(0xffffffffu, accph, 0);
+      ++tcount;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;  // TMEM lane of this thread
+    const int QT = kRows / p.H;
+    int acc = 0;
+    uint32_t accph = 0, esync = 0;
+    bool ok = true;
+    for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x) {
+      const int nN = ntiles_of(p, rt);
+      const int t = rt * QT + row / p.H;
+      const int j = row % p.H;
+      const bool valid = t < p.n_q;
+      const int64_t nc = valid ? causal_blocks(p, p.q_pos0 + t) : 0;
+      float sum = 0.0f;
+      for (int nb = 0; nb < nN; ++nb) {
+        if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(acc * kBlkN);
+        const int64_t m0 = static_cast<int64_t>(nb) * kBlkN;
+#pragma unroll 1
+        for (int c = 0; c < kBlkN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tbase + static_cast<uint32_t>(c * 32), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (m0 + c * 32 + i < nc) sum += relu(__uint_as_float(v[i]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
+        if (++acc == 2) {
+          acc = 0;
+          accph ^= 1;
+        }
+      }
+      if (!ok) break;
+      float r = 0.0f;
+      if (valid) {
+        r = __ldg(p.w + static_cast<int64_t>(t) * p.H + j) * sum;
+        if (p.r_out) p.r_out[static_cast<int64_t>(t) * p.H + j] = r;
+      }
+      r_s[row] = r;
+      // all four epilogue warps have written r_s
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(ESYNC));
+        ok = mbar_wait(bar(ESYNC), esync & 1, abort_flag, p.ctl);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++esync;
+      if (!ok) break;
+      // top-h: one warp per query
+      for (int qq = quad; qq < QT; qq += 4) {
+        const int tq = rt * QT + qq;
+        if (tq >= p.n_q) break;
+        constexpr int SL = 4;  // slots per lane: H <= 128
+        float rv[SL];
+        bool taken[SL];
+#pragma unroll
+        for (int i = 0; i < SL; ++i) {
+          const int jj = lane + 32 * i;
+          taken[i] = jj >= p.H;
+          rv[i] = taken[i] ? 0.0f : r_s[qq * p.H + jj];
+        }
+        for (int round = 0; round < p.h; ++round) {
+          float br = -INFINITY;
+          int bj = 0x7fffffff;
+#pragma unroll
+          for (int i = 0; i < SL; ++i)
+            if (!taken[i]) better(br, bj, rv[i], lane + 32 * i);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            const float orr = __shfl_xor_sync(0xffffffffu, br, off);
+            const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+            better(br, bj, orr, oj);
+          }
+          if (bj < p.H && (bj & 31) == lane) taken[bj >> 5] = true;
+        }
+        // selected heads, written in ascending order
+        int before = 0;
+#pragma unroll
+        for (int i = 0; i < SL; ++i) {
+          const int jj = lane + 32 * i;
+          const bool sel = jj < p.H && taken[i];
+          const uint32_t m = __ballot_sync(0xffffffffu, sel);
+          if (sel)
+            p.heads[static_cast<int64_t>(tq) * p.h + before + __popc(m & ((1u << lane) - 1u))] = jj;
+          before += __popc(m);
+        }
+      }
+      // r_s is reused by the next row tile
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(ESYNC));
+        ok = mbar_wait(bar(ESYNC), esync & 1, abort_flag, p.ctl);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++esync;
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) drain_pause(kDrainNs);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 256);
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const RouteParams& p, const CUtensorMap& qm, const CUtensorMap& km,
+                     cudaStream_t s) {
+  using L = RouteLayout<D>;
+  auto kern = route_heads_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(sm_count(), p.row_tiles);
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, kRouteThreads, L::ALLOC, s>>>(qm, km, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
+                               int n_q, int64_t q_pos0, int64_t n_k, int H, int d, int B, int h,
+                               int32_t* heads, float* r_out, const DevCtl& ctl, cudaStream_t s) {
+  if (n_q <= 0) return cudaSuccess;
+  const int64_t M = (n_k + B - 1) / B;
+  const int64_t rows = static_cast<int64_t>(n_q) * H;
+  const int row_tiles = static_cast<int>((rows + kRows - 1) / kRows);
+  RouteParams p{w, heads, r_out, n_q, q_pos0, n_k, H, B, h, row_tiles, ctl};
+  const int rowb = d >= 64 ? 128 : 64;
+  const CUtensorMapSwizzle swz = rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap qm, km;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(d) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(rowb / 2), static_cast<uint32_t>(kRows)};
+    if (encode_tensor_map(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Q, dims, strides, box, swz) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(M), 2};
+    const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(M * d * 2)};
+    const uint32_t box[3] = {static_cast<uint32_t>(rowb / 2), static_cast<uint32_t>(kBlkN), 1};
+    if (encode_tensor_map(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, kbar_hl, dims, strides, box,
+                          swz) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  switch (d) {
+    case 32: return launch_d<32>(p, qm, km, s);
+    case 64: return launch_d<64>(p, qm, km, s);
+    case 128: return launch_d<128>(p, qm, km, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace misa

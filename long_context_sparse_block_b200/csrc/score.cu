@@ -1,0 +1,402 @@
+// Stage 4 — routed token scoring on the 5th-generation tensor cores.
+//
+//   logit[t, s] = sum_{i<h} w[t, j_i] * ReLU(q[t, j_i] . k_s),  s <= pos(t)
+//
+// ("MISA" technical summary, Metodologia step 2: only the h routed heads score
+// every prefix token; with all heads routed this is the dense DSA lightning
+// indexer of Declaracao do Problema.)
+//
+// Because every head shares the same key vector k_s, the h routed head rows of
+// a group of queries can be stacked into one dense operand: for h = 8, 32
+// queries x 8 heads = 256 rows.  The kernel makes the KEYS the MMA M dimension
+// ("swap-AB"): A = a 128-key tile of K streamed by TMA, B = the 256 gathered
+// (query, head) rows of Q held in shared memory for the whole group, D = 128 x
+// 256 fp32 in TMEM.  TMEM lane = key, column = (query, head), so the epilogue
+// thread that owns a key finds all h heads of a query in its own consecutive
+// columns: ReLU, the head weights and the head-sum are applied in registers and
+// only the fused logit is written to HBM (per-head logits never leave the SM).
+//
+// Warp roles (192 threads, one CTA per SM, persistent):
+//   warp 0     producer: gathers B for each query group (plain 16-byte loads
+//              into the 128-byte-swizzled K-major layout) and streams key tiles
+//              with TMA into a STAGES-deep ring;
+//   warp 1     allocates TMEM (512 columns = two 256-column accumulators) and
+//              issues tcgen05.mma from one thread;
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator, fused ReLU * w head-sum,
+//              causal mask, coalesced fp32 stores (a warp stores 32 consecutive
+//              keys of one query row = 128 bytes).
+// Work is the flattened list of (query group, key tile) pairs, split evenly
+// over the CTAs, so causal triangles stay balanced.
+#include "internal.h"
+
+namespace misa {
+namespace {
+
+constexpr int kTileKeys = 128;   // MMA M
+constexpr int kCols = 256;       // MMA N: (query, head) columns per group
+constexpr int kScoreThreads = 192;
+constexpr uint64_t kDrainNs = 2000000;  // 2 ms
+
+template <int D>
+struct ScoreLayout {
+  static constexpr int ROWB = D >= 64 ? 128 : 64;  // bytes per row of one swizzle chunk
+  static constexpr int KCH = D * 2 / ROWB;         // swizzle chunks along d
+  static constexpr int A_CHUNK = kTileKeys * ROWB;
+  static constexpr int A_BYTES = kTileKeys * D * 2;
+  static constexpr int B_CHUNK = kCols * ROWB;
+  static constexpr int B_BYTES = kCols * D * 2;
+  static constexpr int STAGES = D == 128 ? 4 : 8;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_W = OFF_B + B_BYTES;         // 4 epilogue warps x kCols floats
+  static constexpr int OFF_BAR = OFF_W + 4 * kCols * 4;
+  static constexpr int NBAR = 2 * STAGES + 6;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;            // room to align the base to 1024
+};
+
+struct ScoreParams {
+  const uint16_t* Q;
+  const float* w;
+  const int32_t* heads;  // nullptr: all heads
+  const float* k_scale;  // FP8 keys only
+  float* logits;
+  int64_t ld;
+  int n_q;
+  int64_t q_pos0;
+  int64_t n_k;
+  int H;
+  int64_t total_tiles;
+  DevCtl ctl;
+};
+
+// Flattened schedule over (group g, key tile kt): each role of a CTA walks the
+// same contiguous range, so they agree on every group switch.
+template <int QG>
+struct Sched {
+  int g;
+  int64_t kt, nt, left;
+
+  __device__ static int64_t tiles_of(const ScoreParams& p, int g) {
+    const int t_last = min((g + 1) * QG, p.n_q) - 1;
+    return (p.q_pos0 + t_last) / kTileKeys + 1;
+  }
+  __device__ void init(const ScoreParams& p) {
+    const int64_t start = p.total_tiles * blockIdx.x / gridDim.x;
+    const int64_t end = p.total_tiles * (blockIdx.x + 1) / gridDim.x;
+    left = end - start;
+    g = 0;
+    kt = 0;
+    nt = 0;
+    if (left <= 0) return;
+    int64_t acc = 0;
+    while (true) {
+      const int64_t n = tiles_of(p, g);
+      if (acc + n > start) {
+        kt = start - acc;
+        nt = n;
+        break;
+      }
+      acc += n;
+      ++g;
+    }
+  }
+  __device__ bool last_of_group() const { return kt == nt - 1 || left == 1; }
+  __device__ void next(const ScoreParams& p) {
+    --left;
+    if (++kt == nt && left > 0) {
+      ++g;
+      kt = 0;
+      nt = tiles_of(p, g);
+    }
+  }
+};
+
+template <int D, int HT>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams p) {
+  using L = ScoreLayout<D>;
+  constexpr int QG = kCols / HT;  // queries per group
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sA = smem_u32(smem + L::OFF_A);
+  const uint32_t sB = smem_u32(smem + L::OFF_B);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int FULL = 0, EMPTY = L::STAGES, BFULL = 2 * L::STAGES, BEMPTY = BFULL + 1,
+            ACCFULL = BFULL + 2, ACCEMPTY = BFULL + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::STAGES; ++i) {
+      mbar_init(bar(FULL + i), 1);
+      mbar_init(bar(EMPTY + i), 1);
+    }
+    mbar_init(bar(BFULL), 32);
+    mbar_init(bar(BEMPTY), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(ACCFULL + i), 1);
+      mbar_init(bar(ACCEMPTY + i), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&kmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    Sched<QG> it;
+    it.init(p);
+    int stage = 0;
+    uint32_t phase = 0, gcount = 0;
+    int prev_g = -1;
+    for (; it.left > 0; it.next(p)) {
+      if (it.g != prev_g) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(bar(BEMPTY), (gcount & 1) ^ 1, abort_flag, p.ctl);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        // gather the routed (query, head) rows of group g into B
+        constexpr int UPR = D / 8;  // 16-byte units per row
+        for (int x = lane; x < kCols * UPR; x += 32) {
+          const int n = x / UPR, u = x % UPR;
+          const int qi = n / HT, jj = n % HT;
+          const int t = it.g * QG + qi;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (t < p.n_q) {
+            int j = p.heads ? __ldg(p.heads + static_cast<int64_t>(t) * HT + jj) : jj;
+            if (j < 0 || j >= p.H) {
+              report(p.ctl, DEV_BAD_INPUT);
+              j = 0;
+            }
+            v = __ldg(reinterpret_cast<const uint4*>(
+                p.Q + (static_cast<int64_t>(t) * p.H + j) * D + u * 8));
+          }
+          constexpr int UPC = L::ROWB / 16;  // units per swizzle chunk row
+          const uint32_t off = (u / UPC) * L::B_CHUNK + swz_offset(n, u % UPC, L::ROWB);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sB + off), "r"(v.x),
+                       "r"(v.y), "r"(v.z), "r"(v.w)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(BFULL));
+        prev_g = it.g;
+        ++gcount;
+      }
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
+        if (ok) {
+          mbar_arrive_expect_tx(bar(FULL + stage), L::A_BYTES);
+#pragma unroll
+          for (int c = 0; c < L::KCH; ++c)
+            tma_load_2d(sA + stage * L::A_BYTES + c * L::A_CHUNK, &kmap, bar(FULL + stage),
+                        c * (L::ROWB / 2), static_cast<int>(it.kt * kTileKeys));
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (++stage == L::STAGES) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    Sched<QG> it;
+    it.init(p);
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, accph = 0, gcount = 0;
+    int prev_g = -1;
+    constexpr uint32_t idesc = umma_idesc_bf16_f32(kTileKeys, kCols);
+    for (; it.left > 0; it.next(p)) {
+      const bool new_group = it.g != prev_g;
+      bool ok = true;
+      if (lane == 0) {
+        if (new_group) ok = mbar_wait(bar(BFULL), gcount & 1, abort_flag, p.ctl);
+        ok = ok && mbar_wait(bar(FULL + stage), phase, abort_flag, p.ctl);
+        ok = ok && mbar_wait(bar(ACCEMPTY + acc), accph ^ 1, abort_flag, p.ctl);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kCols);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int c = (kk * 32) / L::ROWB, within = (kk * 32) % L::ROWB;
+            const uint64_t ad =
+                umma_desc_kmajor(sA + stage * L::A_BYTES + c * L::A_CHUNK + within, L::ROWB);
+            const uint64_t bd = umma_desc_kmajor(sB + c * L::B_CHUNK + within, L::ROWB);
+            tc_mma_bf16(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(EMPTY + stage));
+          tc_commit(bar(ACCFULL + acc));
+          if (it.last_of_group()) tc_commit(bar(BEMPTY));
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (new_group) {
+        prev_g = it.g;
+        ++gcount;
+      }
+      if (++stage == L::STAGES) {
+        stage = 0;
+        phase ^= 1;
+      }
+      if (++acc == 2) {
+        acc = 0;
+        accph ^= 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;  // TMEM lanes quad*32 .. quad*32+31
+    float* w_s = reinterpret_cast<float*>(smem + L::OFF_W) + (warp - 2) * kCols;
+    Sched<QG> it;
+    it.init(p);
+    int acc = 0;
+    uint32_t accph = 0;
+    int prev_g = -1;
+    for (; it.left > 0; it.next(p)) {
+      if (it.g != prev_g) {
+        for (int i = lane; i < kCols; i += 32) {
+          const int qi = i / HT, jj = i % HT;
+          const int t = it.g * QG + qi;
+          float wv = 0.0f;
+          if (t < p.n_q) {
+            int j = p.heads ? __ldg(p.heads + static_cast<int64_t>(t) * HT + jj) : jj;
+            if (j < 0 || j >= p.H) j = 0;
+            wv = __ldg(p.w + static_cast<int64_t>(t) * p.H + j);
+          }
+          w_s[i] = wv;
+        }
+        __syncwarp();
+        prev_g = it.g;
+      }
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      tc_fence_after();
+      const int64_t s = it.kt * kTileKeys + quad * 32 + lane;
+      const bool s_ok = s < p.n_k;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * kCols);
+      const int64_t t0 = static_cast<int64_t>(it.g) * QG;
+      float run = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < kCols / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tbase + static_cast<uint32_t>(c * 32), v);
+        tmem_wait_ld();
+        const float4* w4 = reinterpret_cast<const float4*>(w_s + c * 32);
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 wq = w4[i4];
+          const float wl[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = i4 * 4 + e;
+            const int col = c * 32 + i;
+            run = fmaf(wl[e], relu(__uint_as_float(v[i])), run);
+            if ((col % HT) == HT - 1) {
+              const int64_t t = t0 + col / HT;
+              if (t < p.n_q && s_ok) {
+                const float out = (s <= p.q_pos0 + t) ? run : -INFINITY;
+                p.logits[t * p.ld + s] = out;
+              }
+              run = 0.0f;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
+      if (++acc == 2) {
+        acc = 0;
+        accph ^= 1;
+      }
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) drain_pause(kDrainNs);  // let issued copies / MMAs land
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int D, int HT>
+cudaError_t launch_dh(const ScoreParams& p, const CUtensorMap& map, cudaStream_t s) {
+  using L = ScoreLayout<D>;
+  auto kern = score_tokens_kernel<D, HT>;
+  static bool attr_set = false;  // per process; the attribute is per device but idempotent
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int64_t grid = std::min<int64_t>(sm_count(), p.total_tiles);
+  if (grid <= 0) return cudaSuccess;
+  kern<<<static_cast<unsigned>(grid), kScoreThreads, L::ALLOC, s>>>(map, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const ScoreParams& p, int h, const CUtensorMap& map, cudaStream_t s) {
+  switch (h) {
+    case 1: return launch_dh<D, 1>(p, map, s);
+    case 2: return launch_dh<D, 2>(p, map, s);
+    case 4: return launch_dh<D, 4>(p, map, s);
+    case 8: return launch_dh<D, 8>(p, map, s);
+    case 16: return launch_dh<D, 16>(p, map, s);
+    case 32: return launch_dh<D, 32>(p, map, s);
+    case 64: return launch_dh<D, 64>(p, map, s);
+    case 128: return launch_dh<D, 128>(p, map, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads,
+                                const void* K, const float* k_scale, bool fp8, int n_q,
+                                int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
+                                int64_t ld, const DevCtl& ctl, cudaStream_t s) {
+  if (fp8) return cudaErrorNotSupported;
+  if (n_q <= 0) return cudaSuccess;
+  const int QG = kCols / h;
+  const int n_groups = (n_q + QG - 1) / QG;
+  int64_t total = 0;
+  for (int g = 0; g < n_groups; ++g) {
+    const int t_last = std::min((g + 1) * QG, n_q) - 1;
+    total += (q_pos0 + t_last) / kTileKeys + 1;
+  }
+  ScoreParams p{Q, w, heads, k_scale, logits, ld, n_q, q_pos0, n_k, H, total, ctl};
+  CUtensorMap map;
+  const uint64_t dims[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_k)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(d) * 2};
+  const int rowb = d >= 64 ? 128 : 64;
+  const uint32_t box[2] = {static_cast<uint32_t>(rowb / 2), static_cast<uint32_t>(kTileKeys)};
+  if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, dims, strides, box,
+                        rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) !=
+      CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  switch (d) {
+    case 32: return launch_d<32>(p, h, map, s);
+    case 64: return launch_d<64>(p, h, map, s);
+    case 128: return launch_d<128>(p, h, map, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace misa

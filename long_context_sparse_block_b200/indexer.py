@@ -1,0 +1,78 @@
+"""The MISA indexer pipeline over one prefill chunk, through the C ABI.
+
+    pool  -> route (top-h) -> for each query sub-chunk: score -> top-k
+                                                        [-> top-k' -> rerank]
+
+("MISA: Mixture of Indexer Sparse Attention", technical summary: Metodologia
+steps 1-2 and Variante Hierarquica.)  Buffers are allocated once, with torch,
+when the indexer is built; `run` only launches the library's kernels on the
+current stream.  Queries are scored in sub-chunks so that the fp32 logits of a
+whole 8192 x 131072 chunk are never resident at once.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+
+@dataclass
+class IndexerShape:
+    n_q: int
+    q_pos0: int
+    n_k: int
+    H: int
+    d: int
+    B: int
+    h: int          # routed heads (h == H with dense=True: the DSA indexer)
+    k: int
+    kp: int = 0     # MISA-dagger candidate count (0: plain MISA)
+    dense: bool = False
+    sub_chunk: int = 1024
+
+    @property
+    def M(self) -> int:
+        return -(-self.n_k // self.B)
+
+
+class MisaIndexer:
+    def __init__(self, shape: IndexerShape, device="cuda"):
+        s = self.shape = shape
+        dev = torch.device(device)
+        self.sub = min(s.sub_chunk, s.n_q)
+        self.kbar_hl = torch.empty((2, s.M, s.d), dtype=torch.int16, device=dev)
+        self.heads = torch.empty((s.n_q, s.h), dtype=torch.int32, device=dev)
+        self.logits = torch.empty((self.sub, s.n_k), dtype=torch.float32, device=dev)
+        sel = s.kp if s.kp else s.k
+        self.sel = torch.empty((s.n_q, sel), dtype=torch.int32, device=dev)
+        if s.kp:
+            self.final = torch.empty((s.n_q, s.k), dtype=torch.int32, device=dev)
+            nbytes = _lib.misa_workspace_size("rerank", self.sub, s.n_k, s.k, s.kp)
+            self.ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        else:
+            self.final = self.sel
+
+    def run(self, Q, K, w, k_scale=None, on_subchunk=None):
+        """Q [n_q,H,d] bf16 codes, K [n_k,d] bf16 codes (or e4m3 + k_scale), w [n_q,H] f32.
+        Returns the selected token indices [n_q, k] (int32, ascending, -1 padded).
+        on_subchunk(c0, c1, logits) is called after each sub-chunk is scored (for
+        inspection; the logits buffer is reused by the next sub-chunk)."""
+        s = self.shape
+        if not s.dense:
+            _lib.misa_pool_keys(K, s.B, k_scale=k_scale, kbar_hl=self.kbar_hl, want_kbar=False)
+            _lib.misa_route_heads(Q, w, self.kbar_hl, s.q_pos0, s.n_k, s.B, s.h, heads=self.heads)
+        for c0 in range(0, s.n_q, self.sub):
+            c1 = min(s.n_q, c0 + self.sub)
+            n = c1 - c0
+            lg = self.logits[:n]
+            _lib.misa_score_tokens(Q[c0:c1], w[c0:c1], None if s.dense else self.heads[c0:c1], K,
+                                   s.q_pos0 + c0, k_scale=k_scale, logits=lg, h=s.h)
+            if on_subchunk is not None:
+                on_subchunk(c0, c1, lg)
+            _lib.misa_topk(lg, s.q_pos0 + c0, s.n_k, self.sel.shape[1], idx=self.sel[c0:c1])
+            if s.kp:
+                _lib.misa_rerank(Q[c0:c1], w[c0:c1], K, self.sel[c0:c1], s.q_pos0 + c0, s.k,
+                                 k_scale=k_scale, idx=self.final[c0:c1], ws=self.ws)
+        return self.final

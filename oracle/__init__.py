@@ -6,7 +6,8 @@ fp64, single-threaded, written from the method's definitions) with ctypes and
 shares no code with the CUDA library.
 
 Parity status per function (what pins each one is listed in the tests):
-  pool_keys, route, score, dense_logits, topk, topk_f32, rerank — pinned by
+  pool_keys, route, score, dense_logits, topk, topk_f32, rerank,
+  select_candidates — pinned by
   closed forms, brute force on tiny inputs, library-routine reductions and the
   structural invariants of the method.  The router's aggregate (a sum over
   complete causal blocks of w * ReLU(q . kbar)) is a reading of a step the pages
@@ -72,6 +73,8 @@ def _load():
                 "oracle_topk_f32": (None, [_F, _i64, _int, _i64, _i64, _int, _I32]),
                 "oracle_rerank": (None, [_D, _D, _D, _I32, _int, _int, _i64, _i64, _int, _int,
                                          _int, _I32, _D, _I64]),
+                "oracle_select_candidates_f32": (None, [_F, _I32, _int, _int, _i64, _i64, _int,
+                                                        _I32]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -204,6 +207,17 @@ def rerank(Q, w, K, cand, q_pos0: int, k: int, counter=None, want_logits: bool =
                           H, d, k, _p(idx, _I32), _p(full, _D) if full is not None else None,
                           counter.ptr() if counter else None)
     return (idx, full) if want_logits else idx
+
+
+def select_candidates(vals, cand, q_pos0: int, n_k: int, k: int) -> np.ndarray:
+    """Top-k tokens among candidate scores [n_q, kp] (fp32) of tokens cand [n_q, kp]."""
+    vals = _c(vals, np.float32)
+    cand = _c(cand, np.int32)
+    n_q, kp = cand.shape
+    idx = np.empty((n_q, k), dtype=np.int32)
+    _load().oracle_select_candidates_f32(_p(vals, _F), _p(cand, _I32), kp, n_q, q_pos0, n_k, k,
+                                         _p(idx, _I32))
+    return idx
 
 
 # ---- whole-path helpers over stored inputs -----------------------------------

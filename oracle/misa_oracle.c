@@ -292,3 +292,26 @@ void oracle_rerank(const double* Q, const double* w, const double* K, const int3
     }
     free(items);
 }
+
+/* Top-k among candidate scores given in fp32 (scores produced elsewhere):
+ * row t holds vals[t*kp + i] for token cand[t*kp + i].  Entries whose token is
+ * outside 0..pos(t) or whose value is -inf are ignored; selection by (value
+ * desc, token asc); tokens written ascending, -1 padded. */
+void oracle_select_candidates_f32(const float* vals, const int32_t* cand, int kp, int n_q,
+                                  int64_t q_pos0, int64_t n_k, int k, int32_t* idx) {
+    scored* items = (scored*)malloc(sizeof(scored) * (size_t)(kp > 0 ? kp : 1));
+    for (int t = 0; t < n_q; ++t) {
+        int64_t pos = q_pos0 + t;
+        int64_t n = 0;
+        for (int i = 0; i < kp; ++i) {
+            int64_t c = cand[(int64_t)t * kp + i];
+            double v = (double)vals[(int64_t)t * kp + i];
+            if (c < 0 || c > pos || c >= n_k || v == -INFINITY) continue;
+            items[n].v = v;
+            items[n].s = c;
+            ++n;
+        }
+        select_k(items, n, k, idx + (int64_t)t * k);
+    }
+    free(items);
+}

@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point its header declares, and rejects bad arguments before any
+launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "misa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_sparse_block_b200 import build
+    build.build()
+    from long_context_sparse_block_b200 import _lib
+    return _lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(misa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_stage_calls():
+    names = declared_functions()
+    for n in ("misa_pool_keys", "misa_route_heads", "misa_score_tokens", "misa_topk",
+              "misa_rerank", "misa_workspace_size", "misa_status_string",
+              "misa_last_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(so, name), name
+
+
+def test_status_strings(lib):
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.misa_status_string(st) != "unknown status"
+    assert lib.misa_status_string(12345) == "unknown status"
+
+
+def test_workspace_size(lib):
+    assert lib.misa_workspace_size("rerank", 8192, 131072, 2048, 8192) == 8192 * 8192 * 4
+    assert lib.misa_workspace_size("topk", 8192, 131072, 2048, 0) == 0
+    assert lib.misa_workspace_size("rerank", 0, 10, 1, 1) == 0
+
+
+def _so(lib):
+    return lib._lib
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    so = _so(lib)
+    p = ctypes.c_void_p(16 * 1024)          # aligned, never dereferenced
+    odd = ctypes.c_void_p(16 * 1024 + 2)    # not 16-byte aligned
+    INV, UNS = lib.MISA_ERR_INVALID_ARG, lib.MISA_ERR_UNSUPPORTED
+    # pool: null K, bad d, B out of range, fp8 without scales, no outputs
+    assert so.misa_pool_keys(None, None, 0, 128, 128, 64, p, p, None) == INV
+    assert so.misa_pool_keys(p, None, 0, 128, 96, 64, p, p, None) == INV
+    assert so.misa_pool_keys(p, None, 0, 128, 128, 0, p, p, None) == INV
+    assert so.misa_pool_keys(p, None, 1, 128, 128, 64, p, p, None) == INV
+    assert so.misa_pool_keys(p, None, 0, 128, 128, 64, None, None, None) == INV
+    assert so.misa_pool_keys(odd, None, 0, 128, 128, 64, p, p, None) == INV
+    # route: queries past the keys, h > H, H not a power of two
+    assert so.misa_route_heads(p, p, p, 10, 95, 100, 64, 128, 64, 8, p, None, None) == INV
+    assert so.misa_route_heads(p, p, p, 10, 0, 100, 8, 128, 64, 9, p, None, None) == INV
+    assert so.misa_route_heads(p, p, p, 10, 0, 100, 48, 128, 64, 8, p, None, None) == UNS
+    assert so.misa_route_heads(p, p, p, 10, 0, 100, 64, 80, 64, 8, p, None, None) == UNS
+    # score: ld < n_k, dense with h != H, h not a power of two
+    assert so.misa_score_tokens(p, p, p, p, None, 0, 10, 0, 100, 64, 128, 8, p, 99, None) == INV
+    assert so.misa_score_tokens(p, p, None, p, None, 0, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    assert so.misa_score_tokens(p, p, p, p, None, 0, 10, 0, 100, 64, 128, 6, p, 100, None) == UNS
+    assert so.misa_score_tokens(odd, p, p, p, None, 0, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    # top-k: k too large, ld too small
+    assert so.misa_topk(p, 100, 10, 0, 100, 20000, p, None, 0, None) == INV
+    assert so.misa_topk(p, 5, 10, 0, 100, 4, p, None, 0, None) == INV
+    # rerank: k > kp, missing workspace
+    assert so.misa_rerank(p, p, p, None, 0, p, 16, 4, 0, 100, 64, 128, 32, p, None, p, 1 << 20,
+                          None) == INV
+    assert so.misa_rerank(p, p, p, None, 0, p, 16, 4, 0, 100, 64, 128, 8, p, None, None, 0,
+                          None) == lib.MISA_ERR_WORKSPACE
+
+
+def test_empty_work_is_a_no_op(lib):
+    so = _so(lib)
+    p = ctypes.c_void_p(16 * 1024)
+    assert so.misa_topk(p, 100, 0, 0, 100, 4, p, None, 0, None) == 0
+    assert so.misa_topk(p, 100, 10, 0, 100, 0, None, None, 0, None) == 0
+    assert so.misa_score_tokens(p, p, p, p, None, 0, 0, 0, 100, 64, 128, 8, p, 100, None) == 0

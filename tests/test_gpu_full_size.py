@@ -1,0 +1,92 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark times (1024-query sub-chunks), on sampled query rows that the oracle
+computes one by one: the first and last query, the query whose head-0 row was
+planted as needle keys, and seeded random rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_sparse_block_b200 import workloads as W
+from tests.gpu_helpers import assert_logits_close, check_heads, inputs_to_device, recall
+
+pytestmark = pytest.mark.gpu
+
+N_RANDOM = 12
+
+
+def _rows(wl):
+    rng = np.random.default_rng(77)
+    rows = {0, wl.n_q - 1, wl.n_q // 2} | set(rng.choice(wl.n_q, N_RANDOM, replace=False).tolist())
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name", ["chunk_128k", "chunk_128k_h4", "dsv32_32k", "glm5_64k"])
+def test_full_size_sampled_rows(name):
+    from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl)
+    rows = _rows(wl)
+    g = inputs_to_device(inp)
+    ix = MisaIndexer(IndexerShape(wl.n_q, wl.q_pos0, wl.n_k, wl.H, wl.d, wl.B, wl.h, wl.k,
+                                  sub_chunk=1024))
+    dumps = {}
+
+    def grab(c0, c1, lg):
+        for t in rows:
+            if c0 <= t < c1:
+                dumps[t] = lg[t - c0].cpu().numpy()
+
+    idx = ix.run(g["Q"], g["K"], g["w"], on_subchunk=grab).cpu().numpy()
+    heads = ix.heads.cpu().numpy()
+    from long_context_sparse_block_b200 import _lib
+    assert _lib.misa_last_device_status() == 0
+    Kd = oracle.bf16_to_f64(inp["K"])
+    kbar = oracle.pool_keys(Kd, wl.B)
+    sel = np.array(rows)
+    Qd = oracle.bf16_to_f64(inp["Q"][sel])
+    wd = inp["w"][sel].astype(np.float64)
+    matched = 0
+    for i, t in enumerate(rows):
+        pos = wl.q_pos0 + t
+        r_o, h_o = oracle.route(Qd[i:i + 1], wd[i:i + 1], kbar, pos, wl.n_k, wl.B, wl.h)
+        check_heads(heads[t:t + 1], r_o, h_o, wl.h)
+        lg_gpu = dumps[t]
+        # top-k is bit-exact on the GPU's own logits
+        assert np.array_equal(idx[t], oracle.topk(lg_gpu[None, :], pos, wl.n_k, wl.k)[0])
+        if not np.array_equal(heads[t], h_o[0]):
+            continue
+        matched += 1
+        ref = oracle.score(Qd[i:i + 1], wd[i:i + 1], h_o, Kd, pos)[0]
+        hs = h_o[0]
+        mag = (np.abs(wd[i, hs])[:, None] * np.maximum(Qd[i, hs] @ Kd[:pos + 1].T, 0)).sum(0)
+        assert_logits_close(lg_gpu, ref[:pos + 1], mag, what=f"{name} row {t}")
+        assert recall(idx[t:t + 1], oracle.topk(ref[None, :], pos, wl.n_k, wl.k)) >= 0.999
+    assert matched >= len(rows) - 2
+
+
+def test_full_size_dagger_sampled_rows():
+    from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
+    wl = W.WORKLOADS["dagger_128k"]
+    inp = W.generate(wl)
+    rows = _rows(wl)
+    g = inputs_to_device(inp)
+    ix = MisaIndexer(IndexerShape(wl.n_q, wl.q_pos0, wl.n_k, wl.H, wl.d, wl.B, wl.h, wl.k,
+                                  kp=wl.kp, sub_chunk=1024))
+    fin = ix.run(g["Q"], g["K"], g["w"]).cpu().numpy()
+    cand = ix.sel.cpu().numpy()
+    heads = ix.heads.cpu().numpy()
+    Kd = oracle.bf16_to_f64(inp["K"])
+    kbar = oracle.pool_keys(Kd, wl.B)
+    sel = np.array(rows)
+    Qd = oracle.bf16_to_f64(inp["Q"][sel])
+    wd = inp["w"][sel].astype(np.float64)
+    for i, t in enumerate(rows):
+        pos = wl.q_pos0 + t
+        _, h_o = oracle.route(Qd[i:i + 1], wd[i:i + 1], kbar, pos, wl.n_k, wl.B, wl.h)
+        if not np.array_equal(heads[t], h_o[0]):
+            continue
+        # the fine stage on the GPU's own candidates, in fp64
+        ref = oracle.rerank(Qd[i:i + 1], wd[i:i + 1], Kd, cand[t:t + 1], pos, wl.k)
+        assert recall(fin[t:t + 1], ref) >= 0.999
+        assert np.all(np.diff(fin[t][fin[t] >= 0]) > 0)

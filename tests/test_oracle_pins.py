@@ -385,3 +385,32 @@ def test_workload_pair_counts():
     assert W["glm5_64k"].causal_pairs() == 2_147_516_416
     assert W["chunk_128k"].causal_pairs() == 1_040_191_488
     assert W["chunk_128k"].M == 1024
+
+
+# ---------------------------------------------------------------- candidate selection
+
+@pytest.mark.parametrize("seed", range(4))
+def test_select_candidates_matches_brute_force(seed):
+    rng = np.random.default_rng(300 + seed)
+    pos, n_k, k = 11, 14, 3
+    cand = np.array([[0, 2, 3, 5, 6, 9, 11, -1, 13]], dtype=np.int32)   # 13 > pos: ignored
+    vals = rng.integers(-2, 3, size=(1, 9)).astype(np.float32)
+    vals[0, 4] = -np.inf                                                 # absent
+    idx = oracle.select_candidates(vals, cand, pos, n_k, k)[0]
+    valid = [i for i in range(9) if 0 <= cand[0, i] <= pos and vals[0, i] != -np.inf]
+    best = _brute_force_best_subset([float(vals[0, i]) for i in valid], k)
+    assert list(idx) == sorted(int(cand[0, valid[b]]) for b in best)
+
+
+def test_select_candidates_agrees_with_rerank_on_exact_scores():
+    rng = np.random.default_rng(9)
+    n_q, H, d, n_k, pos0 = 4, 3, 4, 20, 12
+    Q = rng.integers(-2, 3, size=(n_q, H, d)).astype(np.float64)
+    K = rng.integers(-2, 3, size=(n_k, d)).astype(np.float64)
+    w = rng.integers(-2, 3, size=(n_q, H)).astype(np.float64) / 2.0
+    cand = np.sort(rng.choice(13, size=(n_q, 8), replace=True), axis=1).astype(np.int32)
+    for t in range(n_q):                                    # distinct, ascending
+        cand[t] = np.sort(rng.choice(pos0 + t + 1, size=8, replace=False))
+    idx, full = oracle.rerank(Q, w, K, cand, pos0, 5, want_logits=True)
+    sel = oracle.select_candidates(full.astype(np.float32), cand, pos0, n_k, 5)
+    assert np.array_equal(sel, idx)      # integer-valued scores: exact in fp32
