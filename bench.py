@@ -290,9 +290,11 @@ def run_ours(args, rank, world, local_rank, inp):
     tflops = score_flops / (score_ms * 1e-3) / 1e12
     topk_gbs = 4.0 * pairs / (stage_ms["topk"] * 1e-3) / 1e9
     pool_gbs = (wl.n_k * wl.d * 2 + 2 * wl.M * wl.d * 2) / (stage_ms["pool"] * 1e-3) / 1e9
-    rt = wl.n_q * wl.H * 2 * wl.d * sum(min((p + 1) // wl.B, wl.n_k // wl.B)
-                                        for p in wl.positions().tolist())
-    route_tflops = 2 * rt / (stage_ms["route"] * 1e-3) / 1e12  # hi and lo contractions
+    # router: H_I * d multiply-adds per (query, complete causal block), done twice
+    # (hi and lo halves of the pooled keys)
+    blocks = sum(min((p + 1) // wl.B, wl.n_k // wl.B) for p in wl.positions().tolist())
+    route_flops = 2.0 * 2.0 * wl.H * wl.d * blocks
+    route_tflops = route_flops / (stage_ms["route"] * 1e-3) / 1e12
     h2d = inp["Q"].nbytes + inp["K"].nbytes + inp["w"].nbytes
     d2h = idx_h.numel() * 4
     out = {

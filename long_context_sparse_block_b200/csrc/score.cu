@@ -16,15 +16,17 @@
 // columns: ReLU, the head weights and the head-sum are applied in registers and
 // only the fused logit is written to HBM (per-head logits never leave the SM).
 //
-// Warp roles (192 threads, one CTA per SM, persistent):
-//   warp 0     producer: gathers B for each query group (plain 16-byte loads
-//              into the 128-byte-swizzled K-major layout) and streams key tiles
-//              with TMA into a STAGES-deep ring;
+// Warp roles (320 threads, one CTA per SM, persistent):
+//   warp 0     producer: gathers B for each query group (16-byte cp.async into
+//              the 128-byte-swizzled K-major layout) and streams key tiles with
+//              TMA into a STAGES-deep ring;
 //   warp 1     allocates TMEM (512 columns = two 256-column accumulators) and
 //              issues tcgen05.mma from one thread;
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, fused ReLU * w head-sum,
-//              causal mask, coalesced fp32 stores (a warp stores 32 consecutive
-//              keys of one query row = 128 bytes).
+//   warps 2-9  epilogue, two warps per TMEM lane quadrant, each owning 128 of
+//              the 256 columns: one tcgen05.ld of its 128 columns, the
+//              accumulator released right after the load lands, then the fused
+//              ReLU * w head-sum (packed fp32 FMA), causal mask and coalesced
+//              fp32 stores (a warp stores 32 consecutive keys of one query row).
 // Work is the flattened list of (query group, key tile) pairs, split evenly
 // over the CTAs, so causal triangles stay balanced.
 #include "internal.h"
@@ -34,7 +36,9 @@ namespace {
 
 constexpr int kTileKeys = 128;   // MMA M
 constexpr int kCols = 256;       // MMA N: (query, head) columns per group
-constexpr int kScoreThreads = 192;
+constexpr int kScoreThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr int kHalfCols = kCols / 2;  // columns per epilogue warp
 constexpr uint64_t kDrainNs = 2000000;  // 2 ms
 
 template <int D>
@@ -48,8 +52,9 @@ struct ScoreLayout {
   static constexpr int STAGES = D == 128 ? 4 : 8;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_W = OFF_B + B_BYTES;         // 4 epilogue warps x kCols floats
-  static constexpr int OFF_BAR = OFF_W + 4 * kCols * 4;
+  static constexpr int OFF_W = OFF_B + B_BYTES;         // 8 epilogue warps x 128 floats
+  static constexpr int OFF_HEADS = OFF_W + kEpiWarps * kHalfCols * 4;  // producer: heads of a group
+  static constexpr int OFF_BAR = OFF_HEADS + kCols * 4;
   static constexpr int NBAR = 2 * STAGES + 6;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
@@ -140,7 +145,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     mbar_init(bar(BEMPTY), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(ACCFULL + i), 1);
-      mbar_init(bar(ACCEMPTY + i), 4);
+      mbar_init(bar(ACCEMPTY + i), kEpiWarps);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -167,28 +172,33 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
         bool ok = true;
         if (lane == 0) ok = mbar_wait(bar(BEMPTY), (gcount & 1) ^ 1, abort_flag, p.ctl);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        // gather the routed (query, head) rows of group g into B
-        constexpr int UPR = D / 8;  // 16-byte units per row
-        for (int x = lane; x < kCols * UPR; x += 32) {
-          const int n = x / UPR, u = x % UPR;
-          const int qi = n / HT, jj = n % HT;
-          const int t = it.g * QG + qi;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        // gather the routed (query, head) rows of group g into B: the group's
+        // head ids first (independent loads), then one cp.async per 16 bytes
+        int32_t* hs = reinterpret_cast<int32_t*>(smem + L::OFF_HEADS);
+        for (int n = lane; n < kCols; n += 32) {
+          const int t = it.g * QG + n / HT;
+          int j = -1;
           if (t < p.n_q) {
-            int j = p.heads ? __ldg(p.heads + static_cast<int64_t>(t) * HT + jj) : jj;
+            j = p.heads ? __ldg(p.heads + static_cast<int64_t>(t) * HT + n % HT) : n % HT;
             if (j < 0 || j >= p.H) {
               report(p.ctl, DEV_BAD_INPUT);
               j = 0;
             }
-            v = __ldg(reinterpret_cast<const uint4*>(
-                p.Q + (static_cast<int64_t>(t) * p.H + j) * D + u * 8));
           }
-          constexpr int UPC = L::ROWB / 16;  // units per swizzle chunk row
-          const uint32_t off = (u / UPC) * L::B_CHUNK + swz_offset(n, u % UPC, L::ROWB);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sB + off), "r"(v.x),
-                       "r"(v.y), "r"(v.z), "r"(v.w)
-                       : "memory");
+          hs[n] = j;
         }
+        __syncwarp();
+        constexpr int UPR = D / 8;             // 16-byte units per row
+        constexpr int UPC = L::ROWB / 16;      // units per swizzle chunk row
+        for (int x = lane; x < kCols * UPR; x += 32) {
+          const int n = x / UPR, u = x % UPR;
+          const int j = hs[n];
+          const int t = it.g * QG + n / HT;
+          const uint16_t* src = j >= 0 ? p.Q + (static_cast<int64_t>(t) * p.H + j) * D + u * 8 : p.Q;
+          const uint32_t off = (u / UPC) * L::B_CHUNK + swz_offset(n, u % UPC, L::ROWB);
+          cp_async16(sB + off, src, j >= 0 ? 16u : 0u);
+        }
+        cp_async_wait_all();
         fence_proxy_async_smem();
         mbar_arrive(bar(BFULL));
         prev_g = it.g;
@@ -258,8 +268,11 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;  // TMEM lanes quad*32 .. quad*32+31
-    float* w_s = reinterpret_cast<float*>(smem + L::OFF_W) + (warp - 2) * kCols;
+    const int e = warp - 2;
+    const int quad = warp & 3;   // TMEM lanes quad*32 .. quad*32+31
+    const int half = e >> 2;     // columns half*128 .. half*128+127
+    constexpr int QPW = kHalfCols / HT;  // queries per warp
+    float* w_s = reinterpret_cast<float*>(smem + L::OFF_W) + e * kHalfCols;
     Sched<QG> it;
     it.init(p);
     int acc = 0;
@@ -267,12 +280,12 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     int prev_g = -1;
     for (; it.left > 0; it.next(p)) {
       if (it.g != prev_g) {
-        for (int i = lane; i < kCols; i += 32) {
-          const int qi = i / HT, jj = i % HT;
-          const int t = it.g * QG + qi;
+        for (int i = lane; i < kHalfCols; i += 32) {
+          const int col = half * kHalfCols + i;
+          const int t = it.g * QG + col / HT;
           float wv = 0.0f;
           if (t < p.n_q) {
-            int j = p.heads ? __ldg(p.heads + static_cast<int64_t>(t) * HT + jj) : jj;
+            int j = p.heads ? __ldg(p.heads + static_cast<int64_t>(t) * HT + col % HT) : col % HT;
             if (j < 0 || j >= p.H) j = 0;
             wv = __ldg(p.w + static_cast<int64_t>(t) * p.H + j);
           }
@@ -285,44 +298,61 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
       if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
-      const int64_t s = it.kt * kTileKeys + quad * 32 + lane;
-      const bool s_ok = s < p.n_k;
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * kCols);
-      const int64_t t0 = static_cast<int64_t>(it.g) * QG;
-      float run = 0.0f;
-#pragma unroll 1
-      for (int c = 0; c < kCols / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tbase + static_cast<uint32_t>(c * 32), v);
-        tmem_wait_ld();
-        const float4* w4 = reinterpret_cast<const float4*>(w_s + c * 32);
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 wq = w4[i4];
-          const float wl[4] = {wq.x, wq.y, wq.z, wq.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = i4 * 4 + e;
-            const int col = c * 32 + i;
-            run = fmaf(wl[e], relu(__uint_as_float(v[i])), run);
-            if ((col % HT) == HT - 1) {
-              const int64_t t = t0 + col / HT;
-              if (t < p.n_q && s_ok) {
-                const float out = (s <= p.q_pos0 + t) ? run : -INFINITY;
-                p.logits[t * p.ld + s] = out;
-              }
-              run = 0.0f;
-            }
-          }
-        }
-      }
+      uint32_t v[kHalfCols];
+      tmem_ld128(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                     static_cast<uint32_t>(acc * kCols + half * kHalfCols),
+                 v);
+      tmem_wait_ld();
+      // the accumulator is in registers: hand it back to the MMA warp now
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
       if (++acc == 2) {
         acc = 0;
         accph ^= 1;
+      }
+      const int64_t s = it.kt * kTileKeys + quad * 32 + lane;
+      const bool s_ok = s < p.n_k;
+      const int64_t tq0 = static_cast<int64_t>(it.g) * QG + half * QPW;
+      float* dst = p.logits + tq0 * p.ld + s;
+      if constexpr (HT >= 4) {
+        // every head-sum first (the shared-memory weight loads never wait
+        // behind a global store), then the stores
+        float sums[QPW];
+#pragma unroll
+        for (int qq = 0; qq < QPW; ++qq) {
+          float2 a2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int j = 0; j < HT; j += 4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(w_s + qq * HT + j);
+            const uint32_t* x = v + qq * HT + j;
+            a2 = fma2(make_float2(w4.x, w4.y),
+                      make_float2(relu(__uint_as_float(x[0])), relu(__uint_as_float(x[1]))), a2);
+            a2 = fma2(make_float2(w4.z, w4.w),
+                      make_float2(relu(__uint_as_float(x[2])), relu(__uint_as_float(x[3]))), a2);
+          }
+          sums[qq] = a2.x + a2.y;
+        }
+#pragma unroll
+        for (int qq = 0; qq < QPW; ++qq) {
+          const int64_t t = tq0 + qq;
+          if (t < p.n_q && s_ok) *dst = (s <= p.q_pos0 + t) ? sums[qq] : -INFINITY;
+          dst += p.ld;
+        }
+      } else {
+#pragma unroll
+        for (int qq = 0; qq < QPW; ++qq) {
+          float sum;
+          if constexpr (HT == 1) {
+            sum = w_s[qq] * relu(__uint_as_float(v[qq]));
+          } else {
+            const float2 w2 = *reinterpret_cast<const float2*>(w_s + qq * 2);
+            sum = fmaf(w2.y, relu(__uint_as_float(v[qq * 2 + 1])), w2.x * relu(__uint_as_float(v[qq * 2])));
+          }
+          const int64_t t = tq0 + qq;
+          if (t < p.n_q && s_ok) *dst = (s <= p.q_pos0 + t) ? sum : -INFINITY;
+          dst += p.ld;
+        }
       }
     }
   }

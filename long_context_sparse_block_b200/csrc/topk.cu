@@ -9,19 +9,26 @@
 //                   (MISA-dagger: final top-k among the re-scored candidates).
 //
 // Values are mapped to order-preserving 32-bit keys (-0.0 folded onto +0.0,
-// -inf and padding to the reserved key 0).  One CTA per row:
-//   pass 1   stream the row once from HBM, 4096-bin histogram of key >> 20;
-//            the bin holding the k-th largest key follows from a block scan;
-//   pass 2   (fast path) stream the row again — normally from L2 — and append,
-//            in position order, every entry whose key is in or above that bin
-//            to a shared-memory list (block scans give each thread its slots);
-//   refine   two 10-bit histogram rounds over the list pin the exact k-th key
-//            T and how many entries equal to T are still needed;
-//   select   one ordered pass over the list keeps key > T, and keys == T while
-//            their rank among equals is below the need: output is ascending by
-//            construction and ties resolve to the lower position.
-// If the candidate list would not fit in shared memory (massive ties), the
-// refine rounds and the ordered selection run over the row in global memory.
+// -inf and padding to the reserved key 0).  One CTA per row.
+//
+// Fast path (k <= 4096):
+//   sample   1/32 of the row (strided float4 loads); the exact m-th largest
+//            sampled key, m ~ 1.5 k * (sample / row), becomes a threshold tau;
+//   stream   ONE pass over the row from HBM with no atomics: every key >= tau
+//            is appended, warp-compacted with ballots, to the warp's own region
+//            of a shared-memory list (warps own interleaved 128-entry chunks);
+//   check    if the list holds at least k entries it holds the whole top-k
+//            (every key above the k-th largest is >= tau), including every
+//            entry equal to the k-th largest key;
+//   select   three radix rounds (12 + 10 + 10 bits) over the list give the
+//            exact k-th key T and how many entries equal to T are kept (the
+//            lowest positions); the kept positions are sorted ascending
+//            (bitonic) and written out.
+// Fallback (sample too optimistic, list overflow, k > 4096): a 4096-bin
+// histogram pass, an ordered collection of the entries in or above the k-th
+// bin (block scans keep position order), the same radix refinement, and an
+// ordered selection pass — over the shared-memory list when it fits, else over
+// the row in global memory.
 #include "internal.h"
 
 namespace misa {
@@ -31,6 +38,10 @@ constexpr int kTopkThreads = 512;
 constexpr int kWarps = kTopkThreads / 32;
 constexpr int kBins1 = 4096;
 constexpr int kChunk = 4 * kTopkThreads;  // entries per block-wide step
+constexpr int kFastMaxK = 4096;           // largest k of the fast path
+constexpr int kSampleTarget = 4096;       // sampled entries per row (at most)
+constexpr int kFastCap = 5120;            // list entries of the fast path (all warps)
+constexpr int kRegion = kFastCap / kWarps;  // list entries per warp region
 
 struct TopkParams {
   const float* vals;
@@ -240,6 +251,213 @@ __device__ void refine(const Src& src, uint32_t b1, uint32_t above1, uint32_t k,
   need_eq = need;
 }
 
+// Entries of the per-warp regions of the fast-path list (flattened; slots past
+// a region's count read as absent).
+struct RegionSrc {
+  const uint32_t* keys;
+  const uint32_t* poss;
+  const uint32_t* counts;  // [kWarps]
+  int64_t n;               // kWarps * kRegion
+  __device__ __forceinline__ void load4(int64_t i0, uint32_t (&key)[4], uint32_t (&pos)[4]) const {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int64_t x = i0 + e;
+      const int w = static_cast<int>(x / kRegion), j = static_cast<int>(x % kRegion);
+      const bool in = x < n && j < static_cast<int>(counts[w]);
+      key[e] = in ? keys[x] : 0u;
+      pos[e] = in ? poss[x] : 0u;
+    }
+  }
+};
+
+// Exact m-th largest key among the present entries of `src` (1 <= m <= present).
+// Returns T; `need` = how many entries equal to T belong to the m largest.
+template <class Src>
+__device__ uint32_t kth_largest(const Src& src, uint32_t m, uint32_t* hist, SmemCtl& sc,
+                                uint32_t& need) {
+  for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) hist[i] = 0u;
+  __syncthreads();
+  for (int64_t base = 0; base < src.n; base += kChunk) {
+    uint32_t key[4], pos[4];
+    src.load4(base + threadIdx.x * 4, key, pos);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (key[e] != 0u) atomicAdd(&hist[key[e] >> 20], 1u);
+  }
+  __syncthreads();
+  find_bin<kBins1>(hist, m, sc);
+  const uint32_t b1 = sc.res[0], above1 = sc.res[1];
+  __syncthreads();
+  uint32_t T;
+  refine(src, b1, above1, m, hist, sc, T, need);
+  return T;
+}
+
+// Ascending bitonic sort of buf[0..n) in shared memory (n <= cap, cap a power of two).
+__device__ void bitonic_sort_asc(uint32_t* buf, uint32_t n, uint32_t cap) {
+  uint32_t P = 1;
+  while (P < n) P <<= 1;
+  for (uint32_t i = n + threadIdx.x; i < P; i += kTopkThreads) buf[i] = 0xFFFFFFFFu;
+  __syncthreads();
+  for (uint32_t size = 2; size <= P; size <<= 1) {
+    for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
+      for (uint32_t i = threadIdx.x; i < P / 2; i += kTopkThreads) {
+        const uint32_t lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
+        const bool asc = (lo & size) == 0;
+        const uint32_t a = buf[lo], b = buf[hi];
+        if ((a > b) == asc) {
+          buf[lo] = b;
+          buf[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  (void)cap;
+}
+
+// Fast path.  Returns false (and writes nothing) when the row must take the
+// fallback path.  Shared memory: hist [kBins1], list keys/poss [kFastCap],
+// sel [kFastMaxK], counts [kWarps].
+__device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit& out,
+                          uint32_t* hist, uint32_t* lkeys, uint32_t* lposs, uint32_t* sel,
+                          uint32_t* counts, SmemCtl& sc) {
+  const uint32_t k = out.k;
+  const int64_t n = src.n;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // ---- threshold from a sample
+  uint32_t tau = 1u;  // collect every present entry
+  if (n > kFastCap) {
+    const int64_t n4 = n / 4;                         // whole float4 groups
+    const int64_t per = n4 / (kSampleTarget / 4);
+    const int64_t step = per > 1 ? per : 1;
+    const int64_t groups = n4 / step < kSampleTarget / 4 ? n4 / step : kSampleTarget / 4;
+    for (int64_t g = threadIdx.x; g < groups; g += kTopkThreads) {
+      uint32_t key[4], pos[4];
+      src.load4(g * step * 4, key, pos);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) lkeys[g * 4 + e] = key[e];
+    }
+    __syncthreads();
+    const uint32_t sn = static_cast<uint32_t>(groups * 4);
+    const double frac = static_cast<double>(sn) / static_cast<double>(n);
+    uint32_t m = static_cast<uint32_t>(1.5 * k * frac) + 8u;
+    const ListSrc ls{lkeys, lposs, static_cast<int64_t>(sn)};
+    // present sampled entries
+    uint32_t c = 0;
+    for (uint32_t i = threadIdx.x; i < sn; i += kTopkThreads) c += lkeys[i] != 0u;
+    uint32_t present;
+    block_excl_scan(c, sc, present);
+    if (m <= present) {
+      uint32_t need;
+      tau = kth_largest(ls, m, hist, sc, need);
+    }
+    __syncthreads();
+  }
+  // ---- one pass: warp-compacted append of every key >= tau.  The test runs on
+  // the float values (x >= value of tau: the same order, -0.0 == +0.0, -inf
+  // never passes); only the few passing values are turned into keys.
+  float tau_f;
+  {
+    const uint32_t b = tau & 0x80000000u ? tau & 0x7FFFFFFFu : ~tau;  // key -> float bits
+    tau_f = tau <= 1u ? -3.402823466e38f : __uint_as_float(b);
+  }
+  uint32_t cnt = 0;  // this warp's entries (warp-uniform)
+  bool overflow = false;
+  uint32_t* wk = lkeys + warp * kRegion;
+  uint32_t* wp = lposs + warp * kRegion;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int64_t nfull = src.aligned ? n / 128 : 0;   // chunks read without bounds checks
+  const int64_t nchunks = (n + 127) / 128;
+  constexpr int U = 8;
+  auto consume = [&](const float (&x)[4], int64_t base) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool pass = x[e] >= tau_f;
+      const uint32_t m = __ballot_sync(0xffffffffu, pass);
+      if (m == 0u) continue;
+      const uint32_t tot = __popc(m);
+      if (cnt + tot > static_cast<uint32_t>(kRegion)) {
+        overflow = true;
+        continue;
+      }
+      if (pass) {
+        const uint32_t slot = cnt + __popc(m & lt_mask);
+        wk[slot] = f2key(x[e]);
+        wp[slot] = static_cast<uint32_t>(base + lane * 4 + e);
+      }
+      cnt += tot;
+    }
+  };
+  int64_t c0 = warp;
+  for (; c0 + (U - 1) * kWarps < nfull; c0 += U * kWarps) {
+    float4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      v[u] = __ldg(reinterpret_cast<const float4*>(src.row + (c0 + u * kWarps) * 128 + lane * 4));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      consume(x, (c0 + u * kWarps) * 128);
+    }
+  }
+  for (; c0 < nchunks; c0 += kWarps) {
+    const int64_t i0 = c0 * 128 + lane * 4;
+    float x[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = i0 + e < n ? __ldg(src.row + i0 + e) : -INFINITY;
+    consume(x, c0 * 128);
+  }
+  if (lane == 0) counts[warp] = overflow ? 0xFFFFFFFFu : cnt;
+  __syncthreads();
+  uint32_t total = 0;
+  bool any_over = false;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    any_over |= counts[w] == 0xFFFFFFFFu;
+    total += counts[w];
+  }
+  if (any_over || (tau > 1u && total < k)) return false;
+  const RegionSrc rs{lkeys, lposs, counts, static_cast<int64_t>(kWarps) * kRegion};
+  // ---- exact k-th key within the list
+  uint32_t T = 0u, need = 0u;
+  if (total > k) T = kth_largest(rs, k, hist, sc, need);
+  // ---- kept positions: key > T, and the `need` lowest positions with key == T
+  uint32_t* nsel = &sc.res[2];
+  uint32_t* neq = &sc.res[3];
+  if (threadIdx.x == 0) {
+    *nsel = 0u;
+    *neq = 0u;
+  }
+  __syncthreads();
+  for (int64_t x = threadIdx.x; x < rs.n; x += kTopkThreads) {
+    const int w = static_cast<int>(x / kRegion), j = static_cast<int>(x % kRegion);
+    if (j >= static_cast<int>(counts[w])) continue;
+    const uint32_t key = lkeys[x];
+    if (key > T) {
+      sel[atomicAdd(nsel, 1u)] = lposs[x];
+    } else if (key == T && key != 0u) {
+      const uint32_t e = atomicAdd(neq, 1u);
+      if (e < static_cast<uint32_t>(kBins1)) hist[e] = lposs[x];
+    }
+  }
+  __syncthreads();
+  const uint32_t n_gt = *nsel, n_eq = *neq;
+  if (n_eq > static_cast<uint32_t>(kBins1)) return false;   // massive ties: fallback
+  if (n_eq > need) bitonic_sort_asc(hist, n_eq, kBins1);      // lowest positions first
+  for (uint32_t i = threadIdx.x; i < need; i += kTopkThreads) sel[n_gt + i] = hist[i];
+  __syncthreads();
+  const uint32_t kept = n_gt + need;
+  bitonic_sort_asc(sel, kept, kFastMaxK);
+  for (uint32_t i = threadIdx.x; i < k; i += kTopkThreads) {
+    if (i < kept)
+      out(i, 0u, sel[i]);
+    else
+      out.out[i] = -1;
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(kTopkThreads)
 topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -247,6 +465,8 @@ topk_kernel(const TopkParams p) {
   SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
   uint32_t* lkeys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
   uint32_t* lposs = lkeys + p.cap;
+  uint32_t* sel = lposs + p.cap;             // fast path only
+  uint32_t* counts = sel + kFastMaxK;        // fast path only
 
   const int t = blockIdx.x;
   const uint32_t k = static_cast<uint32_t>(p.k);
@@ -262,8 +482,12 @@ topk_kernel(const TopkParams p) {
   const RowSrc src{row, n, (reinterpret_cast<uintptr_t>(row) & 15u) == 0u};
   const OutEmit out{p.idx + static_cast<int64_t>(t) * p.k, cand_row, k};
   if (k == 0) return;
+  if (k <= static_cast<uint32_t>(kFastMaxK) &&
+      topk_fast(p, src, out, hist, lkeys, lposs, sel, counts, sc))
+    return;
+  __syncthreads();
 
-  // ---- pass 1: histogram of key >> 20
+  // ---- fallback pass 1: histogram of key >> 20
   for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) hist[i] = 0u;
   __syncthreads();
   {
@@ -299,7 +523,7 @@ topk_kernel(const TopkParams p) {
     const uint32_t in_or_above = above1 + hist[b1];
     __syncthreads();
     if (in_or_above <= static_cast<uint32_t>(p.cap)) {
-      // ---- pass 2: ordered list of the entries in or above bin b1
+      // ordered list of the entries in or above bin b1
       const ListEmit le{lkeys, lposs};
       const uint32_t cnt = ordered_select(src, (b1 << 20) - 1u, 0u, 0xFFFFFFFFu, le, sc);
       __syncthreads();
@@ -320,10 +544,11 @@ cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, 
                         int row_len, const int32_t* cand, int k, int32_t* idx,
                         const DevCtl& ctl, cudaStream_t s) {
   if (n_q <= 0 || k <= 0) return cudaSuccess;
-  int cap = std::max(8192, ((2 * k + 4096) + 1023) / 1024 * 1024);
-  if (cand) cap = std::max(cap, ((row_len + 1023) / 1024) * 1024);
-  cap = std::min(cap, 24576);
-  const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * 8;
+  // list capacity: the fast path needs kFastCap; the fallback wants room for
+  // the entries in or above the k-th histogram bin
+  int cap = k <= kFastMaxK ? kFastCap : std::min(24576, ((2 * k + 4096) + 1023) / 1024 * 1024);
+  const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * 8 +
+                      (k <= kFastMaxK ? (kFastMaxK + kWarps) * 4 : 0);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
