@@ -16,17 +16,18 @@
 // columns: ReLU, the head weights and the head-sum are applied in registers and
 // only the fused logit is written to HBM (per-head logits never leave the SM).
 //
-// Warp roles (320 threads, one CTA per SM, persistent):
+// Warp roles (576 threads for h <= 64, else 320; one CTA per SM, persistent):
 //   warp 0     producer: gathers B for each query group (16-byte cp.async into
 //              the 128-byte-swizzled K-major layout) and streams key tiles with
 //              TMA into a STAGES-deep ring;
 //   warp 1     allocates TMEM (512 columns = two 256-column accumulators) and
 //              issues tcgen05.mma from one thread;
-//   warps 2-9  epilogue, two warps per TMEM lane quadrant, each owning 128 of
-//              the 256 columns: one tcgen05.ld of its 128 columns, the
-//              accumulator released right after the load lands, then the fused
-//              ReLU * w head-sum (packed fp32 FMA), causal mask and coalesced
-//              fp32 stores (a warp stores 32 consecutive keys of one query row).
+//   warps 2-   epilogue, four warps per TMEM lane quadrant each owning 64 of
+//              the 256 columns (two warps owning 128 when h = 128): one
+//              tcgen05.ld of its columns, the accumulator released right after
+//              the load lands, then the fused ReLU * w head-sum (packed fp32
+//              FMA), causal mask and coalesced fp32 stores (a warp stores 32
+//              consecutive keys of one query row).
 // Work is the flattened list of (query group, key tile) pairs, split evenly
 // over the CTAs, so causal triangles stay balanced.
 #include "internal.h"
@@ -36,12 +37,17 @@ namespace {
 
 constexpr int kTileKeys = 128;   // MMA M
 constexpr int kCols = 256;       // MMA N: (query, head) columns per group
-constexpr int kScoreThreads = 320;
-constexpr int kEpiWarps = 8;
-constexpr int kHalfCols = kCols / 2;  // columns per epilogue warp
+// epilogue warps: 4 per TMEM lane quadrant (64 columns each) when a query's h
+// columns fit in 64, else 2 per quadrant (128 columns each)
+template <int HT>
+struct Epi {
+  static constexpr int WARPS = HT <= 64 ? 16 : 8;
+  static constexpr int COLS = kCols / (WARPS / 4);
+  static constexpr int THREADS = 64 + 32 * WARPS;
+};
 constexpr uint64_t kDrainNs = 2000000;  // 2 ms
 
-template <int D>
+template <int D, int HT>
 struct ScoreLayout {
   static constexpr int ROWB = D >= 64 ? 128 : 64;  // bytes per row of one swizzle chunk
   static constexpr int KCH = D * 2 / ROWB;         // swizzle chunks along d
@@ -52,8 +58,8 @@ struct ScoreLayout {
   static constexpr int STAGES = D == 128 ? 4 : 8;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_W = OFF_B + B_BYTES;         // 8 epilogue warps x 128 floats
-  static constexpr int OFF_HEADS = OFF_W + kEpiWarps * kHalfCols * 4;  // producer: heads of a group
+  static constexpr int OFF_W = OFF_B + B_BYTES;         // per epilogue warp: its columns' w
+  static constexpr int OFF_HEADS = OFF_W + Epi<HT>::WARPS * Epi<HT>::COLS * 4;  // producer: heads
   static constexpr int OFF_BAR = OFF_HEADS + kCols * 4;
   static constexpr int NBAR = 2 * STAGES + 6;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -119,9 +125,11 @@ struct Sched {
 };
 
 template <int D, int HT>
-__global__ void __launch_bounds__(kScoreThreads, 1)
+__global__ void __launch_bounds__(Epi<HT>::THREADS, 1)
 score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams p) {
-  using L = ScoreLayout<D>;
+  using L = ScoreLayout<D, HT>;
+  constexpr int EW = Epi<HT>::WARPS;
+  constexpr int EC = Epi<HT>::COLS;
   constexpr int QG = kCols / HT;  // queries per group
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -145,7 +153,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     mbar_init(bar(BEMPTY), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(ACCFULL + i), 1);
-      mbar_init(bar(ACCEMPTY + i), kEpiWarps);
+      mbar_init(bar(ACCEMPTY + i), EW);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -270,9 +278,9 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     // ------------------------------------------------------------ epilogue
     const int e = warp - 2;
     const int quad = warp & 3;   // TMEM lanes quad*32 .. quad*32+31
-    const int half = e >> 2;     // columns half*128 .. half*128+127
-    constexpr int QPW = kHalfCols / HT;  // queries per warp
-    float* w_s = reinterpret_cast<float*>(smem + L::OFF_W) + e * kHalfCols;
+    const int part = e >> 2;     // columns part*EC .. part*EC+EC-1
+    constexpr int QPW = EC / HT;  // queries per warp
+    float* w_s = reinterpret_cast<float*>(smem + L::OFF_W) + e * EC;  // private to this warp
     Sched<QG> it;
     it.init(p);
     int acc = 0;
@@ -280,8 +288,8 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     int prev_g = -1;
     for (; it.left > 0; it.next(p)) {
       if (it.g != prev_g) {
-        for (int i = lane; i < kHalfCols; i += 32) {
-          const int col = half * kHalfCols + i;
+        for (int i = lane; i < EC; i += 32) {
+          const int col = part * EC + i;
           const int t = it.g * QG + col / HT;
           float wv = 0.0f;
           if (t < p.n_q) {
@@ -298,10 +306,13 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
       if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
-      uint32_t v[kHalfCols];
-      tmem_ld128(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                     static_cast<uint32_t>(acc * kCols + half * kHalfCols),
-                 v);
+      uint32_t v[EC];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(acc * kCols + part * EC);
+      if constexpr (EC == 64)
+        tmem_ld64(taddr, v);
+      else
+        tmem_ld128(taddr, v);
       tmem_wait_ld();
       // the accumulator is in registers: hand it back to the MMA warp now
       tc_fence_before();
@@ -313,7 +324,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
       }
       const int64_t s = it.kt * kTileKeys + quad * 32 + lane;
       const bool s_ok = s < p.n_k;
-      const int64_t tq0 = static_cast<int64_t>(it.g) * QG + half * QPW;
+      const int64_t tq0 = static_cast<int64_t>(it.g) * QG + part * QPW;
       float* dst = p.logits + tq0 * p.ld + s;
       if constexpr (HT >= 4) {
         // every head-sum first (the shared-memory weight loads never wait
@@ -367,7 +378,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
 
 template <int D, int HT>
 cudaError_t launch_dh(const ScoreParams& p, const CUtensorMap& map, cudaStream_t s) {
-  using L = ScoreLayout<D>;
+  using L = ScoreLayout<D, HT>;
   auto kern = score_tokens_kernel<D, HT>;
   static bool attr_set = false;  // per process; the attribute is per device but idempotent
   if (!attr_set) {
@@ -377,7 +388,7 @@ cudaError_t launch_dh(const ScoreParams& p, const CUtensorMap& map, cudaStream_t
   }
   const int64_t grid = std::min<int64_t>(sm_count(), p.total_tiles);
   if (grid <= 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), kScoreThreads, L::ALLOC, s>>>(map, p);
+  kern<<<static_cast<unsigned>(grid), Epi<HT>::THREADS, L::ALLOC, s>>>(map, p);
   return cudaGetLastError();
 }
 

@@ -11,9 +11,11 @@
 // Values are mapped to order-preserving 32-bit keys (-0.0 folded onto +0.0,
 // -inf and padding to the reserved key 0).  One CTA per row.
 //
-// Fast path (k <= 4096):
-//   sample   1/32 of the row (strided float4 loads); the exact m-th largest
-//            sampled key, m ~ 1.5 k * (sample / row), becomes a threshold tau;
+// Fast path (k <= 4096, rows of at most 131072 entries):
+//   sample   32 contiguous 128-entry blocks spread over the row; the lower
+//            edge of the 22-bit key bin holding the m-th largest sampled key,
+//            m ~ 1.4 k * (sample / row), becomes a threshold tau (the 2m-th
+//            gives a lower one, used for one re-stream if the list is short);
 //   stream   ONE pass over the row from HBM with no atomics: every key >= tau
 //            is appended, warp-compacted with ballots, to the warp's own region
 //            of a shared-memory list (warps own interleaved 128-entry chunks);
@@ -22,9 +24,9 @@
 //            entry equal to the k-th largest key;
 //   select   three radix rounds (12 + 10 + 10 bits) over the list give the
 //            exact k-th key T and how many entries equal to T are kept (the
-//            lowest positions); the kept positions are sorted ascending
-//            (bitonic) and written out.
-// Fallback (sample too optimistic, list overflow, k > 4096): a 4096-bin
+//            lowest positions); kept positions are set in a bitmap of the row
+//            and a block scan over its words writes them out in ascending order.
+// Fallback (sample too optimistic, list overflow, k > 4096, longer rows): a 4096-bin
 // histogram pass, an ordered collection of the entries in or above the k-th
 // bin (block scans keep position order), the same radix refinement, and an
 // ordered selection pass — over the shared-memory list when it fits, else over
@@ -34,14 +36,17 @@
 namespace misa {
 namespace {
 
-constexpr int kTopkThreads = 512;
+constexpr int kTopkThreads = 256;
 constexpr int kWarps = kTopkThreads / 32;
 constexpr int kBins1 = 4096;
 constexpr int kChunk = 4 * kTopkThreads;  // entries per block-wide step
 constexpr int kFastMaxK = 4096;           // largest k of the fast path
 constexpr int kSampleTarget = 4096;       // sampled entries per row (at most)
 constexpr int kFastCap = 5120;            // list entries of the fast path (all warps)
+constexpr int kCtasPerSm = 3;             // resident CTAs the fast path is sized for
+constexpr double kSampleMargin = 1.4;     // list target: ~1.4 k entries above tau
 constexpr int kRegion = kFastCap / kWarps;  // list entries per warp region
+constexpr int kEqMax = 1024;              // entries equal to the k-th key (fast path)
 
 struct TopkParams {
   const float* vals;
@@ -261,9 +266,9 @@ struct RegionSrc {
   __device__ __forceinline__ void load4(int64_t i0, uint32_t (&key)[4], uint32_t (&pos)[4]) const {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int64_t x = i0 + e;
-      const int w = static_cast<int>(x / kRegion), j = static_cast<int>(x % kRegion);
-      const bool in = x < n && j < static_cast<int>(counts[w]);
+      const uint32_t x = static_cast<uint32_t>(i0) + e;
+      const uint32_t w = x / kRegion, j = x % kRegion;
+      const bool in = x < static_cast<uint32_t>(n) && j < counts[w];
       key[e] = in ? keys[x] : 0u;
       pos[e] = in ? poss[x] : 0u;
     }
@@ -293,16 +298,22 @@ __device__ uint32_t kth_largest(const Src& src, uint32_t m, uint32_t* hist, Smem
   return T;
 }
 
-// Ascending bitonic sort of buf[0..n) in shared memory (n <= cap, cap a power of two).
-__device__ void bitonic_sort_asc(uint32_t* buf, uint32_t n, uint32_t cap) {
-  uint32_t P = 1;
-  while (P < n) P <<= 1;
+// Ascending bitonic sort of buf[0..n) in shared memory (next power of two of n
+// must fit in the buffer).
+__device__ void bitonic_sort_asc(uint32_t* buf, uint32_t n) {
+  uint32_t P = 1, logP = 0;
+  while (P < n) {
+    P <<= 1;
+    ++logP;
+  }
   for (uint32_t i = n + threadIdx.x; i < P; i += kTopkThreads) buf[i] = 0xFFFFFFFFu;
   __syncthreads();
-  for (uint32_t size = 2; size <= P; size <<= 1) {
-    for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
+  for (uint32_t ls = 1; ls <= logP; ++ls) {
+    const uint32_t size = 1u << ls;
+    for (int lst = static_cast<int>(ls) - 1; lst >= 0; --lst) {
+      const uint32_t stride = 1u << lst;
       for (uint32_t i = threadIdx.x; i < P / 2; i += kTopkThreads) {
-        const uint32_t lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
+        const uint32_t lo = ((i >> lst) << (lst + 1)) | (i & (stride - 1)), hi = lo + stride;
         const bool asc = (lo & size) == 0;
         const uint32_t a = buf[lo], b = buf[hi];
         if ((a > b) == asc) {
@@ -313,7 +324,33 @@ __device__ void bitonic_sort_asc(uint32_t* buf, uint32_t n, uint32_t cap) {
       __syncthreads();
     }
   }
-  (void)cap;
+}
+
+// Emits, in ascending order, the positions whose bits are set in bitmap[0..words)
+// to out slots 0.. and pads the rest of the k slots with -1.
+__device__ void emit_bitmap(const uint32_t* bitmap, uint32_t words, const OutEmit& out,
+                            SmemCtl& sc) {
+  constexpr int PER = kBins1 / kTopkThreads;  // words per thread (8)
+  uint32_t wv[PER], c = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const uint32_t wi = threadIdx.x * PER + i;
+    wv[i] = wi < words ? bitmap[wi] : 0u;
+    c += __popc(wv[i]);
+  }
+  uint32_t total;
+  uint32_t slot = block_excl_scan(c, sc, total);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    uint32_t m = wv[i];
+    const uint32_t base = (threadIdx.x * PER + i) * 32u;
+    while (m) {
+      const uint32_t b = __ffs(m) - 1u;
+      out(slot++, 0u, base + b);
+      m &= m - 1u;
+    }
+  }
+  for (uint32_t i = total + threadIdx.x; i < out.k; i += kTopkThreads) out.out[i] = -1;
 }
 
 // Fast path.  Returns false (and writes nothing) when the row must take the
@@ -325,35 +362,60 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   const uint32_t k = out.k;
   const int64_t n = src.n;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // ---- threshold from a sample
-  uint32_t tau = 1u;  // collect every present entry
+  // ---- thresholds from a sample: 32 contiguous 128-entry blocks spread over
+  // the row.  tau (expected ~1.4 k entries above it) is the lower edge of the
+  // 22-bit key bin holding the m-th largest sampled key; tau_retry, used when
+  // the list comes out short, is the same for the 2m-th.
+  uint32_t tau = 1u, tau_retry = 1u;
   if (n > kFastCap) {
-    const int64_t n4 = n / 4;                         // whole float4 groups
-    const int64_t per = n4 / (kSampleTarget / 4);
-    const int64_t step = per > 1 ? per : 1;
-    const int64_t groups = n4 / step < kSampleTarget / 4 ? n4 / step : kSampleTarget / 4;
-    for (int64_t g = threadIdx.x; g < groups; g += kTopkThreads) {
+    constexpr int kBlocks = kSampleTarget / 128;
+    const int64_t gap = (n / kBlocks) & ~static_cast<int64_t>(3);   // keeps float4 alignment
+    for (int i = threadIdx.x; i < kSampleTarget / 4; i += kTopkThreads) {
+      const int b = i / 32, c = i % 32;
       uint32_t key[4], pos[4];
-      src.load4(g * step * 4, key, pos);
+      src.load4(b * gap + c * 4, key, pos);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) lkeys[g * 4 + e] = key[e];
+      for (int e = 0; e < 4; ++e) lkeys[i * 4 + e] = key[e];
     }
     __syncthreads();
-    const uint32_t sn = static_cast<uint32_t>(groups * 4);
+    const uint32_t sn = kSampleTarget;
     const double frac = static_cast<double>(sn) / static_cast<double>(n);
-    uint32_t m = static_cast<uint32_t>(1.5 * k * frac) + 8u;
+    const uint32_t m = static_cast<uint32_t>(kSampleMargin * k * frac) + 8u;
     const ListSrc ls{lkeys, lposs, static_cast<int64_t>(sn)};
-    // present sampled entries
-    uint32_t c = 0;
-    for (uint32_t i = threadIdx.x; i < sn; i += kTopkThreads) c += lkeys[i] != 0u;
+    for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) hist[i] = 0u;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < sn; i += kTopkThreads)
+      if (lkeys[i] != 0u) atomicAdd(&hist[lkeys[i] >> 20], 1u);
+    __syncthreads();
     uint32_t present;
-    block_excl_scan(c, sc, present);
+    {
+      uint32_t c = 0;
+      for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) c += hist[i];
+      block_excl_scan(c, sc, present);
+    }
+    // 22-bit bin lower edges of the m-th and 2m-th largest sampled keys
     if (m <= present) {
-      uint32_t need;
-      tau = kth_largest(ls, m, hist, sc, need);
+      const uint32_t m2 = 2u * m <= present ? 2u * m : present;
+      find_bin<kBins1>(hist, m, sc);
+      const uint32_t b1 = sc.res[0], above1 = sc.res[1];
+      __syncthreads();
+      find_bin<kBins1>(hist, m2, sc);
+      const uint32_t b1r = sc.res[0], above1r = sc.res[1];
+      __syncthreads();
+      digit_hist(ls, 20, b1, 10, hist);
+      find_bin<1024>(hist, m - above1, sc);
+      tau = (b1 << 20) | (sc.res[0] << 10);
+      __syncthreads();
+      digit_hist(ls, 20, b1r, 10, hist);
+      find_bin<1024>(hist, m2 - above1r, sc);
+      tau_retry = (b1r << 20) | (sc.res[0] << 10);
+      if (tau == 0u) tau = 1u;
+      if (tau_retry == 0u) tau_retry = 1u;
     }
     __syncthreads();
   }
+  uint32_t total = 0;
+  for (int attempt = 0; attempt < 2; ++attempt) {
   // ---- one pass: warp-compacted append of every key >= tau.  The test runs on
   // the float values (x >= value of tau: the same order, -0.0 == +0.0, -inf
   // never passes); only the few passing values are turned into keys.
@@ -410,63 +472,65 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   }
   if (lane == 0) counts[warp] = overflow ? 0xFFFFFFFFu : cnt;
   __syncthreads();
-  uint32_t total = 0;
+  total = 0;
   bool any_over = false;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
     any_over |= counts[w] == 0xFFFFFFFFu;
     total += counts[w];
   }
-  if (any_over || (tau > 1u && total < k)) return false;
+  if (any_over) return false;
+  if (tau <= 1u || total >= k) break;
+  // short: every key >= tau is in the list but fewer than k of them; stream
+  // again with the lower threshold (or give up if it is no lower)
+  if (attempt == 1 || tau_retry >= tau) return false;
+  tau = tau_retry;
+  __syncthreads();
+  }  // attempts
   const RegionSrc rs{lkeys, lposs, counts, static_cast<int64_t>(kWarps) * kRegion};
   // ---- exact k-th key within the list
   uint32_t T = 0u, need = 0u;
   if (total > k) T = kth_largest(rs, k, hist, sc, need);
-  // ---- kept positions: key > T, and the `need` lowest positions with key == T
-  uint32_t* nsel = &sc.res[2];
+  // ---- kept positions: key > T, and the `need` lowest positions with key == T,
+  // marked in a bitmap of the row (ascending output without a sort)
+  uint32_t* bitmap = hist;                       // kBins1 words = 131072 positions
+  const uint32_t words = static_cast<uint32_t>((n + 31) / 32);
   uint32_t* neq = &sc.res[3];
-  if (threadIdx.x == 0) {
-    *nsel = 0u;
-    *neq = 0u;
-  }
+  for (uint32_t i = threadIdx.x; i < static_cast<uint32_t>(kBins1); i += kTopkThreads) bitmap[i] = 0u;
+  if (threadIdx.x == 0) *neq = 0u;
   __syncthreads();
-  for (int64_t x = threadIdx.x; x < rs.n; x += kTopkThreads) {
-    const int w = static_cast<int>(x / kRegion), j = static_cast<int>(x % kRegion);
-    if (j >= static_cast<int>(counts[w])) continue;
+  for (uint32_t x = threadIdx.x; x < static_cast<uint32_t>(rs.n); x += kTopkThreads) {
+    const uint32_t w = x / kRegion, j = x % kRegion;
+    if (j >= counts[w]) continue;
     const uint32_t key = lkeys[x];
+    const uint32_t pos = lposs[x];
     if (key > T) {
-      sel[atomicAdd(nsel, 1u)] = lposs[x];
+      atomicOr(&bitmap[pos >> 5], 1u << (pos & 31u));
     } else if (key == T && key != 0u) {
       const uint32_t e = atomicAdd(neq, 1u);
-      if (e < static_cast<uint32_t>(kBins1)) hist[e] = lposs[x];
+      if (e < static_cast<uint32_t>(kEqMax)) sel[e] = pos;
     }
   }
   __syncthreads();
-  const uint32_t n_gt = *nsel, n_eq = *neq;
-  if (n_eq > static_cast<uint32_t>(kBins1)) return false;   // massive ties: fallback
-  if (n_eq > need) bitonic_sort_asc(hist, n_eq, kBins1);      // lowest positions first
-  for (uint32_t i = threadIdx.x; i < need; i += kTopkThreads) sel[n_gt + i] = hist[i];
+  const uint32_t n_eq = *neq;
+  if (n_eq > static_cast<uint32_t>(kEqMax)) return false;      // massive ties: fallback
+  if (n_eq > need) bitonic_sort_asc(sel, n_eq);                // lowest positions first
+  for (uint32_t i = threadIdx.x; i < need; i += kTopkThreads)
+    atomicOr(&bitmap[sel[i] >> 5], 1u << (sel[i] & 31u));
   __syncthreads();
-  const uint32_t kept = n_gt + need;
-  bitonic_sort_asc(sel, kept, kFastMaxK);
-  for (uint32_t i = threadIdx.x; i < k; i += kTopkThreads) {
-    if (i < kept)
-      out(i, 0u, sel[i]);
-    else
-      out.out[i] = -1;
-  }
+  emit_bitmap(bitmap, words, out, sc);
   return true;
 }
 
-__global__ void __launch_bounds__(kTopkThreads)
+__global__ void __launch_bounds__(kTopkThreads, kCtasPerSm)
 topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
   SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
   uint32_t* lkeys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
   uint32_t* lposs = lkeys + p.cap;
-  uint32_t* sel = lposs + p.cap;             // fast path only
-  uint32_t* counts = sel + kFastMaxK;        // fast path only
+  uint32_t* sel = lposs + p.cap;             // fast path only: ties at the k-th key
+  uint32_t* counts = sel + kEqMax;           // fast path only
 
   const int t = blockIdx.x;
   const uint32_t k = static_cast<uint32_t>(p.k);
@@ -482,7 +546,7 @@ topk_kernel(const TopkParams p) {
   const RowSrc src{row, n, (reinterpret_cast<uintptr_t>(row) & 15u) == 0u};
   const OutEmit out{p.idx + static_cast<int64_t>(t) * p.k, cand_row, k};
   if (k == 0) return;
-  if (k <= static_cast<uint32_t>(kFastMaxK) &&
+  if (k <= static_cast<uint32_t>(kFastMaxK) && n <= 32 * kBins1 &&
       topk_fast(p, src, out, hist, lkeys, lposs, sel, counts, sc))
     return;
   __syncthreads();
@@ -548,7 +612,7 @@ cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, 
   // the entries in or above the k-th histogram bin
   int cap = k <= kFastMaxK ? kFastCap : std::min(24576, ((2 * k + 4096) + 1023) / 1024 * 1024);
   const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * 8 +
-                      (k <= kFastMaxK ? (kFastMaxK + kWarps) * 4 : 0);
+                      (k <= kFastMaxK ? (kEqMax + kWarps) * 4 : 0);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
