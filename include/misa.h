@@ -125,6 +125,25 @@ int misa_rerank(const uint16_t* Q, const float* w, const void* K, const float* k
                 const int32_t* cand, int kp, int n_q, int64_t q_pos0, int64_t n_k, int H, int d,
                 int k, int32_t* idx, float* full_logits, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * misa_rerank for callers that cannot allocate device memory.  The MISA pages
+ * have no counterpart: this is a packaging variant of misa_rerank, not a step of
+ * the method.  Callers inside a fixed memory pool they do not own, inside a
+ * region where cudaMalloc is forbidden, or without a device allocator cannot
+ * hand misa_rerank its n_q * kp floats of workspace; this entry point keeps
+ * that scratch in a 16 MiB device array inside the library instead (held on
+ * every GPU that loads the library until exit) and allocates nothing.
+ * Arguments and results are those of misa_rerank without full_logits and
+ * workspace.  Limit: n_q * kp <= 4194304, else MISA_ERR_WORKSPACE before any
+ * launch (call it on smaller query chunks).  All calls on a device share the
+ * scratch: calls that overlap on the GPU (unordered streams) race on it.  The
+ * first call on each device looks the array's address up (a CUDA runtime
+ * call), so make it outside any stream capture.
+ */
+int misa_rerank_noalloc(const uint16_t* Q, const float* w, const void* K, const float* k_scale,
+                        int kdtype, const int32_t* cand, int kp, int n_q, int64_t q_pos0,
+                        int64_t n_k, int H, int d, int k, int32_t* idx, void* stream);
+
 /* Workspace bytes needed by op "topk" or "rerank" for the given sizes (0 if none). */
 size_t misa_workspace_size(const char* op, int n_q, int64_t n_k, int k, int kp);
 

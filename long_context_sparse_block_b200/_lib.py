@@ -42,6 +42,8 @@ _SIGS = {
     "misa_topk": (_int, [_vp, _i64, _int, _i64, _i64, _int, _vp, _vp, _sz, _vp]),
     "misa_rerank": (_int, [_vp, _vp, _vp, _vp, _int, _vp, _int, _int, _i64, _i64, _int, _int, _int,
                            _vp, _vp, _vp, _sz, _vp]),
+    "misa_rerank_noalloc": (_int, [_vp, _vp, _vp, _vp, _int, _vp, _int, _int, _i64, _i64, _int,
+                                   _int, _int, _vp, _vp]),
     "misa_workspace_size": (_sz, [ctypes.c_char_p, _int, _i64, _int, _int]),
     "misa_status_string": (ctypes.c_char_p, [_int]),
     "misa_last_device_status": (_int, [_vp]),
@@ -178,6 +180,21 @@ def misa_rerank(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, want_full: boo
                           _ptr(ws, name="ws") if full is None else None, ws_bytes, _stream())
     _check("misa_rerank", st)
     return (idx, full) if want_full else idx
+
+
+def misa_rerank_noalloc(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, idx=None):
+    """misa_rerank without workspace: the library's own fixed scratch (at most
+    4194304 candidate scores per call) stands in for it."""
+    n_q, H, d = Q.shape
+    kp = cand.shape[1]
+    if idx is None:
+        idx = torch.empty((n_q, k), dtype=torch.int32, device=Q.device)
+    st = _lib.misa_rerank_noalloc(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                                  _ptr(K, name="K"), _ptr(k_scale, (torch.float32,), "k_scale"),
+                                  _kdtype(K), _ptr(cand, (torch.int32,), "cand"), kp, n_q, q_pos0,
+                                  K.shape[0], H, d, k, _ptr(idx, (torch.int32,), "idx"), _stream())
+    _check("misa_rerank_noalloc", st)
+    return idx
 
 
 def misa_last_device_status() -> int:

@@ -60,6 +60,10 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MISA_OK : MISA_ERR_CU
 
 }  // namespace
 
+int* device_status_word() { return status_ptr(); }
+
+unsigned long long wait_limit_ns() { return g_wait_ns.load(); }
+
 int sm_count() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return 148;

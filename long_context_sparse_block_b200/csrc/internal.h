@@ -11,6 +11,10 @@ namespace misa {
 
 int sm_count();  // of the current device
 
+// The current device's status word and the bounded-wait budget (api.cu).
+int* device_status_word();
+unsigned long long wait_limit_ns();
+
 cudaError_t launch_pool_keys(const void* K, const float* k_scale, bool fp8, int64_t n_k, int d,
                              int B, float* kbar, uint16_t* kbar_hl, cudaStream_t s);
 
