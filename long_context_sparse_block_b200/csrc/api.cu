@@ -151,7 +151,6 @@ int misa_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads, c
   if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
   if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
   if (!good_d(d) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
-  if (kdtype == MISA_K_FP8E4M3) return MISA_ERR_UNSUPPORTED;
   if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
   if (n_q == 0) return MISA_OK;
   DevCtl ctl;

@@ -30,6 +30,8 @@
 //              consecutive keys of one query row).
 // Work is the flattened list of (query group, key tile) pairs, split evenly
 // over the CTAs, so causal triangles stay balanced.
+#include <cstring>
+
 #include "internal.h"
 
 namespace misa {
@@ -38,16 +40,19 @@ namespace {
 constexpr int kTileKeys = 128;   // MMA M
 constexpr int kCols = 256;       // MMA N: (query, head) columns per group
 // epilogue warps: 4 per TMEM lane quadrant (64 columns each) when a query's h
-// columns fit in 64, else 2 per quadrant (128 columns each)
-template <int HT>
+// columns fit in 64, else 2 per quadrant (128 columns each).  FP8 keys add 2
+// converter warps (e4m3 -> bf16 into the swizzled key tile) before them.
+template <int HT, bool FP8>
 struct Epi {
   static constexpr int WARPS = HT <= 64 ? 16 : 8;
   static constexpr int COLS = kCols / (WARPS / 4);
-  static constexpr int THREADS = 64 + 32 * WARPS;
+  static constexpr int CONV = FP8 ? 2 : 0;
+  static constexpr int BASE = 2 + CONV;  // first epilogue warp
+  static constexpr int THREADS = 32 * (BASE + WARPS);
 };
 constexpr uint64_t kDrainNs = 2000000;  // 2 ms
 
-template <int D, int HT>
+template <int D, int HT, bool FP8>
 struct ScoreLayout {
   static constexpr int ROWB = D >= 64 ? 128 : 64;  // bytes per row of one swizzle chunk
   static constexpr int KCH = D * 2 / ROWB;         // swizzle chunks along d
@@ -59,7 +64,7 @@ struct ScoreLayout {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_W = OFF_B + B_BYTES;         // per epilogue warp: its columns' w
-  static constexpr int OFF_HEADS = OFF_W + Epi<HT>::WARPS * Epi<HT>::COLS * 4;  // producer: heads
+  static constexpr int OFF_HEADS = OFF_W + Epi<HT, FP8>::WARPS * Epi<HT, FP8>::COLS * 4;  // producer
   static constexpr int OFF_BAR = OFF_HEADS + kCols * 4;
   static constexpr int NBAR = 2 * STAGES + 6;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -72,6 +77,7 @@ struct ScoreParams {
   const float* w;
   const int32_t* heads;  // nullptr: all heads
   const float* k_scale;  // FP8 keys only
+  const uint8_t* K8;     // FP8 keys only
   float* logits;
   int64_t ld;
   int n_q;
@@ -124,12 +130,13 @@ struct Sched {
   }
 };
 
-template <int D, int HT>
-__global__ void __launch_bounds__(Epi<HT>::THREADS, 1)
+template <int D, int HT, bool FP8>
+__global__ void __launch_bounds__(Epi<HT, FP8>::THREADS, 1)
 score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams p) {
-  using L = ScoreLayout<D, HT>;
-  constexpr int EW = Epi<HT>::WARPS;
-  constexpr int EC = Epi<HT>::COLS;
+  using L = ScoreLayout<D, HT, FP8>;
+  constexpr int EW = Epi<HT, FP8>::WARPS;
+  constexpr int EC = Epi<HT, FP8>::COLS;
+  constexpr int CONV = Epi<HT, FP8>::CONV;
   constexpr int QG = kCols / HT;  // queries per group
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -146,7 +153,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::STAGES; ++i) {
-      mbar_init(bar(FULL + i), 1);
+      mbar_init(bar(FULL + i), FP8 ? 32 * CONV : 1);
       mbar_init(bar(EMPTY + i), 1);
     }
     mbar_init(bar(BFULL), 32);
@@ -157,7 +164,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     }
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&kmap);
+    if (!FP8) tma_prefetch_desc(&kmap);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -212,6 +219,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
         prev_g = it.g;
         ++gcount;
       }
+      if (FP8) continue;  // key tiles come from the converter warps
       bool ok = true;
       if (lane == 0) {
         ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
@@ -274,9 +282,52 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
         accph ^= 1;
       }
     }
+  } else if (warp < Epi<HT, FP8>::BASE) {
+    // ------------------------------------------------------------ FP8 key converters
+    // e4m3 key rows -> bf16 (exact) straight into the swizzled key tile
+    if constexpr (FP8) {
+      const int ct = threadIdx.x - 64;  // 0 .. 32*CONV-1
+      constexpr int U8 = D / 16;        // 16-byte e4m3 units per key row
+      constexpr int UPC = L::ROWB / 16; // bf16 16-byte units per swizzle-chunk row
+      Sched<QG> it;
+      it.init(p);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (; it.left > 0; it.next(p)) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        const uint32_t dst = sA + stage * L::A_BYTES;
+        for (int x = ct; x < kTileKeys * U8; x += 32 * CONV) {
+          const int r = x / U8, u = x % U8;
+          const int64_t key = it.kt * kTileKeys + r;
+          uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+          if (key < p.n_k) raw = __ldg(reinterpret_cast<const uint4*>(p.K8 + key * D + u * 16));
+          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t b0 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh] & 0xFFFF));
+            const uint32_t b1 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh] >> 16));
+            const uint32_t b2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh + 1] & 0xFFFF));
+            const uint32_t b3 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh + 1] >> 16));
+            const int u2 = 2 * u + hh;  // bf16 unit of the row
+            const uint32_t off = (u2 / UPC) * L::A_CHUNK + swz_offset(r, u2 % UPC, L::ROWB);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + off), "r"(b0),
+                         "r"(b1), "r"(b2), "r"(b3)
+                         : "memory");
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(FULL + stage));
+        if (++stage == L::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 2;
+    const int e = warp - Epi<HT, FP8>::BASE;
     const int quad = warp & 3;   // TMEM lanes quad*32 .. quad*32+31
     const int part = e >> 2;     // columns part*EC .. part*EC+EC-1
     constexpr int QPW = EC / HT;  // queries per warp
@@ -344,6 +395,12 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
           }
           sums[qq] = a2.x + a2.y;
         }
+        if constexpr (FP8) {
+          // per-token scale > 0: w * ReLU(scale * dot) = scale * w * ReLU(dot)
+          const float ks = s_ok ? __ldg(p.k_scale + s) : 0.0f;
+#pragma unroll
+          for (int qq = 0; qq < QPW; ++qq) sums[qq] *= ks;
+        }
 #pragma unroll
         for (int qq = 0; qq < QPW; ++qq) {
           const int64_t t = tq0 + qq;
@@ -360,6 +417,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
             const float2 w2 = *reinterpret_cast<const float2*>(w_s + qq * 2);
             sum = fmaf(w2.y, relu(__uint_as_float(v[qq * 2 + 1])), w2.x * relu(__uint_as_float(v[qq * 2])));
           }
+          if constexpr (FP8) sum *= s_ok ? __ldg(p.k_scale + s) : 0.0f;
           const int64_t t = tq0 + qq;
           if (t < p.n_q && s_ok) *dst = (s <= p.q_pos0 + t) ? sum : -INFINITY;
           dst += p.ld;
@@ -376,10 +434,10 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
   }
 }
 
-template <int D, int HT>
+template <int D, int HT, bool FP8>
 cudaError_t launch_dh(const ScoreParams& p, const CUtensorMap& map, cudaStream_t s) {
-  using L = ScoreLayout<D, HT>;
-  auto kern = score_tokens_kernel<D, HT>;
+  using L = ScoreLayout<D, HT, FP8>;
+  auto kern = score_tokens_kernel<D, HT, FP8>;
   static bool attr_set = false;  // per process; the attribute is per device but idempotent
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
@@ -388,21 +446,21 @@ cudaError_t launch_dh(const ScoreParams& p, const CUtensorMap& map, cudaStream_t
   }
   const int64_t grid = std::min<int64_t>(sm_count(), p.total_tiles);
   if (grid <= 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), Epi<HT>::THREADS, L::ALLOC, s>>>(map, p);
+  kern<<<static_cast<unsigned>(grid), Epi<HT, FP8>::THREADS, L::ALLOC, s>>>(map, p);
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t launch_d(const ScoreParams& p, int h, const CUtensorMap& map, cudaStream_t s) {
   switch (h) {
-    case 1: return launch_dh<D, 1>(p, map, s);
-    case 2: return launch_dh<D, 2>(p, map, s);
-    case 4: return launch_dh<D, 4>(p, map, s);
-    case 8: return launch_dh<D, 8>(p, map, s);
-    case 16: return launch_dh<D, 16>(p, map, s);
-    case 32: return launch_dh<D, 32>(p, map, s);
-    case 64: return launch_dh<D, 64>(p, map, s);
-    case 128: return launch_dh<D, 128>(p, map, s);
+    case 1: return launch_dh<D, 1, FP8>(p, map, s);
+    case 2: return launch_dh<D, 2, FP8>(p, map, s);
+    case 4: return launch_dh<D, 4, FP8>(p, map, s);
+    case 8: return launch_dh<D, 8, FP8>(p, map, s);
+    case 16: return launch_dh<D, 16, FP8>(p, map, s);
+    case 32: return launch_dh<D, 32, FP8>(p, map, s);
+    case 64: return launch_dh<D, 64, FP8>(p, map, s);
+    case 128: return launch_dh<D, 128, FP8>(p, map, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -413,7 +471,6 @@ cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t
                                 const void* K, const float* k_scale, bool fp8, int n_q,
                                 int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
                                 int64_t ld, const DevCtl& ctl, cudaStream_t s) {
-  if (fp8) return cudaErrorNotSupported;
   if (n_q <= 0) return cudaSuccess;
   const int QG = kCols / h;
   const int n_groups = (n_q + QG - 1) / QG;
@@ -422,8 +479,18 @@ cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t
     const int t_last = std::min((g + 1) * QG, n_q) - 1;
     total += (q_pos0 + t_last) / kTileKeys + 1;
   }
-  ScoreParams p{Q, w, heads, k_scale, logits, ld, n_q, q_pos0, n_k, H, total, ctl};
+  ScoreParams p{Q, w, heads, k_scale, static_cast<const uint8_t*>(K), logits, ld, n_q, q_pos0, n_k,
+                H, total, ctl};
   CUtensorMap map;
+  if (fp8) {
+    std::memset(&map, 0, sizeof map);  // unused: converter warps read the e4m3 keys
+    switch (d) {
+      case 32: return launch_d<32, true>(p, h, map, s);
+      case 64: return launch_d<64, true>(p, h, map, s);
+      case 128: return launch_d<128, true>(p, h, map, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   const uint64_t dims[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_k)};
   const uint64_t strides[1] = {static_cast<uint64_t>(d) * 2};
   const int rowb = d >= 64 ? 128 : 64;
@@ -433,9 +500,9 @@ cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t
       CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   switch (d) {
-    case 32: return launch_d<32>(p, h, map, s);
-    case 64: return launch_d<64>(p, h, map, s);
-    case 128: return launch_d<128>(p, h, map, s);
+    case 32: return launch_d<32, false>(p, h, map, s);
+    case 64: return launch_d<64, false>(p, h, map, s);
+    case 128: return launch_d<128, false>(p, h, map, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -65,18 +65,22 @@ def test_full_size_sampled_rows(name):
     assert matched >= len(rows) - 2
 
 
-def test_full_size_dagger_sampled_rows():
+@pytest.mark.parametrize("fp8", [False, True])
+def test_full_size_dagger_sampled_rows(fp8):
+    # MISA-dagger on the 8192 x 131072 chunk; fp8=True stores the keys as e4m3
+    # with a per-token scale for every stage (pool, route, score, rerank)
     from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
     wl = W.WORKLOADS["dagger_128k"]
-    inp = W.generate(wl)
+    inp = W.generate(wl, fp8_keys=fp8)
     rows = _rows(wl)
-    g = inputs_to_device(inp)
+    g = inputs_to_device(inp, fp8=fp8)
     ix = MisaIndexer(IndexerShape(wl.n_q, wl.q_pos0, wl.n_k, wl.H, wl.d, wl.B, wl.h, wl.k,
                                   kp=wl.kp, sub_chunk=1024))
-    fin = ix.run(g["Q"], g["K"], g["w"]).cpu().numpy()
+    K = g["K8"] if fp8 else g["K"]
+    fin = ix.run(g["Q"], K, g["w"], k_scale=g.get("k_scale")).cpu().numpy()
     cand = ix.sel.cpu().numpy()
     heads = ix.heads.cpu().numpy()
-    Kd = oracle.bf16_to_f64(inp["K"])
+    Kd = oracle.e4m3_keys_to_f64(inp["K8"], inp["k_scale"]) if fp8 else oracle.bf16_to_f64(inp["K"])
     kbar = oracle.pool_keys(Kd, wl.B)
     sel = np.array(rows)
     Qd = oracle.bf16_to_f64(inp["Q"][sel])

@@ -113,6 +113,31 @@ def test_score_matches_oracle(lib, n_q, q_pos0, n_k, H, d, h, dense):
         assert np.all(np.isnan(out[t, n_k:]))                             # never past n_k
 
 
+@pytest.mark.parametrize("n_q,q_pos0,n_k,H,d,h", [(70, 300, 517, 64, 128, 8), (257, 3, 300, 8, 32, 2),
+                                                  (40, 1000, 1100, 32, 64, 16),
+                                                  (9, 200, 250, 64, 128, 64),
+                                                  (100, 0, 100, 64, 128, 4)])
+def test_score_fp8_keys_matches_oracle(lib, n_q, q_pos0, n_k, H, d, h):
+    # keys stored as e4m3 with a per-token fp32 scale, decoded in the kernel
+    wl = _wl(n_q, q_pos0, n_k, H, d, 64, h, 8, seed=11 * n_q + h)
+    inp = W.generate(wl, fp8_keys=True)
+    Qd, Kd, wd = oracle.decode_inputs(inp, fp8_keys=True)
+    rng = np.random.default_rng(n_q + 1)
+    heads = np.sort(np.stack([rng.choice(H, size=h, replace=False) for _ in range(n_q)]),
+                    axis=1).astype(np.int32)
+    ref = oracle.score(Qd, wd, heads, Kd, q_pos0)
+    g = inputs_to_device(inp, fp8=True)
+    logits = torch.full((n_q, n_k), float("nan"), device="cuda")
+    lib.misa_score_tokens(g["Q"], g["w"], dev(heads), g["K8"], q_pos0, k_scale=g["k_scale"],
+                          logits=logits, h=h)
+    assert lib.misa_last_device_status() == 0
+    out = logits.cpu().numpy()
+    for t in range(n_q):
+        pos = q_pos0 + t
+        mag = logit_magnitude(Qd, wd, Kd, heads, t, q_pos0)
+        assert_logits_close(out[t], ref[t, :pos + 1], mag, what=f"fp8 row {t}")
+
+
 def test_exact_arithmetic_is_bitwise(lib):
     # small integers and power-of-two weights: every product and sum is exact in
     # fp32, so pool, router scores, heads, logits and top-k must match exactly.
