@@ -42,6 +42,22 @@ from long_context_sparse_block_b200 import workloads as W  # noqa: E402
 
 METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor peak"
 
+# DRAM bytes (read + write) of one score launch (first 1024-query sub-chunk) from
+# the ncu capture in profiles/score_tokens_chunk_128k.md, valid only for the
+# kernel sources it was taken on.
+SCORE_TRAFFIC = {"sources_sha256_16": "f9d4a13d8e7e739f", "bytes_per_launch": 134.102528e6 + 459.236608e6,
+                 "launch": "queries 0..1023 of chunk_128k"}
+
+
+def _score_sources_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("long_context_sparse_block_b200/csrc/score.cu",
+              "long_context_sparse_block_b200/csrc/common.cuh"):
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
 
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -244,6 +260,12 @@ def run_ours(args, rank, world, local_rank, inp):
     clk = clocks.stop() if rank == 0 else None
     assert _lib.misa_last_device_status() == 0, "device status"
     step_ms = [a.elapsed_time(b) for a, b in spans]
+    variants = None
+    if rank == 0 and world == 1 and not args.no_variants and args.workload == "chunk_128k":
+        del ix
+        variants = run_variants(wl, inp, stream, flush)
+        ix = MisaIndexer(shape)
+        assert _lib.misa_last_device_status() == 0, "device status"
     stage_ms = {}
     for ev in stage_events:
         for name, a, b in ev:
@@ -285,6 +307,9 @@ def run_ours(args, rank, world, local_rank, inp):
 
     peaks = _peaks()
     pairs = wl.causal_pairs()
+    traffic = (SCORE_TRAFFIC["bytes_per_launch"]
+               if h == 8 and wl.name == "chunk_128k"
+               and _score_sources_digest() == SCORE_TRAFFIC["sources_sha256_16"] else None)
     score_flops = 2.0 * h * wl.d * pairs
     score_ms = stage_ms["score"]
     tflops = score_flops / (score_ms * 1e-3) / 1e12
@@ -325,7 +350,8 @@ def run_ours(args, rank, world, local_rank, inp):
             "unit": "TFLOP/s",
             "frac": round(tflops / peaks["bf16_tflops"], 4),
             "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
-            "traffic": None,
+            "traffic": traffic,
+            "traffic_unit": "bytes per launch (ncu dram read+write)",
             "algorithmic": f"2*h*d*pairs = {score_flops:.4g} flop per step, {pairs} causal pairs",
         },
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
@@ -342,6 +368,80 @@ def run_ours(args, rank, world, local_rank, inp):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if variants is not None:
+        out["variants"] = variants
+    return out
+
+
+def _time_ms(fn, stream, flush, reps=5, warm=2):
+    import torch
+    ts = []
+    for i in range(warm + reps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        if i >= warm:
+            ts.append(a.elapsed_time(b))
+    return statistics.mean(ts)
+
+
+def _recall(sel, ref, n_k):
+    """Mean over rows of |sel & ref| / |ref| (token sets, -1 padding ignored)."""
+    import torch
+    hit = tot = 0
+    for r0 in range(0, ref.shape[0], 512):
+        a, b = sel[r0:r0 + 512].long(), ref[r0:r0 + 512].long()
+        mark = torch.zeros((b.shape[0], n_k + 1), dtype=torch.bool, device=b.device)
+        mark.scatter_(1, torch.where(b >= 0, b, n_k), True)
+        mark[:, n_k] = False
+        hit += int(mark.gather(1, torch.where(a >= 0, a, n_k)).sum())
+        tot += int((b >= 0).sum())
+    return hit / max(tot, 1)
+
+
+def run_variants(wl, inp, stream, flush):
+    """The other measured configurations of the chunk: h=4, the dense 64-head
+    indexer in this library, MISA-dagger (k'=8192, all-head rerank to 2048) with
+    bf16 and with FP8 keys, and the recall of each against the dense top-k."""
+    import torch
+
+    from long_context_sparse_block_b200 import workloads as Wm
+    from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
+
+    def d16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+    Q, K, w = d16(inp["Q"]), d16(inp["K"]), torch.from_numpy(inp["w"]).cuda()
+    base = dict(n_q=wl.n_q, q_pos0=wl.q_pos0, n_k=wl.n_k, H=wl.H, d=wl.d, B=wl.B, k=wl.k)
+    out = {}
+    dense = MisaIndexer(IndexerShape(h=wl.H, dense=True, **base))
+    out["dense_h64_ms"] = round(_time_ms(lambda: dense.run(Q, K, w), stream, flush), 4)
+    ref = dense.run(Q, K, w).clone()
+    for h in (8, 4):
+        ix = MisaIndexer(IndexerShape(h=h, **base))
+        out[f"misa_h{h}_ms"] = round(_time_ms(lambda: ix.run(Q, K, w), stream, flush), 4)
+        out[f"misa_h{h}_recall_vs_dense"] = round(_recall(ix.run(Q, K, w), ref, wl.n_k), 4)
+    dg = MisaIndexer(IndexerShape(h=wl.h, kp=8192, **base))
+    out["dagger_ms"] = round(_time_ms(lambda: dg.run(Q, K, w), stream, flush), 4)
+    out["dagger_recall_vs_dense"] = round(_recall(dg.run(Q, K, w), ref, wl.n_k), 4)
+    del dense, ref, dg
+    # FP8 keys (e4m3 + per-token scale), every stage decoding in-kernel
+    K8c, sc = Wm.e4m3_quantize_keys(Wm.bf16_values(inp["K"]).astype(np.float64))
+    K8 = torch.from_numpy(K8c).cuda()
+    ks = torch.from_numpy(sc).cuda()
+    dense8 = MisaIndexer(IndexerShape(h=wl.H, dense=True, **base))
+    ref8 = dense8.run(Q, K8, w, k_scale=ks).clone()
+    del dense8
+    dg8 = MisaIndexer(IndexerShape(h=wl.h, kp=8192, **base))
+    out["dagger_fp8_ms"] = round(_time_ms(lambda: dg8.run(Q, K8, w, k_scale=ks), stream, flush), 4)
+    fin8 = dg8.run(Q, K8, w, k_scale=ks)
+    out["dagger_fp8_recall_vs_dense_fp8"] = round(_recall(fin8, ref8, wl.n_k), 4)
+    dense_bf = MisaIndexer(IndexerShape(h=wl.H, dense=True, **base))
+    out["dagger_fp8_recall_vs_dense_bf16"] = round(_recall(fin8, dense_bf.run(Q, K, w), wl.n_k), 4)
     return out
 
 
@@ -375,6 +475,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the h=4 / dense / MISA-dagger / FP8 measurements")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
