@@ -16,9 +16,14 @@
 // own row's causal columns, then the 4 epilogue warps exchange r through shared
 // memory and one warp per query runs the top-h as h rounds of a warp argmax.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
-// issuer, warps 2-5 epilogue.  Row tiles are distributed round-robin over a
-// persistent grid.
+// Warp roles (256 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
+// issuer, warps 2-5 epilogue (one per TMEM lane quadrant: one tcgen05.ld of
+// the 128 block columns per tile, the accumulator handed back right after it
+// lands), warps 6-7 top-h selection.  The epilogue hands each row tile's
+// partial sums to the top-h warps through a double-buffered shared array, so
+// the (latency-bound) selection of one row tile overlaps the contraction of
+// the next.  Pooled-key tiles stream through a 3-stage ring.  Row tiles are
+// distributed round-robin over a persistent grid.
 #include "internal.h"
 
 namespace misa {
@@ -26,8 +31,10 @@ namespace {
 
 constexpr int kRows = 128;    // MMA M: (query, head) rows per tile
 constexpr int kBlkN = 128;    // MMA N: pooled blocks per tile
-constexpr int kRouteThreads = 192;
-constexpr int kRouteStages = 2;
+constexpr int kRouteEpiWarps = 4;
+constexpr int kRouteTopWarps = 2;
+constexpr int kRouteThreads = 64 + 32 * (kRouteEpiWarps + kRouteTopWarps);
+constexpr int kRouteStages = 3;
 constexpr uint64_t kDrainNs = 2000000;
 
 template <int D>
@@ -40,9 +47,9 @@ struct RouteLayout {
   static constexpr int B_HALF = kBlkN * D * 2;           // hi or lo tile
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + A_BYTES;
-  static constexpr int OFF_R = OFF_B + kRouteStages * 2 * B_HALF;
-  static constexpr int OFF_BAR = OFF_R + kRows * 4;
-  static constexpr int NBAR = 2 * kRouteStages + 7;
+  static constexpr int OFF_R = OFF_B + kRouteStages * 2 * B_HALF;  // [2 buf][kRows] block sums
+  static constexpr int OFF_BAR = OFF_R + 2 * kRows * 4;
+  static constexpr int NBAR = 2 * kRouteStages + 10;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
@@ -96,7 +103,7 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   auto bar = [&](int i) { return smem_u32(bars + i); };
   const int FULL = 0, EMPTY = kRouteStages, AFULL = 2 * kRouteStages, AEMPTY = AFULL + 1,
-            ACCFULL = AFULL + 2, ACCEMPTY = AFULL + 4, ESYNC = AFULL + 6;
+            ACCFULL = AFULL + 2, ACCEMPTY = AFULL + 4, RFULL = AFULL + 6, REMPTY = AFULL + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -110,9 +117,12 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
     mbar_init(bar(AEMPTY), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(ACCFULL + i), 1);
-      mbar_init(bar(ACCEMPTY + i), 4);
+      mbar_init(bar(ACCEMPTY + i), kRouteEpiWarps);
     }
-    mbar_init(bar(ESYNC), 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(RFULL + i), kRouteEpiWarps);
+      mbar_init(bar(REMPTY + i), kRouteTopWarps);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&qmap);
@@ -211,108 +221,121 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
       ++tcount;
     }
   } else {
-    // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;  // TMEM lane of this thread
+    // ------------------------------------------------------------ epilogue / top-h
+    const bool top_role = warp >= 2 + kRouteEpiWarps;
     const int QT = kRows / p.H;
-    int acc = 0;
-    uint32_t accph = 0, esync = 0;
+    uint32_t rcount = 0;  // row tiles handed over so far (buffer = rcount & 1)
     bool ok = true;
-    for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x) {
-      const int nN = ntiles_of(p, rt);
-      const int t = rt * QT + row / p.H;
-      const int j = row % p.H;
-      const bool valid = t < p.n_q;
-      const int64_t nc = valid ? causal_blocks(p, p.q_pos0 + t) : 0;
-      float sum = 0.0f;
-      for (int nb = 0; nb < nN; ++nb) {
-        if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
+    if (!top_role) {
+      const int quad = warp & 3;
+      const int row = quad * 32 + lane;   // TMEM lane of this thread
+      int acc = 0;
+      uint32_t accph = 0;
+      for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x, ++rcount) {
+        const int nN = ntiles_of(p, rt);
+        const int t = rt * QT + row / p.H;
+        const bool valid = t < p.n_q;
+        const int64_t nc = valid ? causal_blocks(p, p.q_pos0 + t) : 0;
+        float sum = 0.0f;
+        for (int nb = 0; nb < nN; ++nb) {
+          if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t v[kBlkN];
+          tmem_ld128(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                         static_cast<uint32_t>(acc * kBlkN),
+                     v);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
+          if (++acc == 2) {
+            acc = 0;
+            accph ^= 1;
+          }
+          const int64_t m0 = static_cast<int64_t>(nb) * kBlkN;
+          if (m0 + kBlkN <= nc) {
+            float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+#pragma unroll
+            for (int i = 0; i < kBlkN; i += 4) {
+              s0 += relu(__uint_as_float(v[i]));
+              s1 += relu(__uint_as_float(v[i + 1]));
+              s2 += relu(__uint_as_float(v[i + 2]));
+              s3 += relu(__uint_as_float(v[i + 3]));
+            }
+            sum += (s0 + s1) + (s2 + s3);
+          } else {
+#pragma unroll
+            for (int i = 0; i < kBlkN; ++i)
+              if (m0 + i < nc) sum += relu(__uint_as_float(v[i]));
+          }
+        }
+        if (!ok) break;
+        // hand the partial sums of this row tile to the top-h warps
+        const uint32_t buf = rcount & 1;
+        if (lane == 0) ok = mbar_wait(bar(REMPTY + buf), ((rcount >> 1) & 1) ^ 1, abort_flag, p.ctl);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        tc_fence_after();
-        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                               static_cast<uint32_t>(acc * kBlkN);
-        const int64_t m0 = static_cast<int64_t>(nb) * kBlkN;
-#pragma unroll 1
-        for (int c = 0; c < kBlkN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tbase + static_cast<uint32_t>(c * 32), v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (m0 + c * 32 + i < nc) sum += relu(__uint_as_float(v[i]));
-        }
-        tc_fence_before();
+        r_s[buf * kRows + row] = sum;
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
-        if (++acc == 2) {
-          acc = 0;
-          accph ^= 1;
-        }
+        if (lane == 0) mbar_arrive(bar(RFULL + buf));
       }
-      if (!ok) break;
-      float r = 0.0f;
-      if (valid) {
-        r = __ldg(p.w + static_cast<int64_t>(t) * p.H + j) * sum;
-        if (p.r_out) p.r_out[static_cast<int64_t>(t) * p.H + j] = r;
-      }
-      r_s[row] = r;
-      // all four epilogue warps have written r_s
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(ESYNC));
-        ok = mbar_wait(bar(ESYNC), esync & 1, abort_flag, p.ctl);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      ++esync;
-      if (!ok) break;
-      // top-h: one warp per query
-      for (int qq = quad; qq < QT; qq += 4) {
-        const int tq = rt * QT + qq;
-        if (tq >= p.n_q) break;
-        constexpr int SL = 4;  // slots per lane: H <= 128
-        float rv[SL];
-        bool taken[SL];
+    } else {
+      // top-h: one warp per query, h rounds of a warp argmax by (r desc, head asc)
+      const int tw = warp - 2 - kRouteEpiWarps;
+      for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x, ++rcount) {
+        const uint32_t buf = rcount & 1;
+        if (lane == 0) ok = mbar_wait(bar(RFULL + buf), (rcount >> 1) & 1, abort_flag, p.ctl);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const float* rb = r_s + buf * kRows;
+        for (int qq = tw; qq < QT; qq += kRouteTopWarps) {
+          const int tq = rt * QT + qq;
+          if (tq >= p.n_q) break;
+          constexpr int SL = 4;  // slots per lane: H <= 128
+          float rv[SL];
+          bool taken[SL];
 #pragma unroll
-        for (int i = 0; i < SL; ++i) {
-          const int jj = lane + 32 * i;
-          taken[i] = jj >= p.H;
-          rv[i] = taken[i] ? 0.0f : r_s[qq * p.H + jj];
-        }
-        for (int round = 0; round < p.h; ++round) {
-          float br = -INFINITY;
-          int bj = 0x7fffffff;
-#pragma unroll
-          for (int i = 0; i < SL; ++i)
-            if (!taken[i]) better(br, bj, rv[i], lane + 32 * i);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) {
-            const float orr = __shfl_xor_sync(0xffffffffu, br, off);
-            const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-            better(br, bj, orr, oj);
+          for (int i = 0; i < SL; ++i) {
+            const int jj = lane + 32 * i;
+            taken[i] = jj >= p.H;
+            rv[i] = 0.0f;
+            if (!taken[i]) {
+              const int rr = qq * p.H + jj;
+              rv[i] = __ldg(p.w + static_cast<int64_t>(tq) * p.H + jj) * rb[rr];
+              if (p.r_out) p.r_out[static_cast<int64_t>(tq) * p.H + jj] = rv[i];
+            }
           }
-          if (bj < p.H && (bj & 31) == lane) taken[bj >> 5] = true;
-        }
-        // selected heads, written in ascending order
-        int before = 0;
+          for (int round = 0; round < p.h; ++round) {
+            float br = -INFINITY;
+            int bj = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < SL; ++i) {
-          const int jj = lane + 32 * i;
-          const bool sel = jj < p.H && taken[i];
-          const uint32_t m = __ballot_sync(0xffffffffu, sel);
-          if (sel)
-            p.heads[static_cast<int64_t>(tq) * p.h + before + __popc(m & ((1u << lane) - 1u))] = jj;
-          before += __popc(m);
+            for (int i = 0; i < SL; ++i)
+              if (!taken[i]) better(br, bj, rv[i], lane + 32 * i);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+              const float orr = __shfl_xor_sync(0xffffffffu, br, off);
+              const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+              better(br, bj, orr, oj);
+            }
+            if (bj < p.H && (bj & 31) == lane) taken[bj >> 5] = true;
+          }
+          // selected heads, written in ascending order
+          int before = 0;
+#pragma unroll
+          for (int i = 0; i < SL; ++i) {
+            const int jj = lane + 32 * i;
+            const bool sel = jj < p.H && taken[i];
+            const uint32_t m = __ballot_sync(0xffffffffu, sel);
+            if (sel)
+              p.heads[static_cast<int64_t>(tq) * p.h + before + __popc(m & ((1u << lane) - 1u))] = jj;
+            before += __popc(m);
+          }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(REMPTY + buf));
       }
-      // r_s is reused by the next row tile
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(ESYNC));
-        ok = mbar_wait(bar(ESYNC), esync & 1, abort_flag, p.ctl);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      ++esync;
     }
   }
 
