@@ -90,9 +90,10 @@ int misa_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
  * dense DSA lightning indexer (Declaracao do Problema).  For FP8 keys the
  * product uses the decoded code and the per-token scale multiplies the dot
  * product before the ReLU.  Entries s > pos(t) are not part of the result:
- * those in a 128-key tile that also holds causal keys are written -inf, the
- * rest are left untouched.  h must be a power of two <= 128; ld >= n_k.
- * Q, K, logits 16-byte aligned.
+ * those in a 128-key tile that also holds causal keys are written -inf (up to
+ * column n_k rounded up to a multiple of 4), the rest are left untouched.  h must be a power of two <= 128; ld >= n_k and a
+ * multiple of 4 (16-byte rows: tiles are written by TMA stores).  Q, K, logits
+ * 16-byte aligned.
  */
 int misa_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
                       const float* k_scale, int kdtype, int n_q, int64_t q_pos0, int64_t n_k,
@@ -144,7 +145,34 @@ int misa_rerank_noalloc(const uint16_t* Q, const float* w, const void* K, const 
                         int kdtype, const int32_t* cand, int kp, int n_q, int64_t q_pos0,
                         int64_t n_k, int H, int d, int k, int32_t* idx, void* stream);
 
-/* Workspace bytes needed by op "topk" or "rerank" for the given sizes (0 if none). */
+/*
+ * Stages 4-5 fused — routed token scoring and top-k in one call (Metodologia
+ * step 2).  Same result as misa_score_tokens followed by misa_topk on its
+ * logits: idx[t, :] = the k tokens s <= pos(t) of largest routed logit, ties to
+ * the lower index, ascending, -1 padded.  Instead of writing all n_q x n_k
+ * logits it scores a 4096-key sample of the prefix 0..q_pos0 first, sets a
+ * per-row threshold from it, stores only the logits at or above the threshold
+ * (a few k per row, flagged in a per-row bit mask) while scoring, and selects
+ * exactly among them.  Rows whose threshold kept fewer than min(k, visible)
+ * logits, or more than max(6144, 3k), are recomputed by the unfused sequence,
+ * so the result is exact for every input.
+ *   logits [n_q, ld]: scratch for the kept logits and the fallback (contents
+ *     unspecified afterwards; ld >= n_k, a multiple of 4, 16-byte aligned).
+ *   ws/ws_bytes: misa_workspace_size("score_topk", n_q, n_k, k, 0) bytes,
+ *     16-byte aligned.  That size is 0 (and the call runs the unfused
+ *     sequence) unless 4096 <= n_k <= 262144 and 1 <= k <= 8192.  The fused
+ *     sequence also needs q_pos0 >= 4095 and h in {4, 8, 16, 32, 64}, else the
+ *     call is unfused.  After a fused call, ws holds n_q + 1 int32 repair flags
+ *     at offset 0: [0] != 0 iff any row took the fallback, [1 + t] for row t.
+ * Shapes and other limits as misa_score_tokens; 0 <= k <= 16384.
+ */
+int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
+                    const float* k_scale, int kdtype, int n_q, int64_t q_pos0, int64_t n_k, int H,
+                    int d, int h, int k, int32_t* idx, float* logits, int64_t ld, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* Workspace bytes needed by op "topk", "rerank" or "score_topk" for the given
+ * sizes (0 if none). */
 size_t misa_workspace_size(const char* op, int n_q, int64_t n_k, int k, int kp);
 
 /* Static text for a misa_status value. */

@@ -44,6 +44,8 @@ _SIGS = {
                            _vp, _vp, _vp, _sz, _vp]),
     "misa_rerank_noalloc": (_int, [_vp, _vp, _vp, _vp, _int, _vp, _int, _int, _i64, _i64, _int,
                                    _int, _int, _vp, _vp]),
+    "misa_score_topk": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _int, _int, _int,
+                               _int, _vp, _vp, _i64, _vp, _sz, _vp]),
     "misa_workspace_size": (_sz, [ctypes.c_char_p, _int, _i64, _int, _int]),
     "misa_status_string": (ctypes.c_char_p, [_int]),
     "misa_last_device_status": (_int, [_vp]),
@@ -132,8 +134,8 @@ def misa_score_tokens(Q, w, heads, K, q_pos0: int, k_scale=None, logits=None, h:
     n_k = K.shape[0]
     if h is None:
         h = heads.shape[1] if heads is not None else H
-    if logits is None:
-        logits = torch.empty((n_q, n_k), dtype=torch.float32, device=Q.device)
+    if logits is None:  # rows padded to 16 bytes (the kernel stores tiles by TMA)
+        logits = torch.empty((n_q, (n_k + 3) // 4 * 4), dtype=torch.float32, device=Q.device)[:, :n_k]
     ld = logits.stride(0) if logits.dim() == 2 else n_k
     st = _lib.misa_score_tokens(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
                                 _ptr(heads, (torch.int32,), "heads"), _ptr(K, name="K"),
@@ -152,6 +154,33 @@ def misa_topk(logits, q_pos0: int, n_k: int, k: int, idx=None, n_q: int | None =
     st = _lib.misa_topk(ctypes.c_void_p(logits.data_ptr()), logits.stride(0), n_q, q_pos0, n_k, k,
                         _ptr(idx, (torch.int32,), "idx"), None, 0, _stream())
     _check("misa_topk", st)
+    return idx
+
+
+def misa_score_topk(Q, w, heads, K, q_pos0: int, k: int, k_scale=None, h: int | None = None,
+                    idx=None, logits=None, ws=None):
+    """Routed scoring and top-k in one call -> idx [n_q, k] int32 (ascending, -1 padded).
+
+    `logits` ([n_q, >= n_k] fp32, rows 16-byte aligned) is the exact fallback's
+    scratch and `ws` the fused path's workspace; both are allocated when absent."""
+    n_q, H, d = Q.shape
+    n_k = K.shape[0]
+    if h is None:
+        h = heads.shape[1] if heads is not None else H
+    if idx is None:
+        idx = torch.empty((n_q, k), dtype=torch.int32, device=Q.device)
+    if logits is None:
+        logits = torch.empty((n_q, (n_k + 3) // 4 * 4), dtype=torch.float32, device=Q.device)
+    ws_bytes = misa_workspace_size("score_topk", n_q, n_k, k, 0)
+    if ws_bytes and (ws is None or ws.numel() * ws.element_size() < ws_bytes):
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    st = _lib.misa_score_topk(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                              _ptr(heads, (torch.int32,), "heads"), _ptr(K, name="K"),
+                              _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K), n_q, q_pos0,
+                              n_k, H, d, h, k, _ptr(idx, (torch.int32,), "idx"),
+                              ctypes.c_void_p(logits.data_ptr()), logits.stride(0),
+                              _ptr(ws, name="ws") if ws_bytes else None, ws_bytes, _stream())
+    _check("misa_score_topk", st)
     return idx
 
 

@@ -58,6 +58,40 @@ bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MISA_OK : MISA_ERR_CUDA; }
 
+// Fused score + top-k: the routed logits of a 32 x 128-key sample of the
+// visible prefix set per-row thresholds; the scoring pass then stores only the
+// logits at or above them (flagged in per-row pass masks) and an exact
+// selection over the flagged logits finishes.
+constexpr int kSampleBlocks = 32;
+constexpr int kSampleKeys = kSampleBlocks * 128;
+constexpr int64_t kFusedMaxKeys = int64_t(1) << 18;  // a 4096-key sample stays representative
+constexpr int kFusedMaxK = 8192;                    // the finish kernel's list fits in shared memory
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+int64_t mask_words(int64_t n_k) { return ((n_k + 31) / 32 + 3) / 4 * 4; }
+
+struct FusedLayout {
+  size_t gate, tau, ks, ks_scale, sample, mask, total;
+  FusedLayout(int n_q, int64_t n_k) {
+    const size_t nq = static_cast<size_t>(n_q);
+    size_t o = 0;
+    gate = o;
+    o += round256((nq + 1) * 4);
+    tau = o;
+    o += round256(nq * 4);
+    ks = o;
+    o += round256(static_cast<size_t>(kSampleKeys) * 256);  // d <= 128 bf16
+    ks_scale = o;
+    o += round256(static_cast<size_t>(kSampleKeys) * 4);
+    sample = o;
+    o += round256(nq * kSampleKeys * 4);
+    mask = o;
+    o += round256(nq * static_cast<size_t>(mask_words(n_k)) * 4);
+    total = o;
+  }
+};
+
 }  // namespace
 
 int* device_status_word() { return status_ptr(); }
@@ -145,7 +179,7 @@ int misa_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads, c
     return MISA_ERR_INVALID_ARG;
   if (heads && !aligned4(heads)) return MISA_ERR_INVALID_ARG;
   if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || H < 1 || h < 1 || h > H ||
-      ld < n_k)
+      ld < n_k || ld % 4 != 0 || !aligned16(logits))
     return MISA_ERR_INVALID_ARG;
   if (!heads && h != H) return MISA_ERR_INVALID_ARG;
   if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
@@ -205,12 +239,99 @@ int misa_rerank(const uint16_t* Q, const float* w, const void* K, const float* k
   return cuda_status(launch_topk(full, kp, n_q, q_pos0, n_k, kp, cand, k, idx, ctl, s));
 }
 
+int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
+                    const float* k_scale, int kdtype, int n_q, int64_t q_pos0, int64_t n_k, int H,
+                    int d, int h, int k, int32_t* idx, float* logits, int64_t ld, void* ws,
+                    size_t ws_bytes, void* stream) {
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !K || !aligned16(K) || !logits ||
+      !aligned16(logits) || (k > 0 && (!idx || !aligned4(idx))))
+    return MISA_ERR_INVALID_ARG;
+  if (heads && !aligned4(heads)) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || H < 1 || h < 1 || h > H ||
+      ld < n_k || ld % 4 != 0 || k < 0 || k > 16384)
+    return MISA_ERR_INVALID_ARG;
+  if (!heads && h != H) return MISA_ERR_INVALID_ARG;
+  if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
+  if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
+  if (!good_d(d) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
+  if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
+  if (n_q == 0 || k == 0) return MISA_OK;
+  const size_t need = misa_workspace_size("score_topk", n_q, n_k, k, 0);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return MISA_ERR_WORKSPACE;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  const cudaStream_t s = as_stream(stream);
+  const bool fp8 = kdtype == MISA_K_FP8E4M3;
+  ScoreLaunch a{};
+  a.Q = Q;
+  a.w = w;
+  a.heads = heads;
+  a.K = K;
+  a.k_scale = k_scale;
+  a.fp8 = fp8;
+  a.n_q = n_q;
+  a.q_pos0 = q_pos0;
+  a.n_k = n_k;
+  a.H = H;
+  a.d = d;
+  a.h = h;
+  a.logits = logits;
+  a.ld = ld;
+  const bool fused = need > 0 && q_pos0 + 1 >= kSampleKeys && score_select_supported(h);
+  if (!fused) {  // unfused: every logit, then the selection
+    cudaError_t e = launch_score(a, ctl, s);
+    if (e != cudaSuccess) return MISA_ERR_CUDA;
+    return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, 0, nullptr, k, idx, ctl, s));
+  }
+  const FusedLayout L(n_q, n_k);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* gate = reinterpret_cast<int*>(base + L.gate);
+  float* tau = reinterpret_cast<float*>(base + L.tau);
+  void* Ks = base + L.ks;
+  float* ks_scale = reinterpret_cast<float*>(base + L.ks_scale);
+  float* sample = reinterpret_cast<float*>(base + L.sample);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(base + L.mask);
+  const int64_t mld = mask_words(n_k);
+  const int row_bytes = fp8 ? d : 2 * d;
+  cudaError_t e = launch_gather_sample(K, fp8 ? k_scale : nullptr, row_bytes, q_pos0 + 1,
+                                       kSampleBlocks, Ks, fp8 ? ks_scale : nullptr, s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  ScoreLaunch sa = a;  // the sample: every sampled key is visible to every query
+  sa.K = Ks;
+  sa.k_scale = fp8 ? ks_scale : nullptr;
+  sa.q_pos0 = kSampleKeys - 1;
+  sa.n_k = kSampleKeys;
+  sa.logits = sample;
+  sa.ld = kSampleKeys;
+  if ((e = launch_score(sa, ctl, s)) != cudaSuccess) return MISA_ERR_CUDA;
+  if ((e = launch_fused_tau(sample, kSampleKeys, kSampleKeys, n_q, q_pos0, n_k, k, tau, gate, s)) !=
+      cudaSuccess)
+    return MISA_ERR_CUDA;
+  ScoreLaunch se = a;  // select mode
+  se.tau = tau;
+  se.mask = mask;
+  se.mask_ld = mld;
+  if ((e = launch_score(se, ctl, s)) != cudaSuccess) return MISA_ERR_CUDA;
+  if ((e = launch_fused_finish(logits, ld, mask, mld, n_q, q_pos0, n_k, k, idx, gate, s)) !=
+      cudaSuccess)
+    return MISA_ERR_CUDA;
+  // exact fallback for the rows the thresholds missed (a no-op launch when none)
+  ScoreLaunch ra = a;
+  ra.gate = gate;
+  if ((e = launch_score(ra, ctl, s)) != cudaSuccess) return MISA_ERR_CUDA;
+  return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, 0, nullptr, k, idx, ctl, s, gate));
+}
+
 size_t misa_workspace_size(const char* op, int n_q, int64_t n_k, int k, int kp) {
-  (void)n_k;
-  (void)k;
   if (!op || n_q <= 0) return 0;
   if (std::strcmp(op, "rerank") == 0 && kp > 0)
     return static_cast<size_t>(n_q) * static_cast<size_t>(kp) * sizeof(float);
+  if (std::strcmp(op, "score_topk") == 0) {
+    // fused only where the sample lies inside every row's prefix and the
+    // position bitmap fits; 0 selects the unfused sequence
+    if (k <= 0 || k > kFusedMaxK || n_k > kFusedMaxKeys || n_k < kSampleKeys) return 0;
+    return FusedLayout(n_q, n_k).total;
+  }
   return 0;
 }
 

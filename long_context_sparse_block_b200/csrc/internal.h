@@ -22,6 +22,32 @@ cudaError_t launch_route_heads(const uint16_t* Q, const float* w, const uint16_t
                                int n_q, int64_t q_pos0, int64_t n_k, int H, int d, int B, int h,
                                int32_t* heads, float* r_out, const DevCtl& ctl, cudaStream_t s);
 
+// Score kernel launch description: store mode writes fused logits (logits,
+// ld); select mode (tau != nullptr) keeps logits >= tau[t] in per-row
+// candidate lists instead.  gate (nullable): do nothing unless *gate != 0.
+struct ScoreLaunch {
+  const uint16_t* Q;
+  const float* w;
+  const int32_t* heads;
+  const void* K;
+  const float* k_scale;
+  bool fp8;
+  int n_q;
+  int64_t q_pos0;
+  int64_t n_k;
+  int H;
+  int d;
+  int h;
+  float* logits;
+  int64_t ld;
+  const float* tau;       // select mode: per-row thresholds (else nullptr)
+  uint32_t* mask;         // select mode: [n_q][mask_ld] pass bits
+  int64_t mask_ld;
+  const int* gate;        // nullable: launch does nothing unless *gate != 0
+};
+cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s);
+bool score_select_supported(int h);
+
 cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads,
                                 const void* K, const float* k_scale, bool fp8, int n_q,
                                 int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
@@ -33,7 +59,18 @@ cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t
 // cand[t*row_len + i] for the selected positions i.
 cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k,
                         int row_len, const int32_t* cand, int k, int32_t* idx,
-                        const DevCtl& ctl, cudaStream_t s);
+                        const DevCtl& ctl, cudaStream_t s, const int* gate = nullptr);
+
+// Fused top-k helpers (topk.cu): sample gather, per-row thresholds from the
+// scored sample, and the exact selection over the select-mode candidates.
+int sample_block_keys();
+cudaError_t launch_gather_sample(const void* K, const float* k_scale, int row_bytes, int64_t span,
+                                 int n_blocks, void* Ks, float* ks_scale, cudaStream_t s);
+cudaError_t launch_fused_tau(const float* sample, int64_t lds, int n_s, int n_q, int64_t q_pos0,
+                             int64_t n_k, int k, float* tau, int* gate, cudaStream_t s);
+cudaError_t launch_fused_finish(const float* logits, int64_t ld, const uint32_t* mask,
+                                int64_t mask_ld, int n_q, int64_t q_pos0, int64_t n_k, int k,
+                                int32_t* idx, int* gate, cudaStream_t s);
 
 // All-head scores of candidate keys: full[t*ldf + i] (-inf where ignored).
 cudaError_t launch_rerank_scores(const uint16_t* Q, const float* w, const void* K,

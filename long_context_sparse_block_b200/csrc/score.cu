@@ -22,7 +22,9 @@
 //              TMA into a STAGES-deep ring;
 //   warp 1     allocates TMEM (512 columns = two 256-column accumulators) and
 //              issues tcgen05.mma from one thread;
-//   warps 2-   epilogue, four warps per TMEM lane quadrant each owning 64 of
+//   warp 2     issues one TMA store per tile of the logits the epilogue staged
+//              in shared memory (double-buffered);
+//   warps 3-   epilogue, four warps per TMEM lane quadrant each owning 64 of
 //              the 256 columns (two warps owning 128 when h = 128): one
 //              tcgen05.ld of its columns, the accumulator released right after
 //              the load lands, then the fused ReLU * w head-sum (packed fp32
@@ -40,19 +42,24 @@ namespace {
 constexpr int kTileKeys = 128;   // MMA M
 constexpr int kCols = 256;       // MMA N: (query, head) columns per group
 // epilogue warps: 4 per TMEM lane quadrant (64 columns each) when a query's h
-// columns fit in 64, else 2 per quadrant (128 columns each).  FP8 keys add 2
-// converter warps (e4m3 -> bf16 into the swizzled key tile) before them.
-template <int HT, bool FP8>
+// columns fit in 64, else 2 per quadrant (128 columns each).  Warp 2 issues the
+// TMA stores of the staged logits; FP8 keys add a converter warp (e4m3 -> bf16
+// into the swizzled key tile) before the epilogue warps.
+template <int HT, bool FP8, bool SEL = false>
 struct Epi {
   static constexpr int WARPS = HT <= 64 ? 16 : 8;
   static constexpr int COLS = kCols / (WARPS / 4);
-  static constexpr int CONV = FP8 ? 2 : 0;
-  static constexpr int BASE = 2 + CONV;  // first epilogue warp
+  static constexpr int CONV = FP8 ? 1 : 0;
+  static constexpr int BASE = 3 + CONV;  // first epilogue warp
   static constexpr int THREADS = 32 * (BASE + WARPS);
+  // a block's warps are spread over the 4 SM sub-partitions (16K registers
+  // each): the largest per-thread count that still lets THREADS threads launch
+  static constexpr int MAXREG_RAW = 16384 / (((THREADS / 32) + 3) / 4 * 32) / 8 * 8;
+  static constexpr int MAXREG = MAXREG_RAW > 255 ? 255 : MAXREG_RAW;
 };
 constexpr uint64_t kDrainNs = 2000000;  // 2 ms
 
-template <int D, int HT, bool FP8>
+template <int D, int HT, bool FP8, bool SEL = false>
 struct ScoreLayout {
   static constexpr int ROWB = D >= 64 ? 128 : 64;  // bytes per row of one swizzle chunk
   static constexpr int KCH = D * 2 / ROWB;         // swizzle chunks along d
@@ -60,13 +67,24 @@ struct ScoreLayout {
   static constexpr int A_BYTES = kTileKeys * D * 2;
   static constexpr int B_CHUNK = kCols * ROWB;
   static constexpr int B_BYTES = kCols * D * 2;
-  static constexpr int STAGES = D == 128 ? 4 : 8;
+  // fused logits of a tile are staged in shared memory ([QG queries][128 keys]
+  // fp32, double-buffered) and written by one TMA store (h >= 4)
+  static constexpr bool TMA_STORE = HT >= 4 && !SEL;
+  static constexpr int QG = kCols / HT;
+  static constexpr int STG_BYTES = TMA_STORE ? QG * kTileKeys * 4 : 0;
+  static constexpr int SMEM_BUDGET = 227 * 1024 - 1024 - 8 * 1024;  // minus alignment, small data
+  static constexpr int STAGES_FIT = (SMEM_BUDGET - B_BYTES - 2 * STG_BYTES) / A_BYTES;
+  static constexpr int STAGES_MAX = D == 128 ? 4 : 8;
+  static constexpr int STAGES = STAGES_FIT < STAGES_MAX ? STAGES_FIT : STAGES_MAX;
+  static_assert(STAGES >= 2, "key ring needs two stages");
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_W = OFF_B + B_BYTES;         // per epilogue warp: its columns' w
-  static constexpr int OFF_HEADS = OFF_W + Epi<HT, FP8>::WARPS * Epi<HT, FP8>::COLS * 4;  // producer
+  static constexpr int OFF_STG = OFF_B + B_BYTES;       // 2 staging buffers (1024-aligned)
+  static constexpr int OFF_W = OFF_STG + 2 * STG_BYTES;  // per epilogue warp: its columns' w
+  static constexpr int OFF_TAU = OFF_W + Epi<HT, FP8>::WARPS * Epi<HT, FP8>::COLS * 4;  // select: tau
+  static constexpr int OFF_HEADS = OFF_TAU + (SEL ? Epi<HT, FP8>::WARPS * 16 * 4 : 0);  // producer
   static constexpr int OFF_BAR = OFF_HEADS + kCols * 4;
-  static constexpr int NBAR = 2 * STAGES + 6;
+  static constexpr int NBAR = 2 * STAGES + 10;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;            // room to align the base to 1024
@@ -86,6 +104,13 @@ struct ScoreParams {
   int H;
   int64_t total_tiles;
   DevCtl ctl;
+  // select mode (fused top-k): only logits >= tau[t] are stored, and flagged
+  const float* tau;
+  uint32_t* mask;        // [n_q][mask_ld] pass bits, bit s%32 of word s/32
+  int64_t mask_ld;
+  // repair launch: nothing unless gate[0] != 0, then only the query groups
+  // holding a row t with gate[1 + t] != 0
+  const int* gate;
 };
 
 // Flattened schedule over (group g, key tile kt): each role of a CTA walks the
@@ -97,7 +122,8 @@ struct Sched {
 
   __device__ static int64_t tiles_of(const ScoreParams& p, int g) {
     const int t_last = min((g + 1) * QG, p.n_q) - 1;
-    return (p.q_pos0 + t_last) / kTileKeys + 1;
+    const int64_t last = min(p.q_pos0 + t_last, p.n_k - 1);  // queries may see every key
+    return last / kTileKeys + 1;
   }
   __device__ void init(const ScoreParams& p) {
     const int64_t start = p.total_tiles * blockIdx.x / gridDim.x;
@@ -118,6 +144,27 @@ struct Sched {
       acc += n;
       ++g;
     }
+    skip_dead(p);
+  }
+  // repair launches (gate set) score only the groups holding a flagged row
+  __device__ static bool live(const ScoreParams& p, int g) {
+    if (!p.gate) return true;
+    const int t1 = min((g + 1) * QG, p.n_q);
+    for (int t = g * QG; t < t1; ++t)
+      if (p.gate[1 + t]) return true;
+    return false;
+  }
+  __device__ void skip_dead(const ScoreParams& p) {
+    while (left > 0 && !live(p, g)) {
+      left -= nt - kt;
+      if (left <= 0) {
+        left = 0;
+        break;
+      }
+      ++g;
+      kt = 0;
+      nt = tiles_of(p, g);
+    }
   }
   __device__ bool last_of_group() const { return kt == nt - 1 || left == 1; }
   __device__ void next(const ScoreParams& p) {
@@ -126,14 +173,18 @@ struct Sched {
       ++g;
       kt = 0;
       nt = tiles_of(p, g);
+      skip_dead(p);
     }
   }
 };
 
-template <int D, int HT, bool FP8>
-__global__ void __launch_bounds__(Epi<HT, FP8>::THREADS, 1)
-score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams p) {
-  using L = ScoreLayout<D, HT, FP8>;
+template <int D, int HT, bool FP8, bool SEL>
+__global__ void __maxnreg__((Epi<HT, FP8>::MAXREG))
+score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap lmap,
+                    const ScoreParams p) {
+  using L = ScoreLayout<D, HT, FP8, SEL>;
+  static_assert(!SEL || HT >= 4, "select mode needs h >= 4");
+  if (p.gate && *p.gate == 0) return;  // repair launch with nothing to repair
   constexpr int EW = Epi<HT, FP8>::WARPS;
   constexpr int EC = Epi<HT, FP8>::COLS;
   constexpr int CONV = Epi<HT, FP8>::CONV;
@@ -146,7 +197,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   auto bar = [&](int i) { return smem_u32(bars + i); };
   const int FULL = 0, EMPTY = L::STAGES, BFULL = 2 * L::STAGES, BEMPTY = BFULL + 1,
-            ACCFULL = BFULL + 2, ACCEMPTY = BFULL + 4;
+            ACCFULL = BFULL + 2, ACCEMPTY = BFULL + 4, SFULL = BFULL + 6, SFREE = BFULL + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -161,10 +212,13 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(ACCFULL + i), 1);
       mbar_init(bar(ACCEMPTY + i), EW);
+      mbar_init(bar(SFULL + i), EW);
+      mbar_init(bar(SFREE + i), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
     if (!FP8) tma_prefetch_desc(&kmap);
+    if (L::TMA_STORE) tma_prefetch_desc(&lmap);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -282,11 +336,32 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
         accph ^= 1;
       }
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ logit store issuer
+    if constexpr (L::TMA_STORE) {
+      if (lane == 0) {
+        Sched<QG> it;
+        it.init(p);
+        uint32_t tcount = 0;
+        for (; it.left > 0; it.next(p), ++tcount) {
+          const uint32_t buf = tcount & 1;
+          if (!mbar_wait(bar(SFULL + buf), (tcount >> 1) & 1, abort_flag, p.ctl)) break;
+          tma_store_2d(&lmap, smem_u32(smem + L::OFF_STG) + buf * L::STG_BYTES,
+                       static_cast<int>(it.kt * kTileKeys),
+                       static_cast<int>(static_cast<int64_t>(it.g) * QG));
+          bulk_commit();
+          bulk_wait_read<1>();  // the previous tile's store has read its buffer
+          if (tcount > 0) mbar_arrive(bar(SFREE + (buf ^ 1)));
+        }
+        bulk_wait_all();
+      }
+      __syncwarp();
+    }
   } else if (warp < Epi<HT, FP8>::BASE) {
     // ------------------------------------------------------------ FP8 key converters
     // e4m3 key rows -> bf16 (exact) straight into the swizzled key tile
     if constexpr (FP8) {
-      const int ct = threadIdx.x - 64;  // 0 .. 32*CONV-1
+      const int ct = threadIdx.x - 96;  // 0 .. 32*CONV-1
       constexpr int U8 = D / 16;        // 16-byte e4m3 units per key row
       constexpr int UPC = L::ROWB / 16; // bf16 16-byte units per swizzle-chunk row
       Sched<QG> it;
@@ -335,9 +410,11 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
     Sched<QG> it;
     it.init(p);
     int acc = 0;
-    uint32_t accph = 0;
+    uint32_t accph = 0, tcount = 0;
     int prev_g = -1;
-    for (; it.left > 0; it.next(p)) {
+    float* tau_s = reinterpret_cast<float*>(smem + L::OFF_TAU) + e * 16;  // select: thresholds
+    (void)tau_s;
+    for (; it.left > 0; it.next(p), ++tcount) {
       if (it.g != prev_g) {
         for (int i = lane; i < EC; i += 32) {
           const int col = part * EC + i;
@@ -349,6 +426,12 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
             wv = __ldg(p.w + static_cast<int64_t>(t) * p.H + j);
           }
           w_s[i] = wv;
+        }
+        if constexpr (SEL) {
+          for (int qq = lane; qq < QPW; qq += 32) {
+            const int64_t t = static_cast<int64_t>(it.g) * QG + part * QPW + qq;
+            tau_s[qq] = t < p.n_q ? __ldg(p.tau + t) : INFINITY;
+          }
         }
         __syncwarp();
         prev_g = it.g;
@@ -377,6 +460,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
       const bool s_ok = s < p.n_k;
       const int64_t tq0 = static_cast<int64_t>(it.g) * QG + part * QPW;
       float* dst = p.logits + tq0 * p.ld + s;
+      (void)dst;
       if constexpr (HT >= 4) {
         // every head-sum first (the shared-memory weight loads never wait
         // behind a global store), then the stores
@@ -401,12 +485,47 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
 #pragma unroll
           for (int qq = 0; qq < QPW; ++qq) sums[qq] *= ks;
         }
+        if constexpr (SEL) {
+          // fused top-k: a logit at or above its row's threshold is stored in
+          // place and flagged in the row's pass mask (one word per 32 keys);
+          // the others are neither stored nor flagged
+          const int64_t cut64 = s - p.q_pos0 - tq0;  // query qq is causal for key s iff qq >= cut
+          const int cut = static_cast<int>(cut64 < 0 ? 0 : (cut64 > QPW ? QPW : cut64));
+          const int64_t rows_left = p.n_q - tq0;
+          const int q_end = static_cast<int>(rows_left < QPW ? rows_left : QPW);
+          const uint32_t valid = s_ok ? (((1u << q_end) - 1u) & ~((1u << cut) - 1u)) : 0u;
+          uint32_t mine = 0u;  // lane qq: the mask word of query qq
 #pragma unroll
-        for (int qq = 0; qq < QPW; ++qq) {
-          const int64_t t = tq0 + qq;
-          if (t < p.n_q && s_ok) *dst = (s <= p.q_pos0 + t) ? sums[qq] : -INFINITY;
-          dst += p.ld;
+          for (int qq = 0; qq < QPW; ++qq) {
+            const bool pass = ((valid >> qq) & 1u) && sums[qq] >= tau_s[qq];
+            const uint32_t m = __ballot_sync(0xffffffffu, pass);
+            if (lane == qq) mine = m;
+            if (pass) *dst = sums[qq];
+            dst += p.ld;
+          }
+          if (lane < q_end)
+            p.mask[(tq0 + lane) * p.mask_ld + it.kt * (kTileKeys / 32) + quad] = mine;
+        } else {
+        // stage [query][key] in shared memory, then one TMA store per tile
+          // (rows past n_q and keys past n_k fall outside the map and are not written)
+          const uint32_t buf = tcount & 1;
+          const uint32_t sbuf = smem_u32(smem + L::OFF_STG) + buf * L::STG_BYTES;
+          bool sok = true;
+          if (lane == 0) sok = mbar_wait(bar(SFREE + buf), ((tcount >> 1) & 1) ^ 1, abort_flag, p.ctl);
+          if (!__shfl_sync(0xffffffffu, sok, 0)) break;
+          const int64_t cut64 = s - p.q_pos0 - tq0;  // query qq is causal for key s iff qq >= cut
+          const int cut = static_cast<int>(cut64 < 0 ? 0 : (cut64 > QPW ? QPW : cut64));
+#pragma unroll
+          for (int qq = 0; qq < QPW; ++qq) {
+            const float val = qq >= cut ? sums[qq] : -INFINITY;
+            const uint32_t a = sbuf + static_cast<uint32_t>(((part * QPW + qq) * kTileKeys + quad * 32 + lane) * 4);
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(val) : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(SFULL + buf));
         }
+        (void)s_ok;
       } else {
 #pragma unroll
         for (int qq = 0; qq < QPW; ++qq) {
@@ -434,77 +553,119 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams 
   }
 }
 
-template <int D, int HT, bool FP8>
-cudaError_t launch_dh(const ScoreParams& p, const CUtensorMap& map, cudaStream_t s) {
-  using L = ScoreLayout<D, HT, FP8>;
-  auto kern = score_tokens_kernel<D, HT, FP8>;
-  static bool attr_set = false;  // per process; the attribute is per device but idempotent
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+template <int D, int HT, bool FP8, bool SEL>
+cudaError_t launch_dhs(const ScoreParams& p, const CUtensorMap& map, cudaStream_t s) {
+  using L = ScoreLayout<D, HT, FP8, SEL>;
+  // fused-logit store map: [n_q rows][n_k keys] fp32 with row pitch ld, box 128 keys x QG queries
+  CUtensorMap lmap;
+  std::memset(&lmap, 0, sizeof lmap);
+  if (L::TMA_STORE) {
+    // the store covers whole 16-byte units: keys up to n_k rounded up to 4 (< ld)
+    const uint64_t dims[2] = {static_cast<uint64_t>((p.n_k + 3) / 4 * 4), static_cast<uint64_t>(p.n_q)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(p.ld) * 4};
+    const uint32_t box[2] = {static_cast<uint32_t>(kTileKeys), static_cast<uint32_t>(L::QG)};
+    if (encode_tensor_map(&lmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.logits, dims, strides, box,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
   }
+  auto kern = score_tokens_kernel<D, HT, FP8, SEL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
   const int64_t grid = std::min<int64_t>(sm_count(), p.total_tiles);
   if (grid <= 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), Epi<HT, FP8>::THREADS, L::ALLOC, s>>>(map, p);
+  kern<<<static_cast<unsigned>(grid), Epi<HT, FP8>::THREADS, L::ALLOC, s>>>(map, lmap, p);
   return cudaGetLastError();
 }
 
 template <int D, bool FP8>
-cudaError_t launch_d(const ScoreParams& p, int h, const CUtensorMap& map, cudaStream_t s) {
+cudaError_t launch_d(const ScoreParams& p, int h, bool sel, const CUtensorMap& map, cudaStream_t s) {
+  if (sel) {
+    switch (h) {
+      case 4: return launch_dhs<D, 4, FP8, true>(p, map, s);
+      case 8: return launch_dhs<D, 8, FP8, true>(p, map, s);
+      case 16: return launch_dhs<D, 16, FP8, true>(p, map, s);
+      case 32: return launch_dhs<D, 32, FP8, true>(p, map, s);
+      case 64: return launch_dhs<D, 64, FP8, true>(p, map, s);
+    }
+    return cudaErrorNotSupported;
+  }
   switch (h) {
-    case 1: return launch_dh<D, 1, FP8>(p, map, s);
-    case 2: return launch_dh<D, 2, FP8>(p, map, s);
-    case 4: return launch_dh<D, 4, FP8>(p, map, s);
-    case 8: return launch_dh<D, 8, FP8>(p, map, s);
-    case 16: return launch_dh<D, 16, FP8>(p, map, s);
-    case 32: return launch_dh<D, 32, FP8>(p, map, s);
-    case 64: return launch_dh<D, 64, FP8>(p, map, s);
-    case 128: return launch_dh<D, 128, FP8>(p, map, s);
+    case 1: return launch_dhs<D, 1, FP8, false>(p, map, s);
+    case 2: return launch_dhs<D, 2, FP8, false>(p, map, s);
+    case 4: return launch_dhs<D, 4, FP8, false>(p, map, s);
+    case 8: return launch_dhs<D, 8, FP8, false>(p, map, s);
+    case 16: return launch_dhs<D, 16, FP8, false>(p, map, s);
+    case 32: return launch_dhs<D, 32, FP8, false>(p, map, s);
+    case 64: return launch_dhs<D, 64, FP8, false>(p, map, s);
+    case 128: return launch_dhs<D, 128, FP8, false>(p, map, s);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
+bool score_select_supported(int h) { return h == 4 || h == 8 || h == 16 || h == 32 || h == 64; }
+
+cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s) {
+  if (a.n_q <= 0) return cudaSuccess;
+  const bool sel = a.tau != nullptr;
+  if (sel && !score_select_supported(a.h)) return cudaErrorNotSupported;
+  const int QG = kCols / a.h;
+  const int n_groups = (a.n_q + QG - 1) / QG;
+  int64_t total = 0;
+  for (int g = 0; g < n_groups; ++g) {
+    const int t_last = std::min((g + 1) * QG, a.n_q) - 1;
+    total += std::min<int64_t>(a.q_pos0 + t_last, a.n_k - 1) / kTileKeys + 1;
+  }
+  ScoreParams p{a.Q, a.w, a.heads, a.k_scale, static_cast<const uint8_t*>(a.K), a.logits, a.ld,
+                a.n_q, a.q_pos0, a.n_k, a.H, total, ctl, a.tau, a.mask, a.mask_ld,
+                a.gate};
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof map);
+  if (a.fp8) {  // converter warps read the e4m3 keys; no key tensor map
+    switch (a.d) {
+      case 32: return launch_d<32, true>(p, a.h, sel, map, s);
+      case 64: return launch_d<64, true>(p, a.h, sel, map, s);
+      case 128: return launch_d<128, true>(p, a.h, sel, map, s);
+    }
+    return cudaErrorInvalidValue;
+  }
+  const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.n_k)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(a.d) * 2};
+  const int rowb = a.d >= 64 ? 128 : 64;
+  const uint32_t box[2] = {static_cast<uint32_t>(rowb / 2), static_cast<uint32_t>(kTileKeys)};
+  if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.K, dims, strides, box,
+                        rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) !=
+      CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  switch (a.d) {
+    case 32: return launch_d<32, false>(p, a.h, sel, map, s);
+    case 64: return launch_d<64, false>(p, a.h, sel, map, s);
+    case 128: return launch_d<128, false>(p, a.h, sel, map, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads,
                                 const void* K, const float* k_scale, bool fp8, int n_q,
                                 int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
                                 int64_t ld, const DevCtl& ctl, cudaStream_t s) {
-  if (n_q <= 0) return cudaSuccess;
-  const int QG = kCols / h;
-  const int n_groups = (n_q + QG - 1) / QG;
-  int64_t total = 0;
-  for (int g = 0; g < n_groups; ++g) {
-    const int t_last = std::min((g + 1) * QG, n_q) - 1;
-    total += (q_pos0 + t_last) / kTileKeys + 1;
-  }
-  ScoreParams p{Q, w, heads, k_scale, static_cast<const uint8_t*>(K), logits, ld, n_q, q_pos0, n_k,
-                H, total, ctl};
-  CUtensorMap map;
-  if (fp8) {
-    std::memset(&map, 0, sizeof map);  // unused: converter warps read the e4m3 keys
-    switch (d) {
-      case 32: return launch_d<32, true>(p, h, map, s);
-      case 64: return launch_d<64, true>(p, h, map, s);
-      case 128: return launch_d<128, true>(p, h, map, s);
-    }
-    return cudaErrorInvalidValue;
-  }
-  const uint64_t dims[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_k)};
-  const uint64_t strides[1] = {static_cast<uint64_t>(d) * 2};
-  const int rowb = d >= 64 ? 128 : 64;
-  const uint32_t box[2] = {static_cast<uint32_t>(rowb / 2), static_cast<uint32_t>(kTileKeys)};
-  if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, dims, strides, box,
-                        rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) !=
-      CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  switch (d) {
-    case 32: return launch_d<32, false>(p, h, map, s);
-    case 64: return launch_d<64, false>(p, h, map, s);
-    case 128: return launch_d<128, false>(p, h, map, s);
-  }
-  return cudaErrorInvalidValue;
+  ScoreLaunch a{};
+  a.Q = Q;
+  a.w = w;
+  a.heads = heads;
+  a.K = K;
+  a.k_scale = k_scale;
+  a.fp8 = fp8;
+  a.n_q = n_q;
+  a.q_pos0 = q_pos0;
+  a.n_k = n_k;
+  a.H = H;
+  a.d = d;
+  a.h = h;
+  a.logits = logits;
+  a.ld = ld;
+  return launch_score(a, ctl, s);
 }
 
 }  // namespace misa

@@ -60,6 +60,7 @@ struct TopkParams {
   int32_t* idx;
   int cap;               // shared-memory list capacity (entries)
   DevCtl ctl;
+  const int* gate;       // nullable: row t is done unless gate[1 + t] != 0
 };
 
 __device__ __forceinline__ uint32_t f2key(float f) {
@@ -327,26 +328,21 @@ __device__ void bitonic_sort_asc(uint32_t* buf, uint32_t n) {
 }
 
 // Emits, in ascending order, the positions whose bits are set in bitmap[0..words)
-// to out slots 0.. and pads the rest of the k slots with -1.
+// to out slots 0.. and pads the rest of the k slots with -1.  Each thread owns a
+// contiguous run of words; a block scan gives every run its first slot.
 __device__ void emit_bitmap(const uint32_t* bitmap, uint32_t words, const OutEmit& out,
                             SmemCtl& sc) {
-  constexpr int PER = kBins1 / kTopkThreads;  // words per thread (8)
-  uint32_t wv[PER], c = 0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const uint32_t wi = threadIdx.x * PER + i;
-    wv[i] = wi < words ? bitmap[wi] : 0u;
-    c += __popc(wv[i]);
-  }
+  const uint32_t per = (words + kTopkThreads - 1) / kTopkThreads;
+  const uint32_t w0 = threadIdx.x * per, w1 = min(w0 + per, words);
+  uint32_t c = 0;
+  for (uint32_t i = w0; i < w1; ++i) c += __popc(bitmap[i]);
   uint32_t total;
   uint32_t slot = block_excl_scan(c, sc, total);
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    uint32_t m = wv[i];
-    const uint32_t base = (threadIdx.x * PER + i) * 32u;
+  for (uint32_t i = w0; i < w1; ++i) {
+    uint32_t m = bitmap[i];
     while (m) {
       const uint32_t b = __ffs(m) - 1u;
-      out(slot++, 0u, base + b);
+      out(slot++, 0u, i * 32u + b);
       m &= m - 1u;
     }
   }
@@ -524,6 +520,7 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
 
 __global__ void __launch_bounds__(kTopkThreads, kCtasPerSm)
 topk_kernel(const TopkParams p) {
+  if (p.gate && p.gate[1 + blockIdx.x] == 0) return;  // row needs no repair
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
   SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
@@ -602,11 +599,162 @@ topk_kernel(const TopkParams p) {
   for (uint32_t i = min(kept, k) + threadIdx.x; i < k; i += kTopkThreads) out.out[i] = -1;
 }
 
+// ---------------------------------------------------------------- fused top-k
+// The scoring kernel in select mode keeps, per row, only the logits at or above
+// a threshold tau; the kernels below choose tau from a scored sample of the
+// row's visible keys and then take the exact top-k among the kept candidates.
+
+constexpr double kFusedMargin = 1.6;  // ~1.6 k candidates expected above tau
+constexpr int kSampleBlock = 128;     // keys per contiguous sample block
+
+// Copies the keys of n_blocks contiguous 128-key blocks, evenly spaced over
+// [0, span), into a dense sample (and their FP8 scales when given).
+__global__ void __launch_bounds__(256)
+gather_sample_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scale,
+                     int row_bytes, int64_t span, int n_blocks, uint8_t* __restrict__ Ks,
+                     float* __restrict__ ks_scale) {
+  const int b = blockIdx.x;
+  const int64_t start = n_blocks > 1 ? (span - kSampleBlock) * b / (n_blocks - 1) : 0;
+  const int units = kSampleBlock * row_bytes / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(K + start * row_bytes);
+  uint4* dst = reinterpret_cast<uint4*>(Ks + static_cast<int64_t>(b) * kSampleBlock * row_bytes);
+  for (int i = threadIdx.x; i < units; i += blockDim.x) dst[i] = __ldg(src + i);
+  if (k_scale)
+    for (int i = threadIdx.x; i < kSampleBlock; i += blockDim.x)
+      ks_scale[b * kSampleBlock + i] = __ldg(k_scale + start + i);
+}
+
+// Per row: tau[t] = lower edge of the 22-bit key bin holding the m-th largest
+// sampled logit, m ~ 1.6 k * n_s / visible(t) (or -inf: keep every visible key).
+// Also zeroes the row's repair flag gate[1 + t] and (block 0) the any-row flag
+// gate[0].
+__global__ void __launch_bounds__(kTopkThreads)
+fused_tau_kernel(const float* __restrict__ sample, int64_t lds, int n_s, int64_t q_pos0,
+                 int64_t n_k, int k, float* __restrict__ tau, int* __restrict__ gate) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
+  const int t = blockIdx.x;
+  if (threadIdx.x == 0) {
+    gate[1 + t] = 0;
+    if (t == 0) gate[0] = 0;
+  }
+  const int64_t visible = min(q_pos0 + t + 1, n_k);
+  const float* row = sample + static_cast<int64_t>(t) * lds;
+  uint32_t c = 0;
+  for (int i = threadIdx.x; i < n_s; i += kTopkThreads) {
+    keys[i] = f2key(__ldg(row + i));
+    c += keys[i] != 0u;
+  }
+  uint32_t present;
+  block_excl_scan(c, sc, present);  // (also orders the key writes before the reads below)
+  const uint32_t m = static_cast<uint32_t>(kFusedMargin * k * static_cast<double>(n_s) /
+                                           static_cast<double>(visible)) + 16u;
+  float tf = -INFINITY;
+  if (m <= present) {
+    for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_s; i += kTopkThreads)
+      if (keys[i] != 0u) atomicAdd(&hist[keys[i] >> 20], 1u);
+    __syncthreads();
+    find_bin<kBins1>(hist, m, sc);
+    const uint32_t b1 = sc.res[0], above1 = sc.res[1];
+    __syncthreads();
+    const ListSrc ls{keys, keys, static_cast<int64_t>(n_s)};
+    digit_hist(ls, 20, b1, 10, hist);
+    find_bin<1024>(hist, m - above1, sc);
+    const uint32_t tk = (b1 << 20) | (sc.res[0] << 10);  // >= every real key's bin floor
+    const uint32_t bits = (tk & 0x80000000u) ? (tk & 0x7FFFFFFFu) : ~tk;  // key -> float bits
+    tf = __uint_as_float(bits);
+  }
+  if (threadIdx.x == 0) tau[t] = tf;
+}
+
+// Per row: the exact top-k among the logits the select-mode scoring kept (the
+// bits of the row's pass mask; their values stored in place).  They hold the
+// whole top-k whenever at least min(k, visible) of them passed.  Rows short of
+// that, or with more than list_cap kept, raise their repair flag (and the
+// any-row flag gate[0]) and write nothing.
+__global__ void __launch_bounds__(kTopkThreads)
+fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t* __restrict__ mask,
+                    int64_t mask_ld, int64_t q_pos0, int64_t n_k, int k, int32_t* __restrict__ idx,
+                    int* __restrict__ gate, int list_cap) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
+  uint32_t* poss = keys + list_cap;
+  const int t = blockIdx.x;
+  const int64_t visible = min(q_pos0 + t + 1, n_k);
+  // every thread owns a run of 4-word units (the scoring pass wrote whole
+  // 128-key tiles, so the words up to the next multiple of 4 exist and hold
+  // no bit past the row's last visible key)
+  const uint32_t units = static_cast<uint32_t>((visible + 127) / 128);
+  const uint32_t per = (units + kTopkThreads - 1) / kTopkThreads;
+  const uint32_t u0 = min(threadIdx.x * per, units), u1 = min(u0 + per, units);
+  const uint4* mrow = reinterpret_cast<const uint4*>(mask + static_cast<int64_t>(t) * mask_ld);
+  uint32_t c = 0;
+  for (uint32_t u = u0; u < u1; ++u) {
+    const uint4 m = __ldg(mrow + u);
+    c += __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
+  }
+  uint32_t total;
+  uint32_t slot = block_excl_scan(c, sc, total);
+  const uint32_t need_total = static_cast<uint32_t>(visible < k ? visible : k);
+  if (total < need_total || total > static_cast<uint32_t>(list_cap)) {
+    if (threadIdx.x == 0) {
+      gate[1 + t] = 1;
+      atomicOr(gate, 1);
+    }
+    return;
+  }
+  // kept positions in ascending order, then their logits (batches of
+  // independent loads)
+  for (uint32_t u = u0; u < u1; ++u) {
+    const uint4 m4 = __ldg(mrow + u);
+    const uint32_t mw[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t m = mw[q];
+      while (m) {
+        poss[slot++] = (u * 4u + q) * 32u + static_cast<uint32_t>(__ffs(m) - 1);
+        m &= m - 1u;
+      }
+    }
+  }
+  __syncthreads();
+  const float* row = logits + static_cast<int64_t>(t) * ld;
+  constexpr int kBatch = 8;
+  for (uint32_t b0 = 0; b0 < total; b0 += kBatch * kTopkThreads) {
+    float v[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const uint32_t i = b0 + j * kTopkThreads + threadIdx.x;
+      v[j] = i < total ? __ldg(row + poss[i]) : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const uint32_t i = b0 + j * kTopkThreads + threadIdx.x;
+      if (i < total) keys[i] = f2key(v[j]);
+    }
+  }
+  __syncthreads();
+  const ListSrc ls{keys, poss, static_cast<int64_t>(total)};
+  const OutEmit out{idx + static_cast<int64_t>(t) * k, nullptr, static_cast<uint32_t>(k)};
+  uint32_t T = 0u, need = 0u;
+  if (total > static_cast<uint32_t>(k)) T = kth_largest(ls, static_cast<uint32_t>(k), hist, sc, need);
+  const uint32_t kept = ordered_select(ls, T, need, static_cast<uint32_t>(k), out, sc);
+  for (uint32_t i = min(kept, static_cast<uint32_t>(k)) + threadIdx.x; i < static_cast<uint32_t>(k);
+       i += kTopkThreads)
+    out.out[i] = -1;
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k,
                         int row_len, const int32_t* cand, int k, int32_t* idx,
-                        const DevCtl& ctl, cudaStream_t s) {
+                        const DevCtl& ctl, cudaStream_t s, const int* gate) {
   if (n_q <= 0 || k <= 0) return cudaSuccess;
   // list capacity: the fast path needs kFastCap; the fallback wants room for
   // the entries in or above the k-th histogram bin
@@ -616,9 +764,46 @@ cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, 
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  TopkParams p{vals, ld, n_q, q_pos0, n_k, row_len, cand, k, idx, cap, ctl};
+  TopkParams p{vals, ld, n_q, q_pos0, n_k, row_len, cand, k, idx, cap, ctl, gate};
   topk_kernel<<<n_q, kTopkThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
+
+cudaError_t launch_gather_sample(const void* K, const float* k_scale, int row_bytes, int64_t span,
+                                 int n_blocks, void* Ks, float* ks_scale, cudaStream_t s) {
+  gather_sample_kernel<<<n_blocks, 256, 0, s>>>(static_cast<const uint8_t*>(K), k_scale, row_bytes,
+                                                span, n_blocks, static_cast<uint8_t*>(Ks), ks_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fused_tau(const float* sample, int64_t lds, int n_s, int n_q, int64_t q_pos0,
+                             int64_t n_k, int k, float* tau, int* gate, cudaStream_t s) {
+  if (n_q <= 0) return cudaSuccess;
+  const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(n_s) * 4;
+  cudaError_t e = cudaFuncSetAttribute(fused_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  fused_tau_kernel<<<n_q, kTopkThreads, smem, s>>>(sample, lds, n_s, q_pos0, n_k, k, tau, gate);
+  return cudaGetLastError();
+}
+
+int fused_list_cap(int k) { return std::max(6144, (3 * k + 1023) / 1024 * 1024); }
+
+cudaError_t launch_fused_finish(const float* logits, int64_t ld, const uint32_t* mask,
+                                int64_t mask_ld, int n_q, int64_t q_pos0, int64_t n_k, int k,
+                                int32_t* idx, int* gate, cudaStream_t s) {
+  if (n_q <= 0 || k <= 0) return cudaSuccess;
+  const int cap = fused_list_cap(k);
+  const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * 8;
+  cudaError_t e = cudaFuncSetAttribute(fused_finish_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  fused_finish_kernel<<<n_q, kTopkThreads, smem, s>>>(logits, ld, mask, mask_ld, q_pos0, n_k, k,
+                                                       idx, gate, cap);
+  return cudaGetLastError();
+}
+
+int sample_block_keys() { return kSampleBlock; }
 
 }  // namespace misa

@@ -44,7 +44,8 @@ class MisaIndexer:
         self.sub = min(s.sub_chunk, s.n_q)
         self.kbar_hl = torch.empty((2, s.M, s.d), dtype=torch.int16, device=dev)
         self.heads = torch.empty((s.n_q, s.h), dtype=torch.int32, device=dev)
-        self.logits = torch.empty((self.sub, s.n_k), dtype=torch.float32, device=dev)
+        ld = (s.n_k + 3) // 4 * 4   # 16-byte rows
+        self.logits = torch.empty((self.sub, ld), dtype=torch.float32, device=dev)[:, :s.n_k]
         sel = s.kp if s.kp else s.k
         self.sel = torch.empty((s.n_q, sel), dtype=torch.int32, device=dev)
         if s.kp:

@@ -77,6 +77,7 @@ def test_invalid_arguments_rejected_before_launch(lib):
     assert so.misa_score_tokens(p, p, None, p, None, 0, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
     assert so.misa_score_tokens(p, p, p, p, None, 0, 10, 0, 100, 64, 128, 6, p, 100, None) == UNS
     assert so.misa_score_tokens(odd, p, p, p, None, 0, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    assert so.misa_score_tokens(p, p, p, p, None, 0, 10, 0, 101, 64, 128, 8, p, 101, None) == INV
     # top-k: k too large, ld too small
     assert so.misa_topk(p, 100, 10, 0, 100, 20000, p, None, 0, None) == INV
     assert so.misa_topk(p, 5, 10, 0, 100, 4, p, None, 0, None) == INV

@@ -1,0 +1,140 @@
+"""GPU parity of the fused routed scoring + top-k call (misa_score_topk).
+
+Its result is defined as that of misa_score_tokens followed by misa_topk, both
+parity-tested against the oracle elsewhere, so every case here is bit-exact
+against that pair on the same device inputs, and a few rows are also checked
+against the oracle's selection.  The repair flags the call leaves at the head of
+its workspace show which rows took the exact fallback; the constructed cases
+force the fallback on purpose (threshold too low: every logit equal; threshold
+too high: the sampled blocks score far above the rest).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_sparse_block_b200 import workloads as W
+from tests.gpu_helpers import dev, inputs_to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_sparse_block_b200 import _lib
+    return _lib
+
+
+def _inputs(n_q, q_pos0, n_k, H, d, B, h, k, seed, fp8=False):
+    wl = W.small_workload(f"fused{seed}", n_q=n_q, q_pos0=q_pos0, n_k=n_k, H=H, d=d, B=B, h=h,
+                          k=k, seed=seed, generator="clustered")
+    inp = W.generate(wl, fp8_keys=fp8)
+    return wl, inp, inputs_to_device(inp, fp8=fp8)
+
+
+def _heads(lib, g, wl, fp8):
+    Kdev = g["K8"] if fp8 else g["K"]
+    _, hl = lib.misa_pool_keys(Kdev, wl.B, k_scale=g.get("k_scale"))
+    heads, _ = lib.misa_route_heads(g["Q"], g["w"], hl, wl.q_pos0, wl.n_k, wl.B, wl.h)
+    return heads
+
+
+def _fused(lib, Q, w, heads, K, q_pos0, k, k_scale=None, h=None):
+    n_q, n_k = Q.shape[0], K.shape[0]
+    nbytes = lib.misa_workspace_size("score_topk", n_q, n_k, k, 0)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
+    ws.fill_(0xA5)    # stale contents must not matter
+    idx = lib.misa_score_topk(Q, w, heads, K, q_pos0, k, k_scale=k_scale, h=h, ws=ws)
+    flags = ws[:4 * (n_q + 1)].view(torch.int32).cpu().numpy() if nbytes else None
+    return idx.cpu().numpy(), flags
+
+
+def _unfused(lib, Q, w, heads, K, q_pos0, k, k_scale=None, h=None):
+    lg = lib.misa_score_tokens(Q, w, heads, K, q_pos0, k_scale=k_scale, h=h)
+    return lib.misa_topk(lg, q_pos0, K.shape[0], k).cpu().numpy(), lg
+
+
+FUSED_CASES = [
+    # n_q, q_pos0, n_k, H, d, B, h, k, fp8
+    (300, 16000, 20000, 64, 128, 128, 8, 512, False),
+    (257, 9000, 12000, 64, 128, 128, 4, 2048, False),
+    (200, 12000, 14000, 32, 64, 64, 16, 256, True),
+    (129, 20000, 24000, 64, 128, 128, 32, 1024, False),
+    (100, 6000, 7000, 64, 128, 128, 8, 8192, False),     # k above most rows' prefix
+    (64, 4095, 4200, 16, 32, 32, 4, 1, False),            # smallest fused prefix, k = 1
+]
+
+
+@pytest.mark.parametrize("n_q,q_pos0,n_k,H,d,B,h,k,fp8", FUSED_CASES)
+def test_score_topk_equals_score_then_topk(lib, n_q, q_pos0, n_k, H, d, B, h, k, fp8):
+    wl, inp, g = _inputs(n_q, q_pos0, n_k, H, d, B, h, k, seed=n_q + k, fp8=fp8)
+    heads = _heads(lib, g, wl, fp8)
+    Kdev, ksc = (g["K8"], g["k_scale"]) if fp8 else (g["K"], None)
+    got, flags = _fused(lib, g["Q"], g["w"], heads, Kdev, q_pos0, k, k_scale=ksc)
+    want, lg = _unfused(lib, g["Q"], g["w"], heads, Kdev, q_pos0, k, k_scale=ksc)
+    assert np.array_equal(got, want)
+    rows = np.linspace(0, n_q - 1, 5).astype(int)
+    lg_np = lg.cpu().numpy()
+    for t in rows:
+        one = oracle.topk(lg_np[t:t + 1], q_pos0 + t, n_k, k)
+        assert np.array_equal(got[t], one[0])
+    assert flags is not None
+    assert flags[0] == int(flags[1:].any())
+    print(f"rows repaired: {int(flags[1:].sum())} of {n_q}")
+
+
+def test_score_topk_dense_heads(lib):
+    # heads = NULL with h = H: the dense indexer through the fused call
+    n_q, q_pos0, n_k, H, d, k = 96, 8000, 9000, 64, 128, 300
+    _, _, g = _inputs(n_q, q_pos0, n_k, H, d, 128, H, k, seed=5)
+    got, _ = _fused(lib, g["Q"], g["w"], None, g["K"], q_pos0, k, h=H)
+    want, _ = _unfused(lib, g["Q"], g["w"], None, g["K"], q_pos0, k, h=H)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("q_pos0,h", [(3000, 8), (9000, 2), (9000, 128)])
+def test_score_topk_unfused_shapes(lib, q_pos0, h):
+    # prefix shorter than the sample, or h without a select kernel: the call
+    # runs the unfused sequence and must give the same result
+    n_q, n_k, H, d, k = 80, q_pos0 + 500, 128 if h == 128 else 64, 128, 200
+    wl, _, g = _inputs(n_q, q_pos0, n_k, H, d, 128, h, k, seed=q_pos0 + h)
+    heads = _heads(lib, g, wl, False)
+    got, flags = _fused(lib, g["Q"], g["w"], heads, g["K"], q_pos0, k)
+    want, _ = _unfused(lib, g["Q"], g["w"], heads, g["K"], q_pos0, k)
+    assert np.array_equal(got, want)
+
+
+def test_score_topk_repairs_ties_everywhere(lib):
+    # every key equal: every visible logit of a row ties, far more than the
+    # candidate list holds, so every row takes the exact fallback
+    n_q, q_pos0, n_k, H, d, k = 40, 12000, 12100, 64, 128, 512
+    wl, inp, g = _inputs(n_q, q_pos0, n_k, H, d, 128, 8, k, seed=21)
+    K = g["K"][:1].expand(n_k, d).contiguous()
+    heads = _heads(lib, {**g, "K": K}, wl, False)
+    got, flags = _fused(lib, g["Q"], g["w"], heads, K, q_pos0, k)
+    want, _ = _unfused(lib, g["Q"], g["w"], heads, K, q_pos0, k)
+    assert np.array_equal(got, want)
+    assert flags[0] == 1 and flags[1:].all()
+
+
+def test_score_topk_repairs_unrepresentative_sample(lib):
+    # the sampled blocks (32 blocks of 128 keys evenly spaced over 0..q_pos0)
+    # hold the only keys that score high, each a different amount, so the
+    # thresholds keep ~1.6 k * 4096 / visible of them: fewer than k
+    n_q, q_pos0, n_k, H, d, k, h = 48, 14000, 14100, 64, 128, 1024, 8
+    rng = np.random.default_rng(22)
+    Q = (1.0 + 0.3 * rng.standard_normal((n_q, H, d))) / np.sqrt(d)
+    K = 0.01 * rng.standard_normal((n_k, d)) / np.sqrt(d)
+    span, nb = q_pos0 + 1, 32
+    for b in range(nb):
+        start = (span - 128) * b // (nb - 1)
+        K[start:start + 128] = rng.uniform(2.0, 4.0, size=(128, 1)) / np.sqrt(d)
+    w = np.full((n_q, H), 1.0 / H, dtype=np.float32)
+    Qg, Kg, wg = dev(W.bf16_bits(Q)), dev(W.bf16_bits(K)), dev(w)
+    B = 128
+    _, hl = lib.misa_pool_keys(Kg, B)
+    heads, _ = lib.misa_route_heads(Qg, wg, hl, q_pos0, n_k, B, h)
+    got, flags = _fused(lib, Qg, wg, heads, Kg, q_pos0, k)
+    want, _ = _unfused(lib, Qg, wg, heads, Kg, q_pos0, k)
+    assert np.array_equal(got, want)
+    assert flags[0] == 1 and flags[1:].all()

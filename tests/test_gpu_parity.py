@@ -99,7 +99,8 @@ def test_score_matches_oracle(lib, n_q, q_pos0, n_k, H, d, h, dense):
                         axis=1).astype(np.int32)
     ref = oracle.score(Qd, wd, heads, Kd, q_pos0)
     g = inputs_to_device(inp)
-    logits = torch.full((n_q, n_k + 4), float("nan"), device="cuda")
+    ld = (n_k + 3) // 4 * 4 + 4            # a padded row pitch
+    logits = torch.full((n_q, ld), float("nan"), device="cuda")
     lib.misa_score_tokens(g["Q"], g["w"], None if dense else dev(heads), g["K"], q_pos0,
                           logits=logits, h=h)
     assert lib.misa_last_device_status() == 0
@@ -108,9 +109,10 @@ def test_score_matches_oracle(lib, n_q, q_pos0, n_k, H, d, h, dense):
         pos = q_pos0 + t
         mag = logit_magnitude(Qd, wd, Kd, heads, t, q_pos0)
         assert_logits_close(out[t], ref[t, :pos + 1], mag, what=f"row {t}")
-        tail = out[t, pos + 1:n_k]
+        n4 = (n_k + 3) // 4 * 4
+        tail = out[t, pos + 1:n4]
         assert np.all(np.isnan(tail) | np.isneginf(tail))
-        assert np.all(np.isnan(out[t, n_k:]))                             # never past n_k
+        assert np.all(np.isnan(out[t, n4:]))                # never past n_k rounded up to 4
 
 
 @pytest.mark.parametrize("n_q,q_pos0,n_k,H,d,h", [(70, 300, 517, 64, 128, 8), (257, 3, 300, 8, 32, 2),
@@ -127,7 +129,7 @@ def test_score_fp8_keys_matches_oracle(lib, n_q, q_pos0, n_k, H, d, h):
                     axis=1).astype(np.int32)
     ref = oracle.score(Qd, wd, heads, Kd, q_pos0)
     g = inputs_to_device(inp, fp8=True)
-    logits = torch.full((n_q, n_k), float("nan"), device="cuda")
+    logits = torch.full((n_q, (n_k + 3) // 4 * 4), float("nan"), device="cuda")
     lib.misa_score_tokens(g["Q"], g["w"], dev(heads), g["K8"], q_pos0, k_scale=g["k_scale"],
                           logits=logits, h=h)
     assert lib.misa_last_device_status() == 0
