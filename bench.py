@@ -6,8 +6,9 @@
 One step = the whole indexer over one long-context prefill chunk: pool the
 131072 keys into 1024 blocks, route every (query, head) against them and keep
 the top-8 heads, score the causal prefix of all 8192 queries with their routed
-heads (fused ReLU * w head-sum on the tensor cores, in 1024-query sub-chunks),
-and select the top-2048 tokens per query.  Inputs are seeded synthetic arrays
+heads and select the top-2048 tokens per query (one fused call: sampled per-row
+thresholds, tensor-core scoring with the ReLU * w head-sum and threshold test in
+the epilogue, exact selection among the kept logits).  Inputs are seeded synthetic arrays
 of the chunk's shape (clustered keys, head-specific query mixtures), resident in
 HBM when the timed region starts.  L2 is flushed (a 256 MiB write) before every
 timed step; all times are CUDA events on the launching stream.
@@ -42,11 +43,10 @@ from long_context_sparse_block_b200 import workloads as W  # noqa: E402
 
 METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor peak"
 
-# DRAM bytes (read + write) of one score launch (first 1024-query sub-chunk) from
-# the ncu capture in profiles/score_tokens_chunk_128k.md, valid only for the
-# kernel sources it was taken on.
-SCORE_TRAFFIC = {"sources_sha256_16": "f9d4a13d8e7e739f", "bytes_per_launch": 134.102528e6 + 459.236608e6,
-                 "launch": "queries 0..1023 of chunk_128k"}
+# DRAM bytes (read + write) of one select-mode scoring launch over all 8192
+# queries of chunk_128k, from the ncu capture summarised under profiles/; valid
+# only for the kernel sources it was taken on (null otherwise).
+SCORE_TRAFFIC = {"sources_sha256_16": "", "bytes_per_launch": None, "queries": 8192}
 
 
 def _score_sources_digest():
@@ -206,7 +206,9 @@ def run_ours(args, rank, world, local_rank, inp):
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
 
-    # per-stage events: wrap the library calls of one step
+    # per-stage events: pool and route from torch events around their calls;
+    # the stages inside the fused score + top-k call from the library's own
+    # profiler (events recorded on the same stream between its launches)
     stage_events = []
 
     def step(record):
@@ -221,24 +223,20 @@ def run_ours(args, rank, world, local_rank, inp):
         e2 = torch.cuda.Event(enable_timing=True)
         e2.record(stream)
         ev += [("pool", e0, e1), ("route", e1, e2)]
-        prev = e2
         for c0 in range(0, s.n_q, ix.sub):
             c1 = min(s.n_q, c0 + ix.sub)
-            lg = ix.logits[:c1 - c0]
-            _lib.misa_score_tokens(Q[c0:c1], w[c0:c1], ix.heads[c0:c1], K, s.q_pos0 + c0,
-                                   logits=lg, h=s.h)
-            ea = torch.cuda.Event(enable_timing=True)
-            ea.record(stream)
-            _lib.misa_topk(lg, s.q_pos0 + c0, s.n_k, s.k, idx=ix.sel[c0:c1])
-            eb = torch.cuda.Event(enable_timing=True)
-            eb.record(stream)
-            ev += [("score", prev, ea), ("topk", ea, eb)]
-            prev = eb
+            _lib.misa_score_topk(Q[c0:c1], w[c0:c1], ix.heads[c0:c1], K, s.q_pos0 + c0, s.k,
+                                 h=s.h, idx=ix.sel[c0:c1], logits=ix.logits[:c1 - c0],
+                                 ws=ix.ws_sel)
+        e3 = torch.cuda.Event(enable_timing=True)
+        e3.record(stream)
+        ev += [("score_topk", e2, e3)]
         if record:
             stage_events.append(ev)
-        return e0, prev
+        return e0, e3
 
-    launches_per_step = 2 + 2 * math.ceil(wl.n_q / ix.sub)
+    fused = _lib.misa_workspace_size("score_topk", ix.sub, wl.n_k, wl.k, 0) > 0
+    launches_per_step = 2 + (7 if fused else 2) * math.ceil(wl.n_q / ix.sub)
     for _ in range(args.warmup):
         flush.zero_()
         step(False)
@@ -249,6 +247,7 @@ def run_ours(args, rank, world, local_rank, inp):
     clocks = ClockSampler(local_rank)
     if rank == 0:
         clocks.start()
+    _lib.misa_profile_start()
     spans = []
     for _ in range(args.steps):
         flush.zero_()
@@ -258,6 +257,8 @@ def run_ours(args, rank, world, local_rank, inp):
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop() if rank == 0 else None
+    fused_stages = _lib.misa_profile_stop()
+    repaired = int(ix.ws_sel[4:4 * (ix.sub + 1)].view(torch.int32).sum()) if fused else None
     assert _lib.misa_last_device_status() == 0, "device status"
     step_ms = [a.elapsed_time(b) for a, b in spans]
     variants = None
@@ -271,6 +272,9 @@ def run_ours(args, rank, world, local_rank, inp):
         for name, a, b in ev:
             stage_ms[name] = stage_ms.get(name, 0.0) + a.elapsed_time(b)
     stage_ms = {k: v / args.steps for k, v in stage_ms.items()}
+    for name, (tot, cnt) in fused_stages.items():
+        if cnt:
+            stage_ms[name] = tot / args.steps
     ms = statistics.mean(step_ms)
     if world > 1:
         t = torch.tensor([ms], device="cuda", dtype=torch.float64)
@@ -308,12 +312,12 @@ def run_ours(args, rank, world, local_rank, inp):
     peaks = _peaks()
     pairs = wl.causal_pairs()
     traffic = (SCORE_TRAFFIC["bytes_per_launch"]
-               if h == 8 and wl.name == "chunk_128k"
+               if h == 8 and wl.name == "chunk_128k" and ix.sub == SCORE_TRAFFIC["queries"]
                and _score_sources_digest() == SCORE_TRAFFIC["sources_sha256_16"] else None)
     score_flops = 2.0 * h * wl.d * pairs
-    score_ms = stage_ms["score"]
+    score_key = "select_score" if "select_score" in stage_ms else "score_topk"
+    score_ms = stage_ms[score_key]
     tflops = score_flops / (score_ms * 1e-3) / 1e12
-    topk_gbs = 4.0 * pairs / (stage_ms["topk"] * 1e-3) / 1e9
     pool_gbs = (wl.n_k * wl.d * 2 + 2 * wl.M * wl.d * 2) / (stage_ms["pool"] * 1e-3) / 1e9
     # router: H_I * d multiply-adds per (query, complete causal block), done twice
     # (hi and lo halves of the pooled keys)
@@ -339,12 +343,15 @@ def run_ours(args, rank, world, local_rank, inp):
             "workload": (f"{wl.name}: {wl.n_q} queries at {wl.q_pos0}..{wl.q_pos0 + wl.n_q - 1} "
                          f"x {wl.n_k} keys, H_I={wl.H}, d={wl.d}, B={wl.B}, h={h}, k={wl.k}"),
             "query_sub_chunk": ix.sub,
+            "fused_score_topk": fused,
+            "rows_repaired_last_subchunk": repaired,
             "l2": "flushed by a 256 MiB write before every timed step",
             "parallelism": f"independent chunks per rank x{world}",
         },
         "roofline": {
             "bound": "tensor",
-            "kernel": "score_tokens (tcgen05, fused ReLU*w head-sum epilogue)",
+            "kernel": ("score_tokens select mode (tcgen05, fused ReLU*w head-sum, "
+                       "threshold + pass-mask epilogue)"),
             "achieved": round(tflops, 1),
             "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s",
@@ -353,12 +360,12 @@ def run_ours(args, rank, world, local_rank, inp):
             "traffic": traffic,
             "traffic_unit": "bytes per launch (ncu dram read+write)",
             "algorithmic": f"2*h*d*pairs = {score_flops:.4g} flop per step, {pairs} causal pairs",
+            "launches_per_step": math.ceil(wl.n_q / ix.sub),
         },
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "stage_rates": {
             "score_tflops": round(tflops, 1),
             "route_tflops_hi_lo": round(route_tflops, 1),
-            "topk_logit_gbs": round(topk_gbs, 1),
             "pool_gbs": round(pool_gbs, 1),
             "hbm_peak_gbs": peaks["hbm_gbs"],
             "pairs_per_s": round(pairs / (ms * 1e-3), 1),
@@ -471,7 +478,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="chunk_128k")
     ap.add_argument("--h", type=int, default=0)
-    ap.add_argument("--sub-chunk", type=int, default=1024)
+    ap.add_argument("--sub-chunk", type=int, default=8192)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")

@@ -171,6 +171,20 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
                     int d, int h, int k, int32_t* idx, float* logits, int64_t ld, void* ws,
                     size_t ws_bytes, void* stream);
 
+/*
+ * Stage timing of misa_score_topk (diagnostic; not a step of the method).
+ * Between misa_profile_start() and misa_profile_stop(), each launch of the fused
+ * sequence is bracketed by CUDA events on the call's stream.  misa_profile_stop
+ * synchronises on those events and writes, for stage i < n, the summed device
+ * milliseconds ms[i] and the number of launches counts[i] (either array may be
+ * NULL); misa_profile_stage_name(i) names stage i (NULL past the last).  The
+ * fused call's stages: sample_gather, sample_score, threshold, select_score,
+ * finish, repair_score, repair_topk.  Not for use inside stream capture.
+ */
+int misa_profile_start(void);
+int misa_profile_stop(double* ms, int* counts, int n);
+const char* misa_profile_stage_name(int i);
+
 /* Workspace bytes needed by op "topk", "rerank" or "score_topk" for the given
  * sizes (0 if none). */
 size_t misa_workspace_size(const char* op, int n_q, int64_t n_k, int k, int kp);

@@ -46,6 +46,9 @@ _SIGS = {
                                    _int, _int, _vp, _vp]),
     "misa_score_topk": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _int, _int, _int,
                                _int, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "misa_profile_start": (_int, []),
+    "misa_profile_stop": (_int, [_vp, _vp, _int]),
+    "misa_profile_stage_name": (ctypes.c_char_p, [_int]),
     "misa_workspace_size": (_sz, [ctypes.c_char_p, _int, _i64, _int, _int]),
     "misa_status_string": (ctypes.c_char_p, [_int]),
     "misa_last_device_status": (_int, [_vp]),
@@ -171,6 +174,8 @@ def misa_score_topk(Q, w, heads, K, q_pos0: int, k: int, k_scale=None, h: int | 
         idx = torch.empty((n_q, k), dtype=torch.int32, device=Q.device)
     if logits is None:
         logits = torch.empty((n_q, (n_k + 3) // 4 * 4), dtype=torch.float32, device=Q.device)
+    if logits.dim() != 2 or logits.stride(1) != 1 or logits.shape[0] < n_q:
+        raise ValueError("logits must be a row-major [n_q, >= n_k] fp32 buffer")
     ws_bytes = misa_workspace_size("score_topk", n_q, n_k, k, 0)
     if ws_bytes and (ws is None or ws.numel() * ws.element_size() < ws_bytes):
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
@@ -224,6 +229,26 @@ def misa_rerank_noalloc(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, idx=No
                                   K.shape[0], H, d, k, _ptr(idx, (torch.int32,), "idx"), _stream())
     _check("misa_rerank_noalloc", st)
     return idx
+
+
+def misa_profile_start() -> None:
+    _check("misa_profile_start", _lib.misa_profile_start())
+
+
+def misa_profile_stop() -> dict:
+    """Per-stage device milliseconds (summed) and launch counts of the fused
+    calls made since misa_profile_start()."""
+    n = 16
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int * n)()
+    _check("misa_profile_stop", _lib.misa_profile_stop(ms, cnt, n))
+    out = {}
+    for i in range(n):
+        name = _lib.misa_profile_stage_name(i)
+        if name is None:
+            break
+        out[name.decode()] = (ms[i], cnt[i])
+    return out
 
 
 def misa_last_device_status() -> int:

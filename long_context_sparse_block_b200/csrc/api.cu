@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
 #include "misa.h"
@@ -68,6 +69,40 @@ constexpr int64_t kFusedMaxKeys = int64_t(1) << 18;  // a 4096-key sample stays 
 constexpr int kFusedMaxK = 8192;                    // the finish kernel's list fits in shared memory
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Optional per-stage timing of misa_score_topk: while enabled, every launch of
+// the fused sequence is bracketed by a pair of CUDA events on its stream.
+constexpr int kStages = 7;
+const char* const kStageNames[kStages] = {"sample_gather", "sample_score", "threshold",
+                                          "select_score",  "finish",       "repair_score",
+                                          "repair_topk"};
+struct Profiler {
+  std::mutex mu;
+  std::atomic<bool> on{false};
+  std::vector<cudaEvent_t> start[kStages], stop[kStages];
+};
+Profiler g_prof;
+
+struct StageMark {
+  int stage;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  StageMark(int st, cudaStream_t str) : stage(st), s(str) {
+    if (g_prof.on.load() && cudaEventCreate(&a) == cudaSuccess) cudaEventRecord(a, s);
+  }
+  ~StageMark() {
+    if (!a) return;
+    cudaEvent_t b = nullptr;
+    if (cudaEventCreate(&b) != cudaSuccess) {
+      cudaEventDestroy(a);
+      return;
+    }
+    cudaEventRecord(b, s);
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    g_prof.start[stage].push_back(a);
+    g_prof.stop[stage].push_back(b);
+  }
+};
 
 int64_t mask_words(int64_t n_k) { return ((n_k + 31) / 32 + 3) / 4 * 4; }
 
@@ -293,8 +328,12 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
   uint32_t* mask = reinterpret_cast<uint32_t*>(base + L.mask);
   const int64_t mld = mask_words(n_k);
   const int row_bytes = fp8 ? d : 2 * d;
-  cudaError_t e = launch_gather_sample(K, fp8 ? k_scale : nullptr, row_bytes, q_pos0 + 1,
-                                       kSampleBlocks, Ks, fp8 ? ks_scale : nullptr, s);
+  cudaError_t e;
+  {
+    StageMark m(0, s);
+    e = launch_gather_sample(K, fp8 ? k_scale : nullptr, row_bytes, q_pos0 + 1, kSampleBlocks, Ks,
+                             fp8 ? ks_scale : nullptr, s);
+  }
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   ScoreLaunch sa = a;  // the sample: every sampled key is visible to every query
   sa.K = Ks;
@@ -303,23 +342,81 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
   sa.n_k = kSampleKeys;
   sa.logits = sample;
   sa.ld = kSampleKeys;
-  if ((e = launch_score(sa, ctl, s)) != cudaSuccess) return MISA_ERR_CUDA;
-  if ((e = launch_fused_tau(sample, kSampleKeys, kSampleKeys, n_q, q_pos0, n_k, k, tau, gate, s)) !=
-      cudaSuccess)
-    return MISA_ERR_CUDA;
+  {
+    StageMark m(1, s);
+    e = launch_score(sa, ctl, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  {
+    StageMark m(2, s);
+    e = launch_fused_tau(sample, kSampleKeys, kSampleKeys, n_q, q_pos0, n_k, k, tau, gate, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
   ScoreLaunch se = a;  // select mode
   se.tau = tau;
   se.mask = mask;
   se.mask_ld = mld;
-  if ((e = launch_score(se, ctl, s)) != cudaSuccess) return MISA_ERR_CUDA;
-  if ((e = launch_fused_finish(logits, ld, mask, mld, n_q, q_pos0, n_k, k, idx, gate, s)) !=
-      cudaSuccess)
-    return MISA_ERR_CUDA;
+  {
+    StageMark m(3, s);
+    e = launch_score(se, ctl, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  {
+    StageMark m(4, s);
+    e = launch_fused_finish(logits, ld, mask, mld, n_q, q_pos0, n_k, k, idx, gate, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
   // exact fallback for the rows the thresholds missed (a no-op launch when none)
   ScoreLaunch ra = a;
   ra.gate = gate;
-  if ((e = launch_score(ra, ctl, s)) != cudaSuccess) return MISA_ERR_CUDA;
+  {
+    StageMark m(5, s);
+    e = launch_score(ra, ctl, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  StageMark m(6, s);
   return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, 0, nullptr, k, idx, ctl, s, gate));
+}
+
+int misa_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  for (int i = 0; i < kStages; ++i) {
+    for (cudaEvent_t e : g_prof.start[i]) cudaEventDestroy(e);
+    for (cudaEvent_t e : g_prof.stop[i]) cudaEventDestroy(e);
+    g_prof.start[i].clear();
+    g_prof.stop[i].clear();
+  }
+  g_prof.on.store(true);
+  return MISA_OK;
+}
+
+int misa_profile_stop(double* ms, int* counts, int n) {
+  g_prof.on.store(false);
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  int status = MISA_OK;
+  for (int i = 0; i < kStages; ++i) {
+    double sum = 0.0;
+    for (size_t j = 0; j < g_prof.start[i].size(); ++j) {
+      float t = 0.0f;
+      if (cudaEventSynchronize(g_prof.stop[i][j]) != cudaSuccess ||
+          cudaEventElapsedTime(&t, g_prof.start[i][j], g_prof.stop[i][j]) != cudaSuccess)
+        status = MISA_ERR_CUDA;
+      sum += t;
+      cudaEventDestroy(g_prof.start[i][j]);
+      cudaEventDestroy(g_prof.stop[i][j]);
+    }
+    if (i < n) {
+      if (ms) ms[i] = sum;
+      if (counts) counts[i] = static_cast<int>(g_prof.start[i].size());
+    }
+    g_prof.start[i].clear();
+    g_prof.stop[i].clear();
+  }
+  return status;
+}
+
+const char* misa_profile_stage_name(int i) {
+  return (i >= 0 && i < kStages) ? kStageNames[i] : nullptr;
 }
 
 size_t misa_workspace_size(const char* op, int n_q, int64_t n_k, int k, int kp) {

@@ -1,13 +1,14 @@
 """The MISA indexer pipeline over one prefill chunk, through the C ABI.
 
-    pool  -> route (top-h) -> for each query sub-chunk: score -> top-k
-                                                        [-> top-k' -> rerank]
+    pool -> route (top-h) -> for each query sub-chunk: fused score + top-k
+                                                       [(top-k') -> rerank]
 
 ("MISA: Mixture of Indexer Sparse Attention", technical summary: Metodologia
 steps 1-2 and Variante Hierarquica.)  Buffers are allocated once, with torch,
 when the indexer is built; `run` only launches the library's kernels on the
-current stream.  Queries are scored in sub-chunks so that the fp32 logits of a
-whole 8192 x 131072 chunk are never resident at once.
+current stream.  Scoring and selection run as one fused call (misa_score_topk),
+which keeps only the logits above per-row sampled thresholds; the logits buffer
+is its scratch.  Queries can be scored in sub-chunks to bound that buffer.
 """
 from __future__ import annotations
 
@@ -30,7 +31,7 @@ class IndexerShape:
     k: int
     kp: int = 0     # MISA-dagger candidate count (0: plain MISA)
     dense: bool = False
-    sub_chunk: int = 1024
+    sub_chunk: int = 8192
 
     @property
     def M(self) -> int:
@@ -48,6 +49,8 @@ class MisaIndexer:
         self.logits = torch.empty((self.sub, ld), dtype=torch.float32, device=dev)[:, :s.n_k]
         sel = s.kp if s.kp else s.k
         self.sel = torch.empty((s.n_q, sel), dtype=torch.int32, device=dev)
+        nbytes = _lib.misa_workspace_size("score_topk", self.sub, s.n_k, sel, 0)
+        self.ws_sel = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
         if s.kp:
             self.final = torch.empty((s.n_q, s.k), dtype=torch.int32, device=dev)
             nbytes = _lib.misa_workspace_size("rerank", self.sub, s.n_k, s.k, s.kp)
@@ -58,8 +61,9 @@ class MisaIndexer:
     def run(self, Q, K, w, k_scale=None, on_subchunk=None):
         """Q [n_q,H,d] bf16 codes, K [n_k,d] bf16 codes (or e4m3 + k_scale), w [n_q,H] f32.
         Returns the selected token indices [n_q, k] (int32, ascending, -1 padded).
-        on_subchunk(c0, c1, logits) is called after each sub-chunk is scored (for
-        inspection; the logits buffer is reused by the next sub-chunk)."""
+        on_subchunk(c0, c1, logits), when given, switches to the unfused sequence
+        (every logit written, then the top-k) and is called after each sub-chunk
+        is scored, for inspection; the logits buffer is reused by the next one."""
         s = self.shape
         if not s.dense:
             _lib.misa_pool_keys(K, s.B, k_scale=k_scale, kbar_hl=self.kbar_hl, want_kbar=False)
@@ -68,11 +72,16 @@ class MisaIndexer:
             c1 = min(s.n_q, c0 + self.sub)
             n = c1 - c0
             lg = self.logits[:n]
-            _lib.misa_score_tokens(Q[c0:c1], w[c0:c1], None if s.dense else self.heads[c0:c1], K,
-                                   s.q_pos0 + c0, k_scale=k_scale, logits=lg, h=s.h)
-            if on_subchunk is not None:
+            heads = None if s.dense else self.heads[c0:c1]
+            if on_subchunk is None:
+                _lib.misa_score_topk(Q[c0:c1], w[c0:c1], heads, K, s.q_pos0 + c0,
+                                     self.sel.shape[1], k_scale=k_scale, h=s.h,
+                                     idx=self.sel[c0:c1], logits=lg, ws=self.ws_sel)
+            else:
+                _lib.misa_score_tokens(Q[c0:c1], w[c0:c1], heads, K, s.q_pos0 + c0,
+                                       k_scale=k_scale, logits=lg, h=s.h)
                 on_subchunk(c0, c1, lg)
-            _lib.misa_topk(lg, s.q_pos0 + c0, s.n_k, self.sel.shape[1], idx=self.sel[c0:c1])
+                _lib.misa_topk(lg, s.q_pos0 + c0, s.n_k, self.sel.shape[1], idx=self.sel[c0:c1])
             if s.kp:
                 _lib.misa_rerank(Q[c0:c1], w[c0:c1], K, self.sel[c0:c1], s.q_pos0 + c0, s.k,
                                  k_scale=k_scale, idx=self.final[c0:c1], ws=self.ws)
