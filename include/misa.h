@@ -159,7 +159,8 @@ int misa_rerank_noalloc(const uint16_t* Q, const float* w, const void* K, const 
  *   logits [n_q, ld]: scratch for the kept logits and the fallback (contents
  *     unspecified afterwards; ld >= n_k, a multiple of 4, 16-byte aligned).
  *   ws/ws_bytes: misa_workspace_size("score_topk", n_q, n_k, k, 0) bytes,
- *     16-byte aligned.  That size is 0 (and the call runs the unfused
+ *     16-byte aligned (it includes room for FP8 keys decoded to bf16, which
+ *     every scoring pass of the fused sequence then reads).  That size is 0 (and the call runs the unfused
  *     sequence) unless 4096 <= n_k <= 262144 and 1 <= k <= 8192.  The fused
  *     sequence also needs q_pos0 >= 4095 and h in {4, 8, 16, 32, 64}, else the
  *     call is unfused.  After a fused call, ws holds n_q + 1 int32 repair flags
@@ -178,8 +179,8 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
  * synchronises on those events and writes, for stage i < n, the summed device
  * milliseconds ms[i] and the number of launches counts[i] (either array may be
  * NULL); misa_profile_stage_name(i) names stage i (NULL past the last).  The
- * fused call's stages: sample_gather, sample_score, threshold, select_score,
- * finish, repair_score, repair_topk.  Not for use inside stream capture.
+ * fused call's stages: prepare (FP8 key decode and sample gather),
+ * sample_score, threshold, select_score, finish, repair_score, repair_topk.  Not for use inside stream capture.
  */
 int misa_profile_start(void);
 int misa_profile_stop(double* ms, int* counts, int n);

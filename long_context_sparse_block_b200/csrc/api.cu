@@ -73,7 +73,7 @@ size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 // Optional per-stage timing of misa_score_topk: while enabled, every launch of
 // the fused sequence is bracketed by a pair of CUDA events on its stream.
 constexpr int kStages = 7;
-const char* const kStageNames[kStages] = {"sample_gather", "sample_score", "threshold",
+const char* const kStageNames[kStages] = {"prepare",       "sample_score", "threshold",
                                           "select_score",  "finish",       "repair_score",
                                           "repair_topk"};
 struct Profiler {
@@ -107,7 +107,7 @@ struct StageMark {
 int64_t mask_words(int64_t n_k) { return ((n_k + 31) / 32 + 3) / 4 * 4; }
 
 struct FusedLayout {
-  size_t gate, tau, ks, ks_scale, sample, mask, total;
+  size_t gate, tau, ks, ks_scale, sample, mask, kbf, total;
   FusedLayout(int n_q, int64_t n_k) {
     const size_t nq = static_cast<size_t>(n_q);
     size_t o = 0;
@@ -123,6 +123,8 @@ struct FusedLayout {
     o += round256(nq * kSampleKeys * 4);
     mask = o;
     o += round256(nq * static_cast<size_t>(mask_words(n_k)) * 4);
+    kbf = o;  // FP8 keys decoded to bf16 (d <= 128)
+    o += round256(static_cast<size_t>(n_k) * 256);
     total = o;
   }
 };
@@ -327,11 +329,17 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
   float* sample = reinterpret_cast<float*>(base + L.sample);
   uint32_t* mask = reinterpret_cast<uint32_t*>(base + L.mask);
   const int64_t mld = mask_words(n_k);
-  const int row_bytes = fp8 ? d : 2 * d;
   cudaError_t e;
   {
     StageMark m(0, s);
-    e = launch_gather_sample(K, fp8 ? k_scale : nullptr, row_bytes, q_pos0 + 1, kSampleBlocks, Ks,
+    if (fp8) {  // decode the keys once; every scoring pass then reads bf16 codes
+      uint16_t* kbf = reinterpret_cast<uint16_t*>(base + L.kbf);
+      e = launch_e4m3_to_bf16(static_cast<const uint8_t*>(K), kbf, n_k * d, s);
+      if (e != cudaSuccess) return MISA_ERR_CUDA;
+      a.K = kbf;
+      a.k_bf16 = true;
+    }
+    e = launch_gather_sample(a.K, fp8 ? k_scale : nullptr, 2 * d, q_pos0 + 1, kSampleBlocks, Ks,
                              fp8 ? ks_scale : nullptr, s);
   }
   if (e != cudaSuccess) return MISA_ERR_CUDA;

@@ -32,6 +32,7 @@ struct ScoreLaunch {
   const void* K;
   const float* k_scale;
   bool fp8;
+  bool k_bf16;            // FP8 keys given already decoded to bf16 codes at K
   int n_q;
   int64_t q_pos0;
   int64_t n_k;
@@ -60,6 +61,9 @@ cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t
 cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k,
                         int row_len, const int32_t* cand, int k, int32_t* idx,
                         const DevCtl& ctl, cudaStream_t s, const int* gate = nullptr);
+
+// Exact decode of FP8 E4M3 key codes to bf16 codes (pool.cu); n multiple of 16.
+cudaError_t launch_e4m3_to_bf16(const uint8_t* src, uint16_t* dst, int64_t n, cudaStream_t s);
 
 // Fused top-k helpers (topk.cu): sample gather, per-row thresholds from the
 // scored sample, and the exact selection over the select-mode candidates.

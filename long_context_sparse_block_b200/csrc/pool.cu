@@ -1,3 +1,4 @@
+#include <algorithm>
 // Stage 1 — block mean-pooling of the shared index keys.
 //
 // kbar[m, :] = (1/n_m) * sum of K rows mB .. mB+n_m-1, n_m = min(B, n_k - mB)
@@ -118,7 +119,35 @@ cudaError_t launch(const void* K, const float* k_scale, int64_t n_k, int B, floa
   return cudaGetLastError();
 }
 
+// 16 E4M3 codes per thread -> 16 bf16 codes (exact: every E4M3 value is a bf16
+// value).
+__global__ void __launch_bounds__(256)
+e4m3_to_bf16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n16) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 raw = __ldg(src + i);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      o[2 * j] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w[j] & 0xFFFF));
+      o[2 * j + 1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w[j] >> 16));
+    }
+    dst[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_e4m3_to_bf16(const uint8_t* src, uint16_t* dst, int64_t n, cudaStream_t s) {
+  const int64_t n16 = n / 16;
+  if (n16 <= 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((n16 + 255) / 256, static_cast<int64_t>(sm_count()) * 8);
+  e4m3_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), n16);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pool_keys(const void* K, const float* k_scale, bool fp8, int64_t n_k, int d,
                              int B, float* kbar, uint16_t* kbar_hl, cudaStream_t s) {

@@ -129,35 +129,72 @@ rerank_scores_kernel(const RerankParams p) {
       fence_proxy_async_smem();
       mbar_arrive(bar(BFULL));
       ++qcount;
+      // each producer thread owns one candidate row of every tile: its index
+      // is loaded a tile ahead, and the row's copies are all in flight at once
+      // (bf16: asynchronous 16-byte copies that arrive on the stage barrier when
+      // they land; FP8: the codes of the next tile's row are loaded while this
+      // tile's are decoded)
+      const int32_t* crow = p.cand + static_cast<int64_t>(t) * p.kp;
+      auto cand_of = [&](int tile) -> int64_t {
+        const int i = tile * kCand + tid;
+        int64_t c = i < p.kp ? static_cast<int64_t>(__ldg(crow + i)) : -1;
+        return (c >= 0 && c <= pos && c < p.n_k) ? c : -1;
+      };
+      constexpr int U8 = D / 16;  // 16-byte units of an e4m3 row
+      int64_t c_next = tiles > 0 ? cand_of(0) : -1;
+      uint4 raw_next[FP8 ? U8 : 1];
+      if constexpr (FP8) {
+#pragma unroll
+        for (int u = 0; u < U8; ++u)
+          raw_next[u] = c_next >= 0 ? __ldg(reinterpret_cast<const uint4*>(p.K + c_next * D) + u)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+      }
       for (int tile = 0; tile < tiles; ++tile) {
+        const int64_t c = c_next;
+        uint4 raw[FP8 ? U8 : 1];
+        if constexpr (FP8) {
+#pragma unroll
+          for (int u = 0; u < U8; ++u) raw[u] = raw_next[u];
+        }
+        if (tile + 1 < tiles) c_next = cand_of(tile + 1);
+        if constexpr (FP8) {
+#pragma unroll
+          for (int u = 0; u < U8; ++u)
+            raw_next[u] = (tile + 1 < tiles && c_next >= 0)
+                              ? __ldg(reinterpret_cast<const uint4*>(p.K + c_next * D) + u)
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
         ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
         if (!ok) break;
         const uint32_t dstA = sA + stage * L::A_BYTES;
-        for (int x = tid; x < kCand * UPR; x += kProducers) {
-          const int r = x / UPR, u = x % UPR;
-          const int i = tile * kCand + r;
-          int64_t c = -1;
-          if (i < p.kp) c = __ldg(p.cand + static_cast<int64_t>(t) * p.kp + i);
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (c >= 0 && c <= pos && c < p.n_k) {
-            if (FP8) {
-              // 8 E4M3 codes -> 8 bf16
-              const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p.K + c * D + u * 8));
-              v.x = e4m3x2_to_bf16x2(static_cast<uint16_t>(raw.x & 0xFFFF));
-              v.y = e4m3x2_to_bf16x2(static_cast<uint16_t>(raw.x >> 16));
-              v.z = e4m3x2_to_bf16x2(static_cast<uint16_t>(raw.y & 0xFFFF));
-              v.w = e4m3x2_to_bf16x2(static_cast<uint16_t>(raw.y >> 16));
-            } else {
-              v = __ldg(reinterpret_cast<const uint4*>(p.K + (c * D + u * 8) * 2));
+        if constexpr (FP8) {
+#pragma unroll
+          for (int u = 0; u < U8; ++u) {
+            const uint32_t wv[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {  // 8 codes -> 8 bf16 (exact)
+              const uint32_t b0 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh] & 0xFFFF));
+              const uint32_t b1 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh] >> 16));
+              const uint32_t b2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh + 1] & 0xFFFF));
+              const uint32_t b3 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh + 1] >> 16));
+              const int u2 = 2 * u + hh;
+              const uint32_t off = (u2 / UPC) * L::A_CHUNK + swz_offset(tid, u2 % UPC, L::ROWB);
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dstA + off), "r"(b0),
+                           "r"(b1), "r"(b2), "r"(b3)
+                           : "memory");
             }
           }
-          const uint32_t off = (u / UPC) * L::A_CHUNK + swz_offset(r, u % UPC, L::ROWB);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dstA + off), "r"(v.x),
-                       "r"(v.y), "r"(v.z), "r"(v.w)
-                       : "memory");
+          fence_proxy_async_smem();
+          mbar_arrive(bar(FULL + stage));
+        } else {
+          const uint8_t* src = p.K + (c >= 0 ? c : 0) * D * 2;
+#pragma unroll
+          for (int u = 0; u < UPR; ++u) {
+            const uint32_t off = (u / UPC) * L::A_CHUNK + swz_offset(tid, u % UPC, L::ROWB);
+            cp_async16(dstA + off, src + u * 16, c >= 0 ? 16u : 0u);
+          }
+          cp_async_mbar_arrive_noinc(bar(FULL + stage));
         }
-        fence_proxy_async_smem();
-        mbar_arrive(bar(FULL + stage));
         if (++stage == L::STAGES) {
           stage = 0;
           phase ^= 1;
@@ -177,6 +214,7 @@ rerank_scores_kernel(const RerankParams p) {
           ok = mbar_wait(bar(FULL + stage), phase, abort_flag, p.ctl) &&
                mbar_wait(bar(ACCEMPTY + acc), accph ^ 1, abort_flag, p.ctl);
           if (!ok) break;
+          fence_proxy_async_smem();  // copies observed through the barrier -> MMA operand reads
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NB);
 #pragma unroll
@@ -219,6 +257,17 @@ rerank_scores_kernel(const RerankParams p) {
       for (int i = lane; i < NB; i += 32)
         w_s[i] = i < p.H ? __ldg(p.w + static_cast<int64_t>(t) * p.H + i) : 0.0f;
       __syncwarp();
+      // this lane's candidate of each tile, loaded two tiles ahead (and, for
+      // FP8 keys, its scale one tile ahead) so no tile waits on them
+      const int32_t* crow = p.cand + static_cast<int64_t>(t) * p.kp;
+      auto cand_of = [&](int tile) -> int64_t {
+        const int i = tile * kCand + quad * 32 + lane;
+        if (tile >= tiles || i >= p.kp) return -1;
+        const int64_t c = __ldg(crow + i);
+        return (c >= 0 && c <= pos && c < p.n_k) ? c : -1;
+      };
+      int64_t c_cur = cand_of(0), c_nxt = cand_of(1);
+      float ks_cur = (FP8 && c_cur >= 0) ? __ldg(p.k_scale + c_cur) : 1.0f;
       for (int tile = 0; tile < tiles; ++tile) {
         if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -226,7 +275,7 @@ rerank_scores_kernel(const RerankParams p) {
         tc_fence_after();
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                static_cast<uint32_t>(acc * NB);
-        float sum = 0.0f;
+        float2 a0 = make_float2(0.0f, 0.0f), a1 = make_float2(0.0f, 0.0f);
         if (NB >= 32) {
 #pragma unroll 1
           for (int c = 0; c < NB / 32; ++c) {
@@ -234,15 +283,28 @@ rerank_scores_kernel(const RerankParams p) {
             tmem_ld32(tbase + static_cast<uint32_t>(c * 32), v);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) sum = fmaf(w_s[c * 32 + e], relu(__uint_as_float(v[e])), sum);
+            for (int e = 0; e < 32; e += 4) {
+              const float4 w4 = *reinterpret_cast<const float4*>(w_s + c * 32 + e);
+              a0 = fma2(make_float2(w4.x, w4.y),
+                        make_float2(relu(__uint_as_float(v[e])), relu(__uint_as_float(v[e + 1]))), a0);
+              a1 = fma2(make_float2(w4.z, w4.w),
+                        make_float2(relu(__uint_as_float(v[e + 2])), relu(__uint_as_float(v[e + 3]))), a1);
+            }
           }
         } else {
           uint32_t v[16];
           tmem_ld16(tbase, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) sum = fmaf(w_s[e], relu(__uint_as_float(v[e])), sum);
+          for (int e = 0; e < 16; e += 4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(w_s + e);
+            a0 = fma2(make_float2(w4.x, w4.y),
+                      make_float2(relu(__uint_as_float(v[e])), relu(__uint_as_float(v[e + 1]))), a0);
+            a1 = fma2(make_float2(w4.z, w4.w),
+                      make_float2(relu(__uint_as_float(v[e + 2])), relu(__uint_as_float(v[e + 3]))), a1);
+          }
         }
+        const float sum = (a0.x + a0.y) + (a1.x + a1.y);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
@@ -251,12 +313,12 @@ rerank_scores_kernel(const RerankParams p) {
           accph ^= 1;
         }
         const int i = tile * kCand + quad * 32 + lane;
-        if (i < p.kp) {
-          const int64_t c = __ldg(p.cand + static_cast<int64_t>(t) * p.kp + i);
-          float out = -INFINITY;
-          if (c >= 0 && c <= pos && c < p.n_k) out = FP8 ? sum * __ldg(p.k_scale + c) : sum;
-          p.full[static_cast<int64_t>(t) * p.ldf + i] = out;
-        }
+        if (i < p.kp)
+          p.full[static_cast<int64_t>(t) * p.ldf + i] =
+              c_cur >= 0 ? (FP8 ? sum * ks_cur : sum) : -INFINITY;
+        c_cur = c_nxt;
+        c_nxt = cand_of(tile + 2);
+        ks_cur = (FP8 && c_cur >= 0) ? __ldg(p.k_scale + c_cur) : 1.0f;
       }
       __syncwarp();  // w_s is rewritten for the next query
     }

@@ -178,10 +178,15 @@ struct Sched {
   }
 };
 
-template <int D, int HT, bool FP8, bool SEL>
-__global__ void __maxnreg__((Epi<HT, FP8>::MAXREG))
+// Key modes: KM 0 = bf16 keys; KM 1 = FP8 E4M3 keys decoded by converter
+// warps in the kernel; KM 2 = FP8 keys already decoded to bf16 (exact) by the
+// caller.  KM 1 and 2 multiply each logit by the key's scale.
+template <int D, int HT, int KM, bool SEL>
+__global__ void __maxnreg__((Epi<HT, KM == 1>::MAXREG))
 score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap lmap,
                     const ScoreParams p) {
+  constexpr bool FP8 = KM == 1;  // converter warps
+  constexpr bool KSC = KM != 0;  // per-key scale
   using L = ScoreLayout<D, HT, FP8, SEL>;
   static_assert(!SEL || HT >= 4, "select mode needs h >= 4");
   if (p.gate && *p.gate == 0) return;  // repair launch with nothing to repair
@@ -479,7 +484,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           }
           sums[qq] = a2.x + a2.y;
         }
-        if constexpr (FP8) {
+        if constexpr (KSC) {
           // per-token scale > 0: w * ReLU(scale * dot) = scale * w * ReLU(dot)
           const float ks = s_ok ? __ldg(p.k_scale + s) : 0.0f;
 #pragma unroll
@@ -536,7 +541,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
             const float2 w2 = *reinterpret_cast<const float2*>(w_s + qq * 2);
             sum = fmaf(w2.y, relu(__uint_as_float(v[qq * 2 + 1])), w2.x * relu(__uint_as_float(v[qq * 2])));
           }
-          if constexpr (FP8) sum *= s_ok ? __ldg(p.k_scale + s) : 0.0f;
+          if constexpr (KSC) sum *= s_ok ? __ldg(p.k_scale + s) : 0.0f;
           const int64_t t = tq0 + qq;
           if (t < p.n_q && s_ok) *dst = (s <= p.q_pos0 + t) ? sum : -INFINITY;
           dst += p.ld;
@@ -553,8 +558,9 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
   }
 }
 
-template <int D, int HT, bool FP8, bool SEL>
+template <int D, int HT, int KM, bool SEL>
 cudaError_t launch_dhs(const ScoreParams& p, const CUtensorMap& map, cudaStream_t s) {
+  constexpr bool FP8 = KM == 1;
   using L = ScoreLayout<D, HT, FP8, SEL>;
   // fused-logit store map: [n_q rows][n_k keys] fp32 with row pitch ld, box 128 keys x QG queries
   CUtensorMap lmap;
@@ -568,7 +574,7 @@ cudaError_t launch_dhs(const ScoreParams& p, const CUtensorMap& map, cudaStream_
                           CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = score_tokens_kernel<D, HT, FP8, SEL>;
+  auto kern = score_tokens_kernel<D, HT, KM, SEL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   const int64_t grid = std::min<int64_t>(sm_count(), p.total_tiles);
@@ -577,27 +583,27 @@ cudaError_t launch_dhs(const ScoreParams& p, const CUtensorMap& map, cudaStream_
   return cudaGetLastError();
 }
 
-template <int D, bool FP8>
+template <int D, int KM>
 cudaError_t launch_d(const ScoreParams& p, int h, bool sel, const CUtensorMap& map, cudaStream_t s) {
   if (sel) {
     switch (h) {
-      case 4: return launch_dhs<D, 4, FP8, true>(p, map, s);
-      case 8: return launch_dhs<D, 8, FP8, true>(p, map, s);
-      case 16: return launch_dhs<D, 16, FP8, true>(p, map, s);
-      case 32: return launch_dhs<D, 32, FP8, true>(p, map, s);
-      case 64: return launch_dhs<D, 64, FP8, true>(p, map, s);
+      case 4: return launch_dhs<D, 4, KM, true>(p, map, s);
+      case 8: return launch_dhs<D, 8, KM, true>(p, map, s);
+      case 16: return launch_dhs<D, 16, KM, true>(p, map, s);
+      case 32: return launch_dhs<D, 32, KM, true>(p, map, s);
+      case 64: return launch_dhs<D, 64, KM, true>(p, map, s);
     }
     return cudaErrorNotSupported;
   }
   switch (h) {
-    case 1: return launch_dhs<D, 1, FP8, false>(p, map, s);
-    case 2: return launch_dhs<D, 2, FP8, false>(p, map, s);
-    case 4: return launch_dhs<D, 4, FP8, false>(p, map, s);
-    case 8: return launch_dhs<D, 8, FP8, false>(p, map, s);
-    case 16: return launch_dhs<D, 16, FP8, false>(p, map, s);
-    case 32: return launch_dhs<D, 32, FP8, false>(p, map, s);
-    case 64: return launch_dhs<D, 64, FP8, false>(p, map, s);
-    case 128: return launch_dhs<D, 128, FP8, false>(p, map, s);
+    case 1: return launch_dhs<D, 1, KM, false>(p, map, s);
+    case 2: return launch_dhs<D, 2, KM, false>(p, map, s);
+    case 4: return launch_dhs<D, 4, KM, false>(p, map, s);
+    case 8: return launch_dhs<D, 8, KM, false>(p, map, s);
+    case 16: return launch_dhs<D, 16, KM, false>(p, map, s);
+    case 32: return launch_dhs<D, 32, KM, false>(p, map, s);
+    case 64: return launch_dhs<D, 64, KM, false>(p, map, s);
+    case 128: return launch_dhs<D, 128, KM, false>(p, map, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -622,11 +628,11 @@ cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s
                 a.gate};
   CUtensorMap map;
   std::memset(&map, 0, sizeof map);
-  if (a.fp8) {  // converter warps read the e4m3 keys; no key tensor map
+  if (a.fp8 && !a.k_bf16) {  // converter warps read the e4m3 keys; no key tensor map
     switch (a.d) {
-      case 32: return launch_d<32, true>(p, a.h, sel, map, s);
-      case 64: return launch_d<64, true>(p, a.h, sel, map, s);
-      case 128: return launch_d<128, true>(p, a.h, sel, map, s);
+      case 32: return launch_d<32, 1>(p, a.h, sel, map, s);
+      case 64: return launch_d<64, 1>(p, a.h, sel, map, s);
+      case 128: return launch_d<128, 1>(p, a.h, sel, map, s);
     }
     return cudaErrorInvalidValue;
   }
@@ -638,10 +644,18 @@ cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s
                         rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) !=
       CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  if (a.fp8) {  // decoded FP8 keys: bf16 operand, per-key scale in the epilogue
+    switch (a.d) {
+      case 32: return launch_d<32, 2>(p, a.h, sel, map, s);
+      case 64: return launch_d<64, 2>(p, a.h, sel, map, s);
+      case 128: return launch_d<128, 2>(p, a.h, sel, map, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (a.d) {
-    case 32: return launch_d<32, false>(p, a.h, sel, map, s);
-    case 64: return launch_d<64, false>(p, a.h, sel, map, s);
-    case 128: return launch_d<128, false>(p, a.h, sel, map, s);
+    case 32: return launch_d<32, 0>(p, a.h, sel, map, s);
+    case 64: return launch_d<64, 0>(p, a.h, sel, map, s);
+    case 128: return launch_d<128, 0>(p, a.h, sel, map, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -138,3 +138,27 @@ def test_score_topk_repairs_unrepresentative_sample(lib):
     want, _ = _unfused(lib, Qg, wg, heads, Kg, q_pos0, k)
     assert np.array_equal(got, want)
     assert flags[0] == 1 and flags[1:].all()
+
+
+def test_score_topk_bursts_of_kept_logits(lib):
+    # runs of 64 consecutive high-scoring keys: their 32-key words keep more
+    # logits than a word's dense slot holds, so the rest go through the row
+    n_q, q_pos0, n_k, H, d, k, h = 64, 10000, 10100, 64, 128, 256, 8
+    rng = np.random.default_rng(23)
+    Q = (1.0 + 0.3 * rng.standard_normal((n_q, H, d))) / np.sqrt(d)
+    K = 0.5 * rng.standard_normal((n_k, d)) / np.sqrt(d)
+    for start in (1000, 5003, 9990):
+        K[start:start + 64] = rng.uniform(2.0, 3.0, size=(64, 1)) / np.sqrt(d)
+    w = np.full((n_q, H), 1.0 / H, dtype=np.float32)
+    Qg, Kg, wg = dev(W.bf16_bits(Q)), dev(W.bf16_bits(K)), dev(w)
+    _, hl = lib.misa_pool_keys(Kg, 128)
+    heads, _ = lib.misa_route_heads(Qg, wg, hl, q_pos0, n_k, 128, h)
+    got, flags = _fused(lib, Qg, wg, heads, Kg, q_pos0, k)
+    want, _ = _unfused(lib, Qg, wg, heads, Kg, q_pos0, k)
+    assert np.array_equal(got, want)
+    assert flags[0] == int(flags[1:].any())
+    for t in range(n_q):   # every burst key visible to row t is selected
+        vis = q_pos0 + t + 1
+        burst = [s for st in (1000, 5003, 9990) for s in range(st, st + 64) if s < vis]
+        assert set(burst) <= set(got[t].tolist())
+    print(f"rows repaired: {int(flags[1:].sum())} of {n_q}")
