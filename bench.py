@@ -44,9 +44,11 @@ from long_context_sparse_block_b200 import workloads as W  # noqa: E402
 METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor peak"
 
 # DRAM bytes (read + write) of one select-mode scoring launch over all 8192
-# queries of chunk_128k, from the ncu capture summarised under profiles/; valid
-# only for the kernel sources it was taken on (null otherwise).
-SCORE_TRAFFIC = {"sources_sha256_16": "", "bytes_per_launch": None, "queries": 8192}
+# queries of chunk_128k: the ncu capture of queries 0..1023 summarised in
+# profiles/score_select_chunk_128k.md, scaled by the query count; valid only for
+# the kernel sources it was taken on (null otherwise).
+SCORE_TRAFFIC = {"sources_sha256_16": "c019c7914cd0f127", "bytes_per_launch": 8 * (170.618112e6 + 120.406784e6),
+                 "queries": 8192}
 
 
 def _score_sources_digest():
@@ -87,7 +89,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -96,9 +98,18 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
-    def stop(self):
+    def wait_first(self, timeout=5.0):
+        """Blocks until nvidia-smi has produced its first sample (it starts slowly)."""
+        t0 = time.monotonic()
+        while self.proc is not None and not self.lines and time.monotonic() - t0 < timeout:
+            time.sleep(0.01)
+
+    def mark(self):
+        return time.monotonic()
+
+    def stop(self, t_begin=None, t_end=None):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -108,7 +119,11 @@ class ClockSampler:
             self.proc.kill()
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = [ln for t, ln in self.lines
+                 if t_begin is None or (t_begin <= t <= t_end + 0.05)]
+        if not lines and self.lines:  # nothing inside: the sample nearest the region
+            lines = [min(self.lines, key=lambda x: abs(x[0] - (t_begin or 0.0)))[1]]
+        for ln in lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -181,6 +196,16 @@ def cpu_baseline(wl: W.Workload, h: int, inp: dict, budget_s: float = 15.0) -> d
 
 # ------------------------------------------------------------------ GPU arm
 
+def _workload(args):
+    """The named workload, cut to its first --queries queries when given (for
+    small profiling captures; the keys and query positions are unchanged)."""
+    import dataclasses
+    wl = W.WORKLOADS[args.workload]
+    if args.queries and args.queries < wl.n_q:
+        wl = dataclasses.replace(wl, n_q=args.queries)
+    return wl
+
+
 def run_ours(args, rank, world, local_rank, inp):
     import torch
     import torch.distributed as dist
@@ -189,7 +214,7 @@ def run_ours(args, rank, world, local_rank, inp):
     from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
 
     torch.cuda.set_device(local_rank)
-    wl = W.WORKLOADS[args.workload]
+    wl = _workload(args)
     h = args.h or wl.h
     if world > 1:
         rng = np.random.default_rng(1000 + rank)
@@ -240,13 +265,15 @@ def run_ours(args, rank, world, local_rank, inp):
     for _ in range(args.warmup):
         flush.zero_()
         step(False)
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+        clocks.wait_first()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local_rank)
-    if rank == 0:
-        clocks.start()
+    t_begin = time.monotonic()
     _lib.misa_profile_start()
     spans = []
     for _ in range(args.steps):
@@ -256,7 +283,8 @@ def run_ours(args, rank, world, local_rank, inp):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clk = clocks.stop() if rank == 0 else None
+    t_end = time.monotonic()
+    clk = clocks.stop(t_begin, t_end) if rank == 0 else None
     fused_stages = _lib.misa_profile_stop()
     repaired = int(ix.ws_sel[4:4 * (ix.sub + 1)].view(torch.int32).sum()) if fused else None
     assert _lib.misa_last_device_status() == 0, "device status"
@@ -473,13 +501,15 @@ def run_reference(args, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="chunk_128k")
     ap.add_argument("--h", type=int, default=0)
     ap.add_argument("--sub-chunk", type=int, default=8192)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--queries", type=int, default=0,
+                    help="index only the first N queries of the chunk (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
     ap.add_argument("--no-variants", action="store_true",
@@ -498,8 +528,10 @@ def main():
         return
 
     # the oracle's process pool is spawned before any CUDA work
-    wl = W.WORKLOADS[args.workload]
-    inp = W.generate(wl)  # each rank indexes its own chunk (same shape)
+    wl = _workload(args)
+    inp = W.generate(W.WORKLOADS[args.workload])  # each rank indexes its own chunk (same shape)
+    if wl.n_q < inp["Q"].shape[0]:
+        inp["Q"], inp["w"] = inp["Q"][:wl.n_q].copy(), inp["w"][:wl.n_q].copy()
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl, args.h or wl.h, inp, budget_s=args.cpu_budget)
