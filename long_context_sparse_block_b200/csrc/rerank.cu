@@ -129,11 +129,11 @@ rerank_scores_kernel(const RerankParams p) {
       fence_proxy_async_smem();
       mbar_arrive(bar(BFULL));
       ++qcount;
-      // each producer thread owns one candidate row of every tile: its index
-      // is loaded a tile ahead, and the row's copies are all in flight at once
-      // (bf16: asynchronous 16-byte copies that arrive on the stage barrier when
-      // they land; FP8: the codes of the next tile's row are loaded while this
-      // tile's are decoded)
+      // each producer thread holds one candidate of every tile, loaded a tile
+      // ahead; all of a tile's copies are in flight at once (bf16: asynchronous
+      // 16-byte copies, whole rows per warp instruction, arriving on the stage
+      // barrier when they land; FP8: each thread loads its own row's codes for
+      // the next tile while decoding this tile's)
       const int32_t* crow = p.cand + static_cast<int64_t>(t) * p.kp;
       auto cand_of = [&](int tile) -> int64_t {
         const int i = tile * kCand + tid;
@@ -187,11 +187,18 @@ rerank_scores_kernel(const RerankParams p) {
           fence_proxy_async_smem();
           mbar_arrive(bar(FULL + stage));
         } else {
-          const uint8_t* src = p.K + (c >= 0 ? c : 0) * D * 2;
+          // warp w copies rows 32w..32w+31, UPR lanes per row so that one
+          // instruction reads whole rows (full 128-byte lines); lane i holds the
+          // candidate of row 32w+i
+          constexpr int RPI = 32 / UPR;  // rows per instruction
+          const int wr0 = tid & ~31;
 #pragma unroll
-          for (int u = 0; u < UPR; ++u) {
-            const uint32_t off = (u / UPC) * L::A_CHUNK + swz_offset(tid, u % UPC, L::ROWB);
-            cp_async16(dstA + off, src + u * 16, c >= 0 ? 16u : 0u);
+          for (int j = 0; j < UPR; ++j) {
+            const int rr = j * RPI + lane / UPR;
+            const int u = lane % UPR;
+            const int64_t cr = __shfl_sync(0xffffffffu, c, rr);
+            const uint32_t off = (u / UPC) * L::A_CHUNK + swz_offset(wr0 + rr, u % UPC, L::ROWB);
+            cp_async16(dstA + off, p.K + ((cr >= 0 ? cr : 0) * D + u * 8) * 2, cr >= 0 ? 16u : 0u);
           }
           cp_async_mbar_arrive_noinc(bar(FULL + stage));
         }
