@@ -14,16 +14,17 @@
 // ReLU * w over the H columns of its own lane.  The work is bound by the gather
 // from L2, not by the MMA.
 //
-// Warp roles (288 threads): warps 0-3 gather producers, warp 4 TMEM allocator
-// and MMA issuer, warps 5-8 epilogue.  Queries are distributed round-robin over
-// a persistent grid.
+// Warp roles (416 threads): warps 0-3 gather producers, warp 4 TMEM allocator
+// and MMA issuer, warps 5-12 epilogue in two groups of four: group g takes the
+// tiles of accumulator g (even / odd tiles of the CTA's sequence).  Queries are
+// distributed round-robin over a persistent grid.
 #include "internal.h"
 
 namespace misa {
 namespace {
 
 constexpr int kCand = 128;  // MMA M: candidates per tile
-constexpr int kRerankThreads = 288;
+constexpr int kRerankThreads = 416;
 constexpr int kProducers = 128;
 constexpr uint64_t kDrainNs = 2000000;
 
@@ -37,8 +38,8 @@ struct RerankLayout {
   static constexpr int STAGES = 4;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_W = OFF_B + ((B_BYTES + 1023) / 1024) * 1024;  // 4 warps x NB floats
-  static constexpr int OFF_BAR = OFF_W + 4 * NB * 4;
+  static constexpr int OFF_W = OFF_B + ((B_BYTES + 1023) / 1024) * 1024;  // 8 warps x NB floats
+  static constexpr int OFF_BAR = OFF_W + 8 * NB * 4;
   static constexpr int NBAR = 2 * STAGES + 6;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
@@ -255,17 +256,19 @@ rerank_scores_kernel(const RerankParams p) {
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
+    const int grp = (warp - 5) >> 2;  // accumulator (and tile parity) of this group
     float* w_s = reinterpret_cast<float*>(smem + L::OFF_W) + (warp - 5) * NB;
-    int acc = 0;
     uint32_t accph = 0;
+    int64_t gtile = 0;  // tiles of the CTA's sequence before this query
     bool ok = true;
     for (int t = blockIdx.x; t < p.n_q && ok; t += gridDim.x) {
       const int64_t pos = p.q_pos0 + t;
       for (int i = lane; i < NB; i += 32)
         w_s[i] = i < p.H ? __ldg(p.w + static_cast<int64_t>(t) * p.H + i) : 0.0f;
       __syncwarp();
-      // this lane's candidate of each tile, loaded two tiles ahead (and, for
-      // FP8 keys, its scale one tile ahead) so no tile waits on them
+      // this lane's candidate of each of the group's tiles, loaded two tiles
+      // ahead (and, for FP8 keys, its scale one tile ahead)
+      const int first = static_cast<int>((grp - gtile % 2 + 2) % 2);
       const int32_t* crow = p.cand + static_cast<int64_t>(t) * p.kp;
       auto cand_of = [&](int tile) -> int64_t {
         const int i = tile * kCand + quad * 32 + lane;
@@ -273,15 +276,15 @@ rerank_scores_kernel(const RerankParams p) {
         const int64_t c = __ldg(crow + i);
         return (c >= 0 && c <= pos && c < p.n_k) ? c : -1;
       };
-      int64_t c_cur = cand_of(0), c_nxt = cand_of(1);
+      int64_t c_cur = cand_of(first), c_nxt = cand_of(first + 2);
       float ks_cur = (FP8 && c_cur >= 0) ? __ldg(p.k_scale + c_cur) : 1.0f;
-      for (int tile = 0; tile < tiles; ++tile) {
-        if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
+      for (int tile = first; tile < tiles; tile += 2) {
+        if (lane == 0) ok = mbar_wait(bar(ACCFULL + grp), accph, abort_flag, p.ctl);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                               static_cast<uint32_t>(acc * NB);
+                               static_cast<uint32_t>(grp * NB);
         float2 a0 = make_float2(0.0f, 0.0f), a1 = make_float2(0.0f, 0.0f);
         if (NB >= 32) {
 #pragma unroll 1
@@ -314,19 +317,17 @@ rerank_scores_kernel(const RerankParams p) {
         const float sum = (a0.x + a0.y) + (a1.x + a1.y);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
-        if (++acc == 2) {
-          acc = 0;
-          accph ^= 1;
-        }
+        if (lane == 0) mbar_arrive(bar(ACCEMPTY + grp));
+        accph ^= 1;
         const int i = tile * kCand + quad * 32 + lane;
         if (i < p.kp)
           p.full[static_cast<int64_t>(t) * p.ldf + i] =
               c_cur >= 0 ? (FP8 ? sum * ks_cur : sum) : -INFINITY;
         c_cur = c_nxt;
-        c_nxt = cand_of(tile + 2);
+        c_nxt = cand_of(tile + 4);
         ks_cur = (FP8 && c_cur >= 0) ? __ldg(p.k_scale + c_cur) : 1.0f;
       }
+      gtile += tiles;
       __syncwarp();  // w_s is rewritten for the next query
     }
   }

@@ -494,20 +494,41 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           // fused top-k: a logit at or above its row's threshold is stored in
           // place and flagged in the row's pass mask (one word per 32 keys);
           // the others are neither stored nor flagged
-          const int64_t cut64 = s - p.q_pos0 - tq0;  // query qq is causal for key s iff qq >= cut
-          const int cut = static_cast<int>(cut64 < 0 ? 0 : (cut64 > QPW ? QPW : cut64));
           const int64_t rows_left = p.n_q - tq0;
           const int q_end = static_cast<int>(rows_left < QPW ? rows_left : QPW);
-          const uint32_t valid = s_ok ? (((1u << q_end) - 1u) & ~((1u << cut) - 1u)) : 0u;
-          uint32_t mine = 0u;  // lane qq: the mask word of query qq
+          // the warp's 32 keys are causal for all its queries and inside n_k: no
+          // per-query validity test (every tile but the diagonal and edge ones)
+          const int64_t s_last = it.kt * kTileKeys + quad * 32 + 31;
+          const bool full = s_last <= p.q_pos0 + tq0 && s_last < p.n_k && q_end == QPW;
+          uint32_t m[QPW];
+          if (full) {
 #pragma unroll
-          for (int qq = 0; qq < QPW; ++qq) {
-            const bool pass = ((valid >> qq) & 1u) && sums[qq] >= tau_s[qq];
-            const uint32_t m = __ballot_sync(0xffffffffu, pass);
-            if (lane == qq) mine = m;
-            if (pass) *dst = sums[qq];
-            dst += p.ld;
+            for (int qq = 0; qq < QPW; ++qq) {
+              const bool pass = sums[qq] >= tau_s[qq];
+              m[qq] = __ballot_sync(0xffffffffu, pass);
+              if (pass) *dst = sums[qq];
+              dst += p.ld;
+            }
+          } else {
+            const int64_t cut64 = s - p.q_pos0 - tq0;  // query qq is causal for key s iff qq >= cut
+            const int cut = static_cast<int>(cut64 < 0 ? 0 : (cut64 > QPW ? QPW : cut64));
+            const uint32_t valid = s_ok ? (((1u << q_end) - 1u) & ~((1u << cut) - 1u)) : 0u;
+#pragma unroll
+            for (int qq = 0; qq < QPW; ++qq) {
+              const bool pass = ((valid >> qq) & 1u) && sums[qq] >= tau_s[qq];
+              m[qq] = __ballot_sync(0xffffffffu, pass);
+              if (pass) *dst = sums[qq];
+              dst += p.ld;
+            }
           }
+          // lane qq stores the mask word of query qq (a select tree on the lane bits)
+          uint32_t mine = m[0];
+#pragma unroll
+          for (int bit = 1; bit < QPW; bit <<= 1) {
+#pragma unroll
+            for (int qq = 0; qq < QPW; qq += 2 * bit) m[qq] = (lane & bit) ? m[qq + bit] : m[qq];
+          }
+          mine = m[0];
           if (lane < q_end)
             p.mask[(tq0 + lane) * p.mask_ld + it.kt * (kTileKeys / 32) + quad] = mine;
         } else {
