@@ -341,11 +341,7 @@ def run_ours(args, rank, world, local_rank, inp):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        Q.copy_(Qh, non_blocking=True)
-        K.copy_(Kh, non_blocking=True)
-        w.copy_(wh, non_blocking=True)
-        out = ix.run(Q, K, w)
-        idx_h.copy_(out, non_blocking=True)
+        ix.run_host(Qh, Kh, wh, out=idx_h)   # copies in, indexes, copies out (overlapped)
         b.record(stream)
         b.synchronize()
         if i >= args.warmup:

@@ -58,6 +58,18 @@ class MisaIndexer:
         else:
             self.final = self.sel
 
+    def _select(self, c0, c1, Q, K, w, k_scale):
+        """Scoring, top-k (and the MISA-dagger rerank) of queries c0..c1-1 whose
+        heads are routed; Q and w hold the whole chunk's rows."""
+        s = self.shape
+        heads = None if s.dense else self.heads[c0:c1]
+        _lib.misa_score_topk(Q[c0:c1], w[c0:c1], heads, K, s.q_pos0 + c0, self.sel.shape[1],
+                             k_scale=k_scale, h=s.h, idx=self.sel[c0:c1],
+                             logits=self.logits[:c1 - c0], ws=self.ws_sel)
+        if s.kp:
+            _lib.misa_rerank(Q[c0:c1], w[c0:c1], K, self.sel[c0:c1], s.q_pos0 + c0, s.k,
+                             k_scale=k_scale, idx=self.final[c0:c1], ws=self.ws)
+
     def run(self, Q, K, w, k_scale=None, on_subchunk=None):
         """Q [n_q,H,d] bf16 codes, K [n_k,d] bf16 codes (or e4m3 + k_scale), w [n_q,H] f32.
         Returns the selected token indices [n_q, k] (int32, ascending, -1 padded).
@@ -70,19 +82,72 @@ class MisaIndexer:
             _lib.misa_route_heads(Q, w, self.kbar_hl, s.q_pos0, s.n_k, s.B, s.h, heads=self.heads)
         for c0 in range(0, s.n_q, self.sub):
             c1 = min(s.n_q, c0 + self.sub)
-            n = c1 - c0
-            lg = self.logits[:n]
-            heads = None if s.dense else self.heads[c0:c1]
             if on_subchunk is None:
-                _lib.misa_score_topk(Q[c0:c1], w[c0:c1], heads, K, s.q_pos0 + c0,
-                                     self.sel.shape[1], k_scale=k_scale, h=s.h,
-                                     idx=self.sel[c0:c1], logits=lg, ws=self.ws_sel)
-            else:
-                _lib.misa_score_tokens(Q[c0:c1], w[c0:c1], heads, K, s.q_pos0 + c0,
-                                       k_scale=k_scale, logits=lg, h=s.h)
-                on_subchunk(c0, c1, lg)
-                _lib.misa_topk(lg, s.q_pos0 + c0, s.n_k, self.sel.shape[1], idx=self.sel[c0:c1])
+                self._select(c0, c1, Q, K, w, k_scale)
+                continue
+            lg = self.logits[:c1 - c0]
+            heads = None if s.dense else self.heads[c0:c1]
+            _lib.misa_score_tokens(Q[c0:c1], w[c0:c1], heads, K, s.q_pos0 + c0,
+                                   k_scale=k_scale, logits=lg, h=s.h)
+            on_subchunk(c0, c1, lg)
+            _lib.misa_topk(lg, s.q_pos0 + c0, s.n_k, self.sel.shape[1], idx=self.sel[c0:c1])
             if s.kp:
                 _lib.misa_rerank(Q[c0:c1], w[c0:c1], K, self.sel[c0:c1], s.q_pos0 + c0, s.k,
                                  k_scale=k_scale, idx=self.final[c0:c1], ws=self.ws)
         return self.final
+
+    def run_host(self, Qh, Kh, wh, out=None, k_scale_h=None, pieces: int = 4):
+        """End to end from host buffers (pin them for asynchronous copies): Q, K, w
+        (and FP8 key scales) as in run(); returns the selected indices in `out`, a
+        pinned host int32 [n_q, k] tensor (allocated when None), complete when the
+        current stream reaches this point.  The queries go in `pieces` pieces on
+        three streams (copy in, index, copy out) so that the copies of one piece
+        overlap the indexing of another; the keys go first."""
+        s = self.shape
+        dev = self.heads.device
+        if getattr(self, "_dev", None) is None:
+            self._dev = (torch.empty(Qh.shape, dtype=Qh.dtype, device=dev),
+                         torch.empty(Kh.shape, dtype=Kh.dtype, device=dev),
+                         torch.empty(wh.shape, dtype=wh.dtype, device=dev),
+                         None if k_scale_h is None else
+                         torch.empty(k_scale_h.shape, dtype=k_scale_h.dtype, device=dev))
+            self._streams = (torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev))
+        Q, K, w, ks = self._dev
+        cin, cout = self._streams
+        if out is None:
+            out = torch.empty(tuple(self.final.shape), dtype=torch.int32, pin_memory=True)
+        compute = torch.cuda.current_stream(dev)
+        cin.wait_stream(compute)   # the device buffers are free again
+        cout.wait_stream(compute)
+        step = -(-s.n_q // max(1, pieces))
+        bounds = [(c0, min(s.n_q, c0 + step)) for c0 in range(0, s.n_q, step)]
+        ev_in = []
+        with torch.cuda.stream(cin):
+            K.copy_(Kh, non_blocking=True)
+            if ks is not None:
+                ks.copy_(k_scale_h, non_blocking=True)
+            ev_k = torch.cuda.Event()
+            ev_k.record(cin)
+            for c0, c1 in bounds:
+                Q[c0:c1].copy_(Qh[c0:c1], non_blocking=True)
+                w[c0:c1].copy_(wh[c0:c1], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(cin)
+                ev_in.append(e)
+        compute.wait_event(ev_k)
+        if not s.dense:
+            _lib.misa_pool_keys(K, s.B, k_scale=ks, kbar_hl=self.kbar_hl, want_kbar=False)
+        for (c0, c1), e in zip(bounds, ev_in):
+            compute.wait_event(e)
+            if not s.dense:
+                _lib.misa_route_heads(Q[c0:c1], w[c0:c1], self.kbar_hl, s.q_pos0 + c0, s.n_k,
+                                      s.B, s.h, heads=self.heads[c0:c1])
+            for a0 in range(c0, c1, self.sub):
+                self._select(a0, min(c1, a0 + self.sub), Q, K, w, ks)
+            done = torch.cuda.Event()
+            done.record(compute)
+            cout.wait_event(done)
+            with torch.cuda.stream(cout):
+                out[c0:c1].copy_(self.final[c0:c1], non_blocking=True)
+        compute.wait_stream(cout)
+        return out

@@ -162,3 +162,22 @@ def test_score_topk_bursts_of_kept_logits(lib):
         burst = [s for st in (1000, 5003, 9990) for s in range(st, st + 64) if s < vis]
         assert set(burst) <= set(got[t].tolist())
     print(f"rows repaired: {int(flags[1:].sum())} of {n_q}")
+
+
+@pytest.mark.parametrize("kp", [0, 1024])
+def test_indexer_host_pipeline_equals_device_run(lib, kp):
+    # run_host (copies of one query piece overlapping the indexing of another)
+    # gives what run gives on device-resident inputs
+    from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
+    n_q, q_pos0, n_k, H, d, B, h, k = 600, 20000, 24000, 64, 128, 128, 8, 256
+    wl, inp, g = _inputs(n_q, q_pos0, n_k, H, d, B, h, k, seed=31)
+    shape = IndexerShape(n_q, q_pos0, n_k, H, d, B, h, k, kp=kp, sub_chunk=256)
+    want = MisaIndexer(shape).run(g["Q"], g["K"], g["w"]).cpu().numpy()
+    ix = MisaIndexer(shape)
+    Qh = torch.from_numpy(np.ascontiguousarray(inp["Q"]).view(np.int16)).pin_memory()
+    Kh = torch.from_numpy(np.ascontiguousarray(inp["K"]).view(np.int16)).pin_memory()
+    wh = torch.from_numpy(inp["w"]).pin_memory()
+    for pieces in (1, 3):
+        out = ix.run_host(Qh, Kh, wh, pieces=pieces)
+        torch.cuda.current_stream().synchronize()
+        assert np.array_equal(out.numpy(), want)
