@@ -40,12 +40,11 @@ constexpr int kTopkThreads = 256;
 constexpr int kWarps = kTopkThreads / 32;
 constexpr int kBins1 = 4096;
 constexpr int kChunk = 4 * kTopkThreads;  // entries per block-wide step
-constexpr int kFastMaxK = 4096;           // largest k of the fast path
+constexpr int kFastMaxK = 12288;          // largest k of the fast path
 constexpr int kSampleTarget = 4096;       // sampled entries per row (at most)
 constexpr int kFastCap = 5120;            // list entries of the fast path (all warps)
 constexpr int kCtasPerSm = 3;             // resident CTAs the fast path is sized for
 constexpr double kSampleMargin = 1.4;     // list target: ~1.4 k entries above tau
-constexpr int kRegion = kFastCap / kWarps;  // list entries per warp region
 constexpr int kEqMax = 1024;              // entries equal to the k-th key (fast path)
 
 struct TopkParams {
@@ -263,12 +262,14 @@ struct RegionSrc {
   const uint32_t* keys;
   const uint32_t* poss;
   const uint32_t* counts;  // [kWarps]
-  int64_t n;               // kWarps * kRegion
+  int64_t n;               // kWarps * region
+  uint32_t region;         // entries per warp region
+  uint32_t inv;            // ceil(2^32 / region): x / region = umulhi(x, inv) for x < 2^16
   __device__ __forceinline__ void load4(int64_t i0, uint32_t (&key)[4], uint32_t (&pos)[4]) const {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const uint32_t x = static_cast<uint32_t>(i0) + e;
-      const uint32_t w = x / kRegion, j = x % kRegion;
+      const uint32_t w = __umulhi(x, inv), j = x - w * region;
       const bool in = x < static_cast<uint32_t>(n) && j < counts[w];
       key[e] = in ? keys[x] : 0u;
       pos[e] = in ? poss[x] : 0u;
@@ -350,8 +351,8 @@ __device__ void emit_bitmap(const uint32_t* bitmap, uint32_t words, const OutEmi
 }
 
 // Fast path.  Returns false (and writes nothing) when the row must take the
-// fallback path.  Shared memory: hist [kBins1], list keys/poss [kFastCap],
-// sel [kFastMaxK], counts [kWarps].
+// fallback path.  Shared memory: hist [kBins1], list keys/poss [cap] (kFastCap
+// for k <= 4096, more for larger k), sel [kEqMax], counts [kWarps].
 __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit& out,
                           uint32_t* hist, uint32_t* lkeys, uint32_t* lposs, uint32_t* sel,
                           uint32_t* counts, SmemCtl& sc) {
@@ -363,7 +364,7 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   // 22-bit key bin holding the m-th largest sampled key; tau_retry, used when
   // the list comes out short, is the same for the 2m-th.
   uint32_t tau = 1u, tau_retry = 1u;
-  if (n > kFastCap) {
+  if (n > p.cap) {
     constexpr int kBlocks = kSampleTarget / 128;
     const int64_t gap = (n / kBlocks) & ~static_cast<int64_t>(3);   // keeps float4 alignment
     for (int i = threadIdx.x; i < kSampleTarget / 4; i += kTopkThreads) {
@@ -410,6 +411,7 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
     }
     __syncthreads();
   }
+  const uint32_t region = static_cast<uint32_t>(p.cap / kWarps);  // list entries per warp
   uint32_t total = 0;
   for (int attempt = 0; attempt < 2; ++attempt) {
   // ---- one pass: warp-compacted append of every key >= tau.  The test runs on
@@ -422,8 +424,8 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   }
   uint32_t cnt = 0;  // this warp's entries (warp-uniform)
   bool overflow = false;
-  uint32_t* wk = lkeys + warp * kRegion;
-  uint32_t* wp = lposs + warp * kRegion;
+  uint32_t* wk = lkeys + warp * region;
+  uint32_t* wp = lposs + warp * region;
   const uint32_t lt_mask = (1u << lane) - 1u;
   const int64_t nfull = src.aligned ? n / 128 : 0;   // chunks read without bounds checks
   const int64_t nchunks = (n + 127) / 128;
@@ -435,7 +437,7 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
       const uint32_t m = __ballot_sync(0xffffffffu, pass);
       if (m == 0u) continue;
       const uint32_t tot = __popc(m);
-      if (cnt + tot > static_cast<uint32_t>(kRegion)) {
+      if (cnt + tot > region) {
         overflow = true;
         continue;
       }
@@ -483,7 +485,8 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   tau = tau_retry;
   __syncthreads();
   }  // attempts
-  const RegionSrc rs{lkeys, lposs, counts, static_cast<int64_t>(kWarps) * kRegion};
+  const uint32_t inv = static_cast<uint32_t>((0x100000000ull + region - 1) / region);
+  const RegionSrc rs{lkeys, lposs, counts, static_cast<int64_t>(kWarps) * region, region, inv};
   // ---- exact k-th key within the list
   uint32_t T = 0u, need = 0u;
   if (total > k) T = kth_largest(rs, k, hist, sc, need);
@@ -496,7 +499,7 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   if (threadIdx.x == 0) *neq = 0u;
   __syncthreads();
   for (uint32_t x = threadIdx.x; x < static_cast<uint32_t>(rs.n); x += kTopkThreads) {
-    const uint32_t w = x / kRegion, j = x % kRegion;
+    const uint32_t w = __umulhi(x, inv), j = x - w * region;
     if (j >= counts[w]) continue;
     const uint32_t key = lkeys[x];
     const uint32_t pos = lposs[x];
@@ -756,9 +759,10 @@ cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, 
                         int row_len, const int32_t* cand, int k, int32_t* idx,
                         const DevCtl& ctl, cudaStream_t s, const int* gate) {
   if (n_q <= 0 || k <= 0) return cudaSuccess;
-  // list capacity: the fast path needs kFastCap; the fallback wants room for
-  // the entries in or above the k-th histogram bin
-  int cap = k <= kFastMaxK ? kFastCap : std::min(24576, ((2 * k + 4096) + 1023) / 1024 * 1024);
+  // list capacity: kFastCap for k <= 4096 (three CTAs per SM); larger k need
+  // room for ~1.4 k sampled-threshold entries (fast path) or for the entries in
+  // or above the k-th histogram bin (fallback)
+  int cap = k <= 4096 ? kFastCap : std::min(24576, ((2 * k + 4096) + 1023) / 1024 * 1024);
   const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * 8 +
                       (k <= kFastMaxK ? (kEqMax + kWarps) * 4 : 0);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -199,7 +199,7 @@ def _adversarial_rows(n, rng):
     return np.stack(rows)
 
 
-@pytest.mark.parametrize("k", [1, 7, 64, 2048, 4096, 16384])
+@pytest.mark.parametrize("k", [1, 7, 64, 2048, 4096, 8192, 12288, 16384])
 def test_topk_adversarial_rows(lib, k):
     rng = np.random.default_rng(k)
     n = 40000
