@@ -728,7 +728,7 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
   }
   __syncthreads();
   const float* row = logits + static_cast<int64_t>(t) * ld;
-  constexpr int kBatch = 8;
+  constexpr int kBatch = 16;
   for (uint32_t b0 = 0; b0 < total; b0 += kBatch * kTopkThreads) {
     float v[kBatch];
 #pragma unroll
