@@ -16,20 +16,27 @@
 // columns: ReLU, the head weights and the head-sum are applied in registers and
 // only the fused logit is written to HBM (per-head logits never leave the SM).
 //
-// Warp roles (576 threads for h <= 64, else 320; one CTA per SM, persistent):
+// Warp roles (608 threads for h <= 64, else 352, plus a warp for FP8 keys
+// decoded in the kernel; one CTA per SM, persistent):
 //   warp 0     producer: gathers B for each query group (16-byte cp.async into
 //              the 128-byte-swizzled K-major layout) and streams key tiles with
 //              TMA into a STAGES-deep ring;
 //   warp 1     allocates TMEM (512 columns = two 256-column accumulators) and
 //              issues tcgen05.mma from one thread;
-//   warp 2     issues one TMA store per tile of the logits the epilogue staged
-//              in shared memory (double-buffered);
-//   warps 3-   epilogue, four warps per TMEM lane quadrant each owning 64 of
+//   warp 2     store mode: issues one TMA store per tile of the logits the
+//              epilogue staged in shared memory (double-buffered);
+//   (warp 3    FP8 keys decoded here: e4m3 rows -> bf16 into the key tile;)
+//   then       epilogue, four warps per TMEM lane quadrant each owning 64 of
 //              the 256 columns (two warps owning 128 when h = 128): one
 //              tcgen05.ld of its columns, the accumulator released right after
 //              the load lands, then the fused ReLU * w head-sum (packed fp32
-//              FMA), causal mask and coalesced fp32 stores (a warp stores 32
-//              consecutive keys of one query row).
+//              FMA) and, per mode:
+//                store   the causal-masked logits staged for the TMA store;
+//                select  each logit compared with its row's threshold: a ballot
+//                        per query gives the row's 32-key pass-mask word, the
+//                        kept logits are stored in place (fused top-k);
+//                repair  store mode over only the query groups that hold a row
+//                        flagged by the fused top-k (nothing when none is).
 // Work is the flattened list of (query group, key tile) pairs, split evenly
 // over the CTAs, so causal triangles stay balanced.
 #include <cstring>

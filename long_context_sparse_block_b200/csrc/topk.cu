@@ -11,7 +11,7 @@
 // Values are mapped to order-preserving 32-bit keys (-0.0 folded onto +0.0,
 // -inf and padding to the reserved key 0).  One CTA per row.
 //
-// Fast path (k <= 4096, rows of at most 131072 entries):
+// Fast path (k <= 12288, rows of at most 131072 entries):
 //   sample   32 contiguous 128-entry blocks spread over the row; the lower
 //            edge of the 22-bit key bin holding the m-th largest sampled key,
 //            m ~ 1.4 k * (sample / row), becomes a threshold tau (the 2m-th
@@ -26,11 +26,16 @@
 //            exact k-th key T and how many entries equal to T are kept (the
 //            lowest positions); kept positions are set in a bitmap of the row
 //            and a block scan over its words writes them out in ascending order.
-// Fallback (sample too optimistic, list overflow, k > 4096, longer rows): a 4096-bin
+// Fallback (sample too optimistic, list overflow, k > 12288, longer rows): a 4096-bin
 // histogram pass, an ordered collection of the entries in or above the k-th
 // bin (block scans keep position order), the same radix refinement, and an
 // ordered selection pass — over the shared-memory list when it fits, else over
 // the row in global memory.
+//
+// Fused top-k helpers (used by misa_score_topk with the select-mode scoring):
+// a sample gather of 32 x 128 keys, a per-row threshold from the scored sample,
+// and the exact selection over the logits the select pass kept (pass-mask bits,
+// values in place), which flags rows it cannot finish for the exact repair.
 #include "internal.h"
 
 namespace misa {
