@@ -452,9 +452,11 @@ def _recall(sel, ref, n_k):
 
 
 def run_variants(wl, inp, stream, flush):
-    """The other measured configurations of the chunk: h=4, the dense 64-head
+    """The other measured configurations: on the chunk, h=4, the dense 64-head
     indexer in this library, MISA-dagger (k'=8192, all-head rerank to 2048) with
-    bf16 and with FP8 keys, and the recall of each against the dense top-k."""
+    bf16 and with FP8 keys (with the recall of each against the dense top-k), and
+    the unfused score + top-k sequence; and the DeepSeek-V3.2- and GLM-5-shaped
+    whole-sequence prefills (32768 and 65536 tokens)."""
     import torch
 
     from long_context_sparse_block_b200 import workloads as Wm
@@ -490,6 +492,48 @@ def run_variants(wl, inp, stream, flush):
     out["dagger_fp8_recall_vs_dense_fp8"] = round(_recall(fin8, ref8, wl.n_k), 4)
     dense_bf = MisaIndexer(IndexerShape(h=wl.H, dense=True, **base))
     out["dagger_fp8_recall_vs_dense_bf16"] = round(_recall(fin8, dense_bf.run(Q, K, w), wl.n_k), 4)
+    del dense_bf, dg8, fin8, ref8, K8, ks
+
+    # the unfused sequence on the chunk: every logit written (store mode), then
+    # the standalone top-k reading them once (HBM-bound: 4 bytes per causal pair)
+    from long_context_sparse_block_b200 import _lib
+    ixu = MisaIndexer(IndexerShape(h=wl.h, **base))
+    ixu.run(Q, K, w)   # routes the heads
+    lg = ixu.logits
+    pairs = wl.causal_pairs()
+    t_s = _time_ms(lambda: _lib.misa_score_tokens(Q, w, ixu.heads, K, wl.q_pos0, logits=lg, h=wl.h),
+                   stream, flush)
+    t_k = _time_ms(lambda: _lib.misa_topk(lg, wl.q_pos0, wl.n_k, wl.k, idx=ixu.sel), stream, flush)
+    out["unfused_score_ms"] = round(t_s, 4)
+    out["unfused_score_tflops"] = round(2.0 * wl.h * wl.d * pairs / (t_s * 1e-3) / 1e12, 1)
+    out["unfused_topk_ms"] = round(t_k, 4)
+    out["unfused_topk_logit_gbs"] = round(4.0 * pairs / (t_k * 1e-3) / 1e9, 1)
+    del ixu, lg, Q, K, w
+
+    # the prefill configurations (whole-sequence prefill, the fused path per
+    # 8192-query sub-chunk; the first sub-chunk, whose prefix is shorter than
+    # the 4096-key sample, takes the unfused sequence)
+    for name in ("dsv32_32k", "glm5_64k"):
+        cw = Wm.WORKLOADS[name]
+        ci = Wm.generate(cw)
+        Qc, Kc, wc = d16(ci["Q"]), d16(ci["K"]), torch.from_numpy(ci["w"]).cuda()
+        ixc = MisaIndexer(IndexerShape(cw.n_q, cw.q_pos0, cw.n_k, cw.H, cw.d, cw.B, cw.h, cw.k))
+        t = _time_ms(lambda: ixc.run(Qc, Kc, wc), stream, flush)
+        _lib.misa_profile_start()
+        ixc.run(Qc, Kc, wc)
+        st = _lib.misa_profile_stop()
+        cp = cw.causal_pairs()
+        sel_ms = st["select_score"][0]
+        # pairs of the sub-chunks that ran the select pass (prefix >= the sample)
+        fused_pairs = sum(
+            sum(cw.q_pos0 + t + 1 for t in (c0, c1 - 1)) * (c1 - c0) // 2
+            for c0, c1 in ((c0, min(cw.n_q, c0 + ixc.sub)) for c0 in range(0, cw.n_q, ixc.sub))
+            if cw.q_pos0 + c0 + 1 >= 4096)
+        out[f"{name}_ms"] = round(t, 4)
+        out[f"{name}_pairs_per_s"] = round(cp / (t * 1e-3), 1)
+        out[f"{name}_select_tflops"] = (
+            round(2.0 * cw.h * cw.d * fused_pairs / (sel_ms * 1e-3) / 1e12, 1) if sel_ms > 0 else None)
+        del ixc, Qc, Kc, wc, ci
     return out
 
 
