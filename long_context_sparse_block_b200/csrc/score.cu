@@ -452,14 +452,42 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
       if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
+      constexpr bool SPLIT = EC == 64 && HT >= 4 && HT <= 32;  // no query spans the halves
       uint32_t v[EC];
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * kCols + part * EC);
-      if constexpr (EC == 64)
-        tmem_ld64(taddr, v);
-      else
-        tmem_ld128(taddr, v);
-      tmem_wait_ld();
+      float sums[HT >= 4 ? QPW : 1];
+      auto qsum = [&](int qq) {
+        float2 a2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int j = 0; j < HT; j += 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(w_s + qq * HT + j);
+          const uint32_t* x = v + qq * HT + j;
+          a2 = fma2(make_float2(w4.x, w4.y),
+                    make_float2(relu(__uint_as_float(x[0])), relu(__uint_as_float(x[1]))), a2);
+          a2 = fma2(make_float2(w4.z, w4.w),
+                    make_float2(relu(__uint_as_float(x[2])), relu(__uint_as_float(x[3]))), a2);
+        }
+        return a2.x + a2.y;
+      };
+      if constexpr (SPLIT) {
+        // two 32-column halves: the second lands while the first half's
+        // queries are summed
+        uint32_t (&va)[32] = *reinterpret_cast<uint32_t(*)[32]>(v);
+        uint32_t (&vb)[32] = *reinterpret_cast<uint32_t(*)[32]>(v + 32);
+        tmem_ld32(taddr, va);
+        tmem_wait_ld_regs(va);
+        tmem_ld32(taddr + 32, vb);
+#pragma unroll
+        for (int qq = 0; qq < QPW / 2; ++qq) sums[qq] = qsum(qq);
+        tmem_wait_ld_regs(vb);
+      } else {
+        if constexpr (EC == 64)
+          tmem_ld64(taddr, v);
+        else
+          tmem_ld128(taddr, v);
+        tmem_wait_ld();
+      }
       // the accumulator is in registers: hand it back to the MMA warp now
       tc_fence_before();
       __syncwarp();
@@ -474,23 +502,8 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
       float* dst = p.logits + tq0 * p.ld + s;
       (void)dst;
       if constexpr (HT >= 4) {
-        // every head-sum first (the shared-memory weight loads never wait
-        // behind a global store), then the stores
-        float sums[QPW];
 #pragma unroll
-        for (int qq = 0; qq < QPW; ++qq) {
-          float2 a2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-          for (int j = 0; j < HT; j += 4) {
-            const float4 w4 = *reinterpret_cast<const float4*>(w_s + qq * HT + j);
-            const uint32_t* x = v + qq * HT + j;
-            a2 = fma2(make_float2(w4.x, w4.y),
-                      make_float2(relu(__uint_as_float(x[0])), relu(__uint_as_float(x[1]))), a2);
-            a2 = fma2(make_float2(w4.z, w4.w),
-                      make_float2(relu(__uint_as_float(x[2])), relu(__uint_as_float(x[3]))), a2);
-          }
-          sums[qq] = a2.x + a2.y;
-        }
+        for (int qq = SPLIT ? QPW / 2 : 0; qq < QPW; ++qq) sums[qq] = qsum(qq);
         if constexpr (KSC) {
           // per-token scale > 0: w * ReLU(scale * dot) = scale * w * ReLU(dot)
           const float ks = s_ok ? __ldg(p.k_scale + s) : 0.0f;
