@@ -66,17 +66,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // try_wait that may suspend the thread (up to `hint_ns`) until the phase
 // completes instead of returning at once: keeps waiting warps off the issue slots.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
 
 // Waits for the phase of parity `parity` of barrier `bar`.  Gives up (returns
 // false) when another role of the CTA has raised `*abort`, or when the wait

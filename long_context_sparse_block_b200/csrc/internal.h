@@ -67,7 +67,6 @@ cudaError_t launch_e4m3_to_bf16(const uint8_t* src, uint16_t* dst, int64_t n, cu
 
 // Fused top-k helpers (topk.cu): sample gather, per-row thresholds from the
 // scored sample, and the exact selection over the select-mode candidates.
-int sample_block_keys();
 cudaError_t launch_gather_sample(const void* K, const float* k_scale, int row_bytes, int64_t span,
                                  int n_blocks, void* Ks, float* ks_scale, cudaStream_t s);
 cudaError_t launch_fused_tau(const float* sample, int64_t lds, int n_s, int n_q, int64_t q_pos0,

@@ -813,6 +813,5 @@ cudaError_t launch_fused_finish(const float* logits, int64_t ld, const uint32_t*
   return cudaGetLastError();
 }
 
-int sample_block_keys() { return kSampleBlock; }
 
 }  // namespace misa
