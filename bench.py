@@ -206,6 +206,11 @@ def _workload(args):
     return wl
 
 
+def _workload_name(wl, h: int) -> str:
+    return (f"{wl.name}: {wl.n_q} queries at {wl.q_pos0}..{wl.q_pos0 + wl.n_q - 1} "
+            f"x {wl.n_k} keys, H_I={wl.H}, d={wl.d}, B={wl.B}, h={h}, k={wl.k}")
+
+
 def rank_inputs(inp: dict, rank: int, world: int) -> dict:
     """Every rank indexes its own chunk of the same shape: the shared keys and its
     own seeded permutation of the queries (and their head weights)."""
@@ -381,8 +386,7 @@ def run_ours(args, rank, world, local_rank, inp):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": (f"{wl.name}: {wl.n_q} queries at {wl.q_pos0}..{wl.q_pos0 + wl.n_q - 1} "
-                         f"x {wl.n_k} keys, H_I={wl.H}, d={wl.d}, B={wl.B}, h={h}, k={wl.k}"),
+            "workload": _workload_name(wl, h),
             "query_sub_chunk": ix.sub,
             "fused_score_topk": fused,
             "rows_repaired_last_subchunk": repaired,
@@ -544,11 +548,13 @@ def run_reference(args, rank):
     h = args.h or wl.h
     t0 = time.perf_counter()
     cb = cpu_baseline(wl, h, W.generate(wl), budget_s=args.cpu_budget)
-    return {"metric": METRIC, "value": cb["value"], "unit": "ms", "n_gpus": 1,
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    return {"metric": METRIC, "value": cb["value"], "unit": "ms", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["value"],
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"{wl.name}", "h": h},
+            "config": {"workload": _workload_name(wl, h),
+                       "parallelism": "one host process pool (the oracle arm)"},
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "ms", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
