@@ -459,8 +459,9 @@ def run_variants(wl, inp, stream, flush):
     """The other measured configurations: on the chunk, h=4, the dense 64-head
     indexer in this library, MISA-dagger (k'=8192, all-head rerank to 2048) with
     bf16 and with FP8 keys (with the recall of each against the dense top-k), and
-    the unfused score + top-k sequence; and the DeepSeek-V3.2- and GLM-5-shaped
-    whole-sequence prefills (32768 and 65536 tokens)."""
+    the unfused score + top-k sequence, one decode step on the full cache; and the
+    DeepSeek-V3.2- and GLM-5-shaped whole-sequence prefills (32768 and 65536
+    tokens)."""
     import torch
 
     from long_context_sparse_block_b200 import workloads as Wm
@@ -512,6 +513,23 @@ def run_variants(wl, inp, stream, flush):
     out["unfused_score_tflops"] = round(2.0 * wl.h * wl.d * pairs / (t_s * 1e-3) / 1e12, 1)
     out["unfused_topk_ms"] = round(t_k, 4)
     out["unfused_topk_logit_gbs"] = round(4.0 * pairs / (t_k * 1e-3) / 1e9, 1)
+
+    # one decode step on the full cache: the newest query (position n_k - 1)
+    # after its key was appended: re-pool the last block, route, score, select
+    M = -(-wl.n_k // wl.B)
+    kbar_hl = ixu.kbar_hl
+    q1, w1 = Q[-1:].contiguous(), w[-1:].contiguous()
+    heads1 = torch.empty((1, wl.h), dtype=torch.int32, device="cuda")
+    lg1 = torch.empty((1, (wl.n_k + 3) // 4 * 4), dtype=torch.float32, device="cuda")[:, :wl.n_k]
+    idx1 = torch.empty((1, wl.k), dtype=torch.int32, device="cuda")
+
+    def decode_step():
+        _lib.misa_pool_keys_range(K, wl.B, M - 1, M, kbar_hl=kbar_hl)
+        _lib.misa_route_heads(q1, w1, kbar_hl, wl.n_k - 1, wl.n_k, wl.B, wl.h, heads=heads1)
+        _lib.misa_score_tokens(q1, w1, heads1, K, wl.n_k - 1, logits=lg1, h=wl.h)
+        _lib.misa_topk(lg1, wl.n_k - 1, wl.n_k, wl.k, idx=idx1)
+
+    out["decode_step_ms"] = round(_time_ms(decode_step, stream, flush), 4)
     del ixu, lg, Q, K, w
 
     # the prefill configurations (whole-sequence prefill, the fused path per

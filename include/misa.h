@@ -68,6 +68,21 @@ int misa_pool_keys(const void* K, const float* k_scale, int kdtype, int64_t n_k,
                    float* kbar, uint16_t* kbar_hl, void* stream);
 
 /*
+ * Stage 1 for a growing key cache (decode): misa_pool_keys restricted to blocks
+ * m0 <= m < m1 of the n_k keys, M = ceil(n_k/B); every other entry of kbar and
+ * kbar_hl is left as it is.  kbar_hl keeps the [2, M, d] layout of the current
+ * n_k, so after appending keys: while M is unchanged only the last block needs
+ * pooling again (m0 = M-1, m1 = M); when M grows, pool every block (the lo
+ * plane moves).  Pooling each block is the same arithmetic whatever the range,
+ * so the result equals misa_pool_keys bit for bit.  0 <= m0 <= m1 <= M (m0 == m1
+ * is a no-op); other arguments as misa_pool_keys.  (Not a step of the pages'
+ * method, which they evaluate on prefill only: an incremental form of stage 1.)
+ */
+int misa_pool_keys_range(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d,
+                         int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
+                         void* stream);
+
+/*
  * Stages 2-3 — router and top-h (Metodologia step 1: per-head affinities
  * against the pooled keys, aggregated into one importance per head; keep the
  * top-h heads).  The aggregate is

@@ -35,6 +35,7 @@ class MisaError(RuntimeError):
 _vp, _i64, _int, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 _SIGS = {
     "misa_pool_keys": (_int, [_vp, _vp, _int, _i64, _int, _int, _vp, _vp, _vp]),
+    "misa_pool_keys_range": (_int, [_vp, _vp, _int, _i64, _int, _int, _i64, _i64, _vp, _vp, _vp]),
     "misa_route_heads": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _int, _int, _int, _int, _vp, _vp,
                                 _vp]),
     "misa_score_tokens": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _int, _int, _int,
@@ -113,6 +114,21 @@ def misa_pool_keys(K, B: int, k_scale=None, kbar=None, kbar_hl=None, want_kbar: 
                              _kdtype(K), n_k, d, B, _ptr(kbar, (torch.float32,), "kbar"),
                              _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), _stream())
     _check("misa_pool_keys", st)
+    return kbar, kbar_hl
+
+
+def misa_pool_keys_range(K, B: int, m0: int, m1: int, kbar=None, kbar_hl=None, k_scale=None,
+                         n_k: int | None = None):
+    """Re-pool blocks m0..m1-1 of the first n_k rows of K (default all rows) into
+    existing kbar [>=M, d] f32 / kbar_hl [2, M, d] buffers (M = ceil(n_k/B))."""
+    if n_k is None:
+        n_k = K.shape[0]
+    d = K.shape[1]
+    st = _lib.misa_pool_keys_range(_ptr(K, name="K"), _ptr(k_scale, (torch.float32,), "k_scale"),
+                                   _kdtype(K), n_k, d, B, m0, m1,
+                                   _ptr(kbar, (torch.float32,), "kbar"),
+                                   _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), _stream())
+    _check("misa_pool_keys_range", st)
     return kbar, kbar_hl
 
 

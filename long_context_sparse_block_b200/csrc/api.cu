@@ -177,17 +177,27 @@ using namespace misa;
 
 extern "C" {
 
-int misa_pool_keys(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d, int B,
-                   float* kbar, uint16_t* kbar_hl, void* stream) {
+int misa_pool_keys_range(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d,
+                         int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
+                         void* stream) {
   if (!K || !aligned16(K) || n_k < 1 || !good_d(d) || B < 1 || B > 4096) return MISA_ERR_INVALID_ARG;
   if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
   if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
   if (!kbar && !kbar_hl) return MISA_ERR_INVALID_ARG;
   if ((kbar && !aligned4(kbar)) || (kbar_hl && (reinterpret_cast<uintptr_t>(kbar_hl) & 1u)))
     return MISA_ERR_INVALID_ARG;
-  if ((n_k + B - 1) / B > 0x7fffffff) return MISA_ERR_INVALID_ARG;
-  return cuda_status(launch_pool_keys(K, k_scale, kdtype == MISA_K_FP8E4M3, n_k, d, B, kbar, kbar_hl,
-                                      as_stream(stream)));
+  const int64_t M = (n_k + B - 1) / B;
+  if (M > 0x7fffffff || m0 < 0 || m1 < m0 || m1 > M) return MISA_ERR_INVALID_ARG;
+  if (m0 == m1) return MISA_OK;
+  return cuda_status(launch_pool_keys(K, k_scale, kdtype == MISA_K_FP8E4M3, n_k, d, B, m0, m1,
+                                      kbar, kbar_hl, as_stream(stream)));
+}
+
+int misa_pool_keys(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d, int B,
+                   float* kbar, uint16_t* kbar_hl, void* stream) {
+  if (B < 1) return MISA_ERR_INVALID_ARG;
+  return misa_pool_keys_range(K, k_scale, kdtype, n_k, d, B, 0, (n_k + B - 1) / B, kbar, kbar_hl,
+                              stream);
 }
 
 int misa_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl, int n_q,

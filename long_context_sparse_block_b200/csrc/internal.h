@@ -15,8 +15,10 @@ int sm_count();  // of the current device
 int* device_status_word();
 unsigned long long wait_limit_ns();
 
+// Pools blocks m0 <= m < min(m1, ceil(n_k / B)) (pool.cu).
 cudaError_t launch_pool_keys(const void* K, const float* k_scale, bool fp8, int64_t n_k, int d,
-                             int B, float* kbar, uint16_t* kbar_hl, cudaStream_t s);
+                             int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
+                             cudaStream_t s);
 
 cudaError_t launch_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
                                int n_q, int64_t q_pos0, int64_t n_k, int H, int d, int B, int h,

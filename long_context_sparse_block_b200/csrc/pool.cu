@@ -18,7 +18,8 @@ constexpr int kPoolThreads = 256;
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kPoolThreads)
 pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scale, int64_t n_k,
-                 int B, int64_t M, float* __restrict__ kbar, uint16_t* __restrict__ kbar_hl) {
+                 int B, int64_t M, int64_t m0, float* __restrict__ kbar,
+                 uint16_t* __restrict__ kbar_hl) {
   // elements per 16-byte unit and units per row
   constexpr int EPU = FP8 ? 16 : 8;
   constexpr int UPR = D / EPU;                 // column groups
@@ -26,7 +27,7 @@ pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scal
   static_assert(kPoolThreads % UPR == 0, "column groups must tile the block");
   __shared__ float part[PHASES][D];
 
-  const int64_t m = blockIdx.x;
+  const int64_t m = m0 + blockIdx.x;  // this CTA's block
   const int64_t first = m * B;
   const int n_m = static_cast<int>(n_k - first < B ? n_k - first : static_cast<int64_t>(B));
   const int u = threadIdx.x % UPR;
@@ -110,12 +111,13 @@ pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scal
 }
 
 template <int D, bool FP8>
-cudaError_t launch(const void* K, const float* k_scale, int64_t n_k, int B, float* kbar,
-                   uint16_t* kbar_hl, cudaStream_t s) {
+cudaError_t launch(const void* K, const float* k_scale, int64_t n_k, int B, int64_t m0,
+                   int64_t m1, float* kbar, uint16_t* kbar_hl, cudaStream_t s) {
   const int64_t M = (n_k + B - 1) / B;
-  if (M == 0) return cudaSuccess;
-  pool_keys_kernel<D, FP8><<<static_cast<unsigned>(M), kPoolThreads, 0, s>>>(
-      static_cast<const uint8_t*>(K), k_scale, n_k, B, M, kbar, kbar_hl);
+  if (m1 > M) m1 = M;
+  if (m1 <= m0) return cudaSuccess;
+  pool_keys_kernel<D, FP8><<<static_cast<unsigned>(m1 - m0), kPoolThreads, 0, s>>>(
+      static_cast<const uint8_t*>(K), k_scale, n_k, B, M, m0, kbar, kbar_hl);
   return cudaGetLastError();
 }
 
@@ -150,18 +152,19 @@ cudaError_t launch_e4m3_to_bf16(const uint8_t* src, uint16_t* dst, int64_t n, cu
 }
 
 cudaError_t launch_pool_keys(const void* K, const float* k_scale, bool fp8, int64_t n_k, int d,
-                             int B, float* kbar, uint16_t* kbar_hl, cudaStream_t s) {
+                             int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
+                             cudaStream_t s) {
   if (fp8) {
     switch (d) {
-      case 32: return launch<32, true>(K, k_scale, n_k, B, kbar, kbar_hl, s);
-      case 64: return launch<64, true>(K, k_scale, n_k, B, kbar, kbar_hl, s);
-      case 128: return launch<128, true>(K, k_scale, n_k, B, kbar, kbar_hl, s);
+      case 32: return launch<32, true>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
+      case 64: return launch<64, true>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
+      case 128: return launch<128, true>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
     }
   } else {
     switch (d) {
-      case 32: return launch<32, false>(K, k_scale, n_k, B, kbar, kbar_hl, s);
-      case 64: return launch<64, false>(K, k_scale, n_k, B, kbar, kbar_hl, s);
-      case 128: return launch<128, false>(K, k_scale, n_k, B, kbar, kbar_hl, s);
+      case 32: return launch<32, false>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
+      case 64: return launch<64, false>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
+      case 128: return launch<128, false>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
     }
   }
   return cudaErrorInvalidValue;

@@ -67,6 +67,10 @@ def test_invalid_arguments_rejected_before_launch(lib):
     assert so.misa_pool_keys(p, None, 1, 128, 128, 64, p, p, None) == INV
     assert so.misa_pool_keys(p, None, 0, 128, 128, 64, None, None, None) == INV
     assert so.misa_pool_keys(odd, None, 0, 128, 128, 64, p, p, None) == INV
+    # pool range: m1 past the blocks, m0 > m1, negative m0
+    assert so.misa_pool_keys_range(p, None, 0, 256, 128, 64, 0, 5, p, p, None) == INV
+    assert so.misa_pool_keys_range(p, None, 0, 256, 128, 64, 3, 2, p, p, None) == INV
+    assert so.misa_pool_keys_range(p, None, 0, 256, 128, 64, -1, 2, p, p, None) == INV
     # route: queries past the keys, h > H, H not a power of two
     assert so.misa_route_heads(p, p, p, 10, 95, 100, 64, 128, 64, 8, p, None, None) == INV
     assert so.misa_route_heads(p, p, p, 10, 0, 100, 8, 128, 64, 9, p, None, None) == INV
@@ -93,4 +97,5 @@ def test_empty_work_is_a_no_op(lib):
     p = ctypes.c_void_p(16 * 1024)
     assert so.misa_topk(p, 100, 0, 0, 100, 4, p, None, 0, None) == 0
     assert so.misa_topk(p, 100, 10, 0, 100, 0, None, None, 0, None) == 0
+    assert so.misa_pool_keys_range(p, None, 0, 256, 128, 64, 2, 2, p, p, None) == 0
     assert so.misa_score_tokens(p, p, p, p, None, 0, 0, 0, 100, 64, 128, 8, p, 100, None) == 0
