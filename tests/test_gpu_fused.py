@@ -181,3 +181,26 @@ def test_indexer_host_pipeline_equals_device_run(lib, kp):
         out = ix.run_host(Qh, Kh, wh, pieces=pieces)
         torch.cuda.current_stream().synchronize()
         assert np.array_equal(out.numpy(), want)
+
+
+def test_score_topk_long_kept_lists(lib):
+    # the sampled blocks hold the only small keys, so the threshold sits low and
+    # every other visible key is kept: ~5.7k kept logits per row, near the top of
+    # what the finish kernel's list holds; every row must still come out exact
+    # without the repair path
+    n_q, q_pos0, n_k, H, d, k, h = 64, 8999, 9100, 64, 128, 1024, 8
+    rng = np.random.default_rng(24)
+    Q = (1.0 + 0.3 * rng.standard_normal((n_q, H, d))) / np.sqrt(d)
+    K = (1.0 + 0.5 * rng.standard_normal((n_k, d))) / np.sqrt(d)
+    span, nb = q_pos0 + 1, 32
+    for b in range(nb):
+        start = (span - 128) * b // (nb - 1)
+        K[start:start + 128] *= 0.01
+    w = np.full((n_q, H), 1.0 / H, dtype=np.float32)
+    Qg, Kg, wg = dev(W.bf16_bits(Q)), dev(W.bf16_bits(K)), dev(w)
+    _, hl = lib.misa_pool_keys(Kg, 128)
+    heads, _ = lib.misa_route_heads(Qg, wg, hl, q_pos0, n_k, 128, h)
+    got, flags = _fused(lib, Qg, wg, heads, Kg, q_pos0, k)
+    want, _ = _unfused(lib, Qg, wg, heads, Kg, q_pos0, k)
+    assert np.array_equal(got, want)
+    assert flags[0] == 0 and not flags[1:].any()    # no repair: the list held them
