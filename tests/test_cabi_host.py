@@ -51,6 +51,19 @@ def test_workspace_size(lib):
     assert lib.misa_workspace_size("rerank", 0, 10, 1, 1) == 0
 
 
+def test_workspace_size_fused(lib):
+    ws = lambda n_q, n_k, k: lib.misa_workspace_size("score_topk", n_q, n_k, k, 0)
+    assert ws(8192, 131072, 2048) > 0
+    assert ws(8192, 131072, 8192) > 0
+    assert ws(8192, 4095, 64) == 0            # prefix shorter than the sample
+    assert ws(8192, (1 << 18) + 1, 2048) == 0  # past the largest fused key count
+    assert ws(8192, 131072, 8193) == 0         # k past the finish kernel's list
+    assert ws(8192, 131072, 0) == 0
+    assert ws(0, 131072, 2048) == 0
+    # grows with the queries (per-row flags, thresholds, sample logits, masks)
+    assert ws(2048, 131072, 2048) < ws(8192, 131072, 2048)
+
+
 def _so(lib):
     return lib._lib
 
@@ -82,6 +95,16 @@ def test_invalid_arguments_rejected_before_launch(lib):
     assert so.misa_score_tokens(p, p, p, p, None, 0, 10, 0, 100, 64, 128, 6, p, 100, None) == UNS
     assert so.misa_score_tokens(odd, p, p, p, None, 0, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
     assert so.misa_score_tokens(p, p, p, p, None, 0, 10, 0, 101, 64, 128, 8, p, 101, None) == INV
+    # fused score + top-k: ld not a multiple of 4, k too large, missing workspace
+    # where the sizes need one, d unsupported
+    assert so.misa_score_topk(p, p, p, p, None, 0, 10, 8000, 9000, 64, 128, 8, 64, p, p, 9001,
+                              p, 1 << 30, None) == INV
+    assert so.misa_score_topk(p, p, p, p, None, 0, 10, 8000, 9000, 64, 128, 8, 20000, p, p, 9000,
+                              p, 1 << 30, None) == INV
+    assert so.misa_score_topk(p, p, p, p, None, 0, 10, 8000, 9000, 64, 128, 8, 64, p, p, 9000,
+                              None, 0, None) == lib.MISA_ERR_WORKSPACE
+    assert so.misa_score_topk(p, p, p, p, None, 0, 10, 8000, 9000, 64, 96, 8, 64, p, p, 9000,
+                              p, 1 << 30, None) == UNS
     # top-k: k too large, ld too small
     assert so.misa_topk(p, 100, 10, 0, 100, 20000, p, None, 0, None) == INV
     assert so.misa_topk(p, 5, 10, 0, 100, 4, p, None, 0, None) == INV
