@@ -38,6 +38,20 @@ class IndexerShape:
         return -(-self.n_k // self.B)
 
 
+def _piece_bounds(n: int, pieces: int):
+    """Query ranges of run_host: with three or more pieces the first and the last
+    are half the even share (the first copy-in and the last copy-out are the
+    only copies that nothing overlaps), the rest split what remains evenly."""
+    pieces = max(1, min(pieces, n))
+    if pieces < 3:
+        step = -(-n // pieces)
+        return [(c0, min(n, c0 + step)) for c0 in range(0, n, step)]
+    edge = max(1, n // (2 * pieces))
+    mid = n - 2 * edge
+    cuts = [0, edge] + [edge + mid * i // (pieces - 2) for i in range(1, pieces - 2)] + [n - edge, n]
+    return [(a, b) for a, b in zip(cuts, cuts[1:]) if b > a]
+
+
 class MisaIndexer:
     def __init__(self, shape: IndexerShape, device="cuda"):
         s = self.shape = shape
@@ -102,7 +116,8 @@ class MisaIndexer:
         pinned host int32 [n_q, k] tensor (allocated when None), complete when the
         current stream reaches this point.  The queries go in `pieces` pieces on
         three streams (copy in, index, copy out) so that the copies of one piece
-        overlap the indexing of another; the keys go first."""
+        overlap the indexing of another; the keys go first, and the first and
+        last pieces are small."""
         s = self.shape
         dev = self.heads.device
         if getattr(self, "_dev", None) is None:
@@ -119,8 +134,7 @@ class MisaIndexer:
         compute = torch.cuda.current_stream(dev)
         cin.wait_stream(compute)   # the device buffers are free again
         cout.wait_stream(compute)
-        step = -(-s.n_q // max(1, pieces))
-        bounds = [(c0, min(s.n_q, c0 + step)) for c0 in range(0, s.n_q, step)]
+        bounds = _piece_bounds(s.n_q, pieces)
         ev_in = []
         with torch.cuda.stream(cin):
             K.copy_(Kh, non_blocking=True)

@@ -122,3 +122,17 @@ def test_empty_work_is_a_no_op(lib):
     assert so.misa_topk(p, 100, 10, 0, 100, 0, None, None, 0, None) == 0
     assert so.misa_pool_keys_range(p, None, 0, 256, 128, 64, 2, 2, p, p, None) == 0
     assert so.misa_score_tokens(p, p, p, p, None, 0, 0, 0, 100, 64, 128, 8, p, 100, None) == 0
+
+
+def test_host_pipeline_pieces(lib):
+    # run_host's query pieces cover the chunk in order, none empty, with small
+    # first and last pieces from three pieces on
+    from long_context_sparse_block_b200.indexer import _piece_bounds
+    for n, pieces in ((8192, 1), (8192, 2), (8192, 3), (8192, 4), (8192, 8), (600, 4), (5, 4), (1, 4)):
+        b = _piece_bounds(n, pieces)
+        assert b[0][0] == 0 and b[-1][1] == n
+        assert all(x[1] == y[0] for x, y in zip(b, b[1:]))
+        assert all(y > x for x, y in b)
+        assert len(b) <= pieces
+    sizes = [y - x for x, y in _piece_bounds(8192, 4)]
+    assert sizes == [1024, 3072, 3072, 1024]
