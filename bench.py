@@ -47,7 +47,7 @@ METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor 
 # queries of chunk_128k: the ncu capture of queries 0..1023 summarised in
 # profiles/score_select_chunk_128k.md, scaled by the query count; valid only for
 # the kernel sources it was taken on (null otherwise).
-SCORE_TRAFFIC = {"sources_sha256_16": "2f7f251fe0a318d9", "bytes_per_launch": 8 * (169.202688e6 + 123.251712e6),
+SCORE_TRAFFIC = {"sources_sha256_16": "926a9d27082ee4c4", "bytes_per_launch": 8 * (169.202688e6 + 123.251712e6),
                  "queries": 8192}
 
 

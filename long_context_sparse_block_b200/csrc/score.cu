@@ -80,14 +80,21 @@ struct ScoreLayout {
   static constexpr int QG = kCols / HT;
   static constexpr int STG_BYTES = TMA_STORE ? QG * kTileKeys * 4 : 0;
   static constexpr int SMEM_BUDGET = 227 * 1024 - 1024 - 8 * 1024;  // minus alignment, small data
-  static constexpr int STAGES_FIT = (SMEM_BUDGET - B_BYTES - 2 * STG_BYTES) / A_BYTES;
+  // FP8 keys decoded in the kernel: raw e4m3 tiles staged by cp.async, two
+  // (the next one prefetched) when that still leaves two key stages, else one
+  static constexpr int RAW_TILE = FP8 ? kTileKeys * D : 0;
+  static constexpr int NRAW =
+      !FP8 ? 0 : ((SMEM_BUDGET - B_BYTES - 2 * STG_BYTES - 2 * RAW_TILE) / A_BYTES >= 2 ? 2 : 1);
+  static constexpr int STAGES_FIT =
+      (SMEM_BUDGET - B_BYTES - 2 * STG_BYTES - NRAW * RAW_TILE) / A_BYTES;
   static constexpr int STAGES_MAX = D == 128 ? 4 : 8;
   static constexpr int STAGES = STAGES_FIT < STAGES_MAX ? STAGES_FIT : STAGES_MAX;
   static_assert(STAGES >= 2, "key ring needs two stages");
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_STG = OFF_B + B_BYTES;       // 2 staging buffers (1024-aligned)
-  static constexpr int OFF_W = OFF_STG + 2 * STG_BYTES;  // per epilogue warp: its columns' w
+  static constexpr int OFF_RAW = OFF_STG + 2 * STG_BYTES;  // FP8: 2 raw key tiles
+  static constexpr int OFF_W = OFF_RAW + NRAW * RAW_TILE;  // per epilogue warp: its columns' w
   static constexpr int OFF_TAU = OFF_W + Epi<HT, FP8>::WARPS * Epi<HT, FP8>::COLS * 4;  // select: tau
   static constexpr int OFF_HEADS = OFF_TAU + (SEL ? Epi<HT, FP8>::WARPS * 16 * 4 : 0);  // producer
   static constexpr int OFF_BAR = OFF_HEADS + kCols * 4;
@@ -216,7 +223,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::STAGES; ++i) {
-      mbar_init(bar(FULL + i), FP8 ? 32 * CONV : 1);
+      mbar_init(bar(FULL + i), 1);
       mbar_init(bar(EMPTY + i), 1);
     }
     mbar_init(bar(BFULL), 32);
@@ -373,24 +380,56 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
     // ------------------------------------------------------------ FP8 key converters
     // e4m3 key rows -> bf16 (exact) straight into the swizzled key tile
     if constexpr (FP8) {
-      const int ct = threadIdx.x - 96;  // 0 .. 32*CONV-1
+      // the e4m3 rows of the next tile are copied into a raw staging tile by
+      // cp.async while this tile's are decoded (shared memory to shared memory)
       constexpr int U8 = D / 16;        // 16-byte e4m3 units per key row
       constexpr int UPC = L::ROWB / 16; // bf16 16-byte units per swizzle-chunk row
-      Sched<QG> it;
+      const uint32_t raw0 = smem_u32(smem + L::OFF_RAW);
+      auto issue = [&](int64_t kt, int rb) {
+        for (int x = lane; x < kTileKeys * U8; x += 32) {
+          const int r = x / U8, u = x % U8;
+          const int64_t key = kt * kTileKeys + r;
+          const bool in = key < p.n_k;
+          cp_async16(raw0 + rb * L::RAW_TILE + x * 16, p.K8 + (in ? key : 0) * D + u * 16,
+                     in ? 16u : 0u);
+        }
+        cp_async_commit();
+      };
+      Sched<QG> it, nx;
       it.init(p);
-      int stage = 0;
+      nx = it;
+      int stage = 0, rb = 0;
       uint32_t phase = 0;
+      if (L::NRAW == 2 && it.left > 0) {
+        issue(it.kt, 0);
+        nx.next(p);
+      }
       for (; it.left > 0; it.next(p)) {
+        if constexpr (L::NRAW == 2) {
+          if (nx.left > 0) {
+            issue(nx.kt, rb ^ 1);
+            nx.next(p);
+          } else {
+            cp_async_commit();  // (empty group: keeps the wait below uniform)
+          }
+          cp_async_wait_group<1>();  // this tile's rows have landed
+        } else {
+          issue(it.kt, 0);
+          cp_async_wait_group<0>();
+        }
+        __syncwarp();
         bool ok = true;
         if (lane == 0) ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         const uint32_t dst = sA + stage * L::A_BYTES;
-        for (int x = ct; x < kTileKeys * U8; x += 32 * CONV) {
+        const uint32_t src = raw0 + rb * L::RAW_TILE;
+#pragma unroll 4
+        for (int x = lane; x < kTileKeys * U8; x += 32) {
           const int r = x / U8, u = x % U8;
-          const int64_t key = it.kt * kTileKeys + r;
-          uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-          if (key < p.n_k) raw = __ldg(reinterpret_cast<const uint4*>(p.K8 + key * D + u * 16));
-          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t wv[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(wv[0]), "=r"(wv[1]), "=r"(wv[2]), "=r"(wv[3])
+                       : "r"(src + x * 16));
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const uint32_t b0 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[2 * hh] & 0xFFFF));
@@ -405,12 +444,15 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           }
         }
         fence_proxy_async_smem();
-        mbar_arrive(bar(FULL + stage));
+        __syncwarp();  // every lane has read the raw tile before it is refilled
+        if (lane == 0) mbar_arrive(bar(FULL + stage));
         if (++stage == L::STAGES) {
           stage = 0;
           phase ^= 1;
         }
+        if constexpr (L::NRAW == 2) rb ^= 1;
       }
+      cp_async_wait_all();
     }
   } else {
     // ------------------------------------------------------------ epilogue
