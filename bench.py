@@ -47,7 +47,7 @@ METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor 
 # queries of chunk_128k: the ncu capture of queries 0..1023 summarised in
 # profiles/score_select_chunk_128k.md, scaled by the query count; valid only for
 # the kernel sources it was taken on (null otherwise).
-SCORE_TRAFFIC = {"sources_sha256_16": "926a9d27082ee4c4", "bytes_per_launch": 8 * (169.202688e6 + 123.251712e6),
+SCORE_TRAFFIC = {"sources_sha256_16": "926a9d27082ee4c4", "bytes_per_launch": 8 * (170.414592e6 + 122.709760e6),
                  "queries": 8192}
 
 
@@ -415,7 +415,7 @@ def run_ours(args, rank, world, local_rank, inp):
             "hbm_peak_gbs": peaks["hbm_gbs"],
             "pairs_per_s": round(pairs / (ms * 1e-3), 1),
         },
-        "e2e": {"value": round(whole_job_ms(e2e, world), 4), "unit": "ms", "h2d_bytes_per_step": int(h2d),
+        "e2e": {"value": round(whole_job_ms(e2e, world), 4) if e2e_ms else None, "unit": "ms", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
