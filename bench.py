@@ -47,7 +47,7 @@ METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor 
 # queries of chunk_128k: the ncu capture of queries 0..1023 summarised in
 # profiles/score_select_chunk_128k.md, scaled by the query count; valid only for
 # the kernel sources it was taken on (null otherwise).
-SCORE_TRAFFIC = {"sources_sha256_16": "926a9d27082ee4c4", "bytes_per_launch": 8 * (170.414592e6 + 122.709760e6),
+SCORE_TRAFFIC = {"sources_sha256_16": "7799d366cb83581e", "bytes_per_launch": 8 * (168.861440e6 + 121.014528e6),
                  "queries": 8192}
 
 
@@ -458,8 +458,9 @@ def _recall(sel, ref, n_k):
 def run_variants(wl, inp, stream, flush):
     """The other measured configurations: on the chunk, h=4, the dense 64-head
     indexer in this library, MISA-dagger (k'=8192, all-head rerank to 2048) with
-    bf16 and with FP8 keys (with the recall of each against the dense top-k), and
-    the unfused score + top-k sequence, one decode step on the full cache; and the
+    bf16 and with FP8 keys (with the recall of each against the dense top-k), the
+    unfused score + top-k sequence, the scoring with e4m3 queries and keys, one
+    decode step on the full cache; and the
     DeepSeek-V3.2- and GLM-5-shaped whole-sequence prefills (32768 and 65536
     tokens)."""
     import torch
@@ -497,7 +498,7 @@ def run_variants(wl, inp, stream, flush):
     out["dagger_fp8_recall_vs_dense_fp8"] = round(_recall(fin8, ref8, wl.n_k), 4)
     dense_bf = MisaIndexer(IndexerShape(h=wl.H, dense=True, **base))
     out["dagger_fp8_recall_vs_dense_bf16"] = round(_recall(fin8, dense_bf.run(Q, K, w), wl.n_k), 4)
-    del dense_bf, dg8, fin8, ref8, K8, ks
+    del dense_bf, dg8, fin8, ref8, K8, ks     # (K8c, sc stay on the host)
 
     # the unfused sequence on the chunk: every logit written (store mode), then
     # the standalone top-k reading them once (HBM-bound: 4 bytes per causal pair)
@@ -513,6 +514,22 @@ def run_variants(wl, inp, stream, flush):
     out["unfused_score_tflops"] = round(2.0 * wl.h * wl.d * pairs / (t_s * 1e-3) / 1e12, 1)
     out["unfused_topk_ms"] = round(t_k, 4)
     out["unfused_topk_logit_gbs"] = round(4.0 * pairs / (t_k * 1e-3) / 1e9, 1)
+
+    # the same scoring with e4m3 queries and keys (a scale per (query, head) row
+    # and per key) multiplied as e4m3 on the tensor cores, and the top-2048 of
+    # those logits against the bf16 selection
+    Q8c, qs = Wm.e4m3_quantize_queries(Wm.bf16_values(inp["Q"]).astype(np.float64))
+    Q8, qsc = torch.from_numpy(Q8c).cuda(), torch.from_numpy(qs).cuda()
+    K8, ks = torch.from_numpy(K8c).cuda(), torch.from_numpy(sc).cuda()
+    del Q8c
+    sel_bf16 = ixu.sel.clone()
+    t_8 = _time_ms(lambda: _lib.misa_score_tokens_fp8(Q8, qsc, w, ixu.heads, K8, ks, wl.q_pos0,
+                                                      logits=lg, h=wl.h), stream, flush)
+    out["fp8_qk_score_ms"] = round(t_8, 4)
+    out["fp8_qk_score_tflops"] = round(2.0 * wl.h * wl.d * pairs / (t_8 * 1e-3) / 1e12, 1)
+    _lib.misa_topk(lg, wl.q_pos0, wl.n_k, wl.k, idx=ixu.sel)
+    out["fp8_qk_recall_vs_bf16"] = round(_recall(ixu.sel, sel_bf16, wl.n_k), 4)
+    del Q8, qsc, K8, ks, sel_bf16
 
     # one decode step on the full cache: the newest query (position n_k - 1)
     # after its key was appended: re-pool the last block, route, score, select

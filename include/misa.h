@@ -115,6 +115,26 @@ int misa_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads, c
                       int H, int d, int h, float* logits, int64_t ld, void* stream);
 
 /*
+ * Stage 4 with FP8 queries as well as FP8 keys, multiplied on the tensor cores
+ * as E4M3 (kind::f8f6f4, twice the bf16 rate).  The integration issue runs the
+ * indexer with FP8 operands in vLLM but fixes no scale rule; here every
+ * (query, head) row and every key row carries its own fp32 scale:
+ *   q[t, j] = e4m3(Q8[t, j, :]) * q_scale[t, j],  k_s = e4m3(K8[s, :]) * k_scale[s]
+ *   logits[t, s] = sum_{i < h} w[t, j_i] * ReLU(q[t, j_i] . k_s),  s <= pos(t)
+ * computed as k_scale[s] * sum_i (w[t, j_i] * q_scale[t, j_i]) * ReLU(e4m3 dot),
+ * the same in real arithmetic because every scale must be positive and finite
+ * (not checked).  Q8 [n_q, H, d] and K8 [n_k, d] hold e4m3 codes (NaN codes
+ * not allowed), 16-byte aligned; q_scale [n_q, H], k_scale [n_k] fp32.
+ * d in {64, 128}; the other arguments, the layout of logits and the -inf
+ * entries are those of misa_score_tokens.  Returns MISA_ERR_UNSUPPORTED for
+ * other d, MISA_ERR_INVALID_ARG for bad pointers or sizes.
+ */
+int misa_score_tokens_fp8(const uint8_t* Q8, const float* q_scale, const float* w,
+                          const int32_t* heads, const uint8_t* K8, const float* k_scale, int n_q,
+                          int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
+                          int64_t ld, void* stream);
+
+/*
  * Stage 5 — top-k token selection (technical summary, Metodologia step 2: the
  * final top-k tokens come from the reduced scores).  For each row t, among
  * logits[t, 0..min(pos(t), n_k-1)] keep the k largest, ties to the lower token

@@ -40,6 +40,8 @@ _SIGS = {
                                 _vp]),
     "misa_score_tokens": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _int, _int, _int,
                                  _vp, _i64, _vp]),
+    "misa_score_tokens_fp8": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _int, _int,
+                                     _int, _vp, _i64, _vp]),
     "misa_topk": (_int, [_vp, _i64, _int, _i64, _i64, _int, _vp, _vp, _sz, _vp]),
     "misa_rerank": (_int, [_vp, _vp, _vp, _vp, _int, _vp, _int, _int, _i64, _i64, _int, _int, _int,
                            _vp, _vp, _vp, _sz, _vp]),
@@ -161,6 +163,29 @@ def misa_score_tokens(Q, w, heads, K, q_pos0: int, k_scale=None, logits=None, h:
                                 _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K), n_q, q_pos0,
                                 n_k, H, d, h, ctypes.c_void_p(logits.data_ptr()), ld, _stream())
     _check("misa_score_tokens", st)
+    return logits
+
+
+_E4M3_CODES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def misa_score_tokens_fp8(Q8, q_scale, w, heads, K8, k_scale, q_pos0: int, logits=None,
+                          h: int | None = None):
+    """Routed logits [n_q, ld] f32 from e4m3 queries [n_q, H, d] (scales [n_q, H]) and e4m3
+    keys [n_k, d] (scales [n_k]), multiplied as e4m3 on the tensor cores."""
+    n_q, H, d = Q8.shape
+    n_k = K8.shape[0]
+    if h is None:
+        h = heads.shape[1] if heads is not None else H
+    if logits is None:
+        logits = torch.empty((n_q, (n_k + 3) // 4 * 4), dtype=torch.float32, device=Q8.device)[:, :n_k]
+    ld = logits.stride(0) if logits.dim() == 2 else n_k
+    st = _lib.misa_score_tokens_fp8(_ptr(Q8, _E4M3_CODES, "Q8"), _ptr(q_scale, (torch.float32,), "q_scale"),
+                                    _ptr(w, (torch.float32,), "w"), _ptr(heads, (torch.int32,), "heads"),
+                                    _ptr(K8, _E4M3_CODES, "K8"), _ptr(k_scale, (torch.float32,), "k_scale"),
+                                    n_q, q_pos0, n_k, H, d, h, ctypes.c_void_p(logits.data_ptr()), ld,
+                                    _stream())
+    _check("misa_score_tokens_fp8", st)
     return logits
 
 

@@ -240,6 +240,43 @@ int misa_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads, c
                                          q_pos0, n_k, H, d, h, logits, ld, ctl, as_stream(stream)));
 }
 
+int misa_score_tokens_fp8(const uint8_t* Q8, const float* q_scale, const float* w,
+                          const int32_t* heads, const uint8_t* K8, const float* k_scale, int n_q,
+                          int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
+                          int64_t ld, void* stream) {
+  if (!Q8 || !aligned16(Q8) || !q_scale || !aligned4(q_scale) || !w || !aligned4(w) || !K8 ||
+      !aligned16(K8) || !k_scale || !aligned4(k_scale) || !logits || !aligned16(logits))
+    return MISA_ERR_INVALID_ARG;
+  if (heads && !aligned4(heads)) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || H < 1 || h < 1 || h > H ||
+      ld < n_k || ld % 4 != 0)
+    return MISA_ERR_INVALID_ARG;
+  if (!heads && h != H) return MISA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
+  if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
+  if (n_q == 0) return MISA_OK;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  ScoreLaunch a{};
+  a.Q = reinterpret_cast<const uint16_t*>(Q8);
+  a.q8 = true;
+  a.q_scale = q_scale;
+  a.w = w;
+  a.heads = heads;
+  a.K = K8;
+  a.k_scale = k_scale;
+  a.fp8 = true;
+  a.n_q = n_q;
+  a.q_pos0 = q_pos0;
+  a.n_k = n_k;
+  a.H = H;
+  a.d = d;
+  a.h = h;
+  a.logits = logits;
+  a.ld = ld;
+  return cuda_status(launch_score(a, ctl, as_stream(stream)));
+}
+
 int misa_topk(const float* logits, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k, int k,
               int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
   (void)ws;

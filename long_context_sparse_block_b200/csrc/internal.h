@@ -47,6 +47,8 @@ struct ScoreLaunch {
   uint32_t* mask;         // select mode: [n_q][mask_ld] pass bits
   int64_t mask_ld;
   const int* gate;        // nullable: launch does nothing unless *gate != 0
+  bool q8;                // Q holds e4m3 codes ([n_q, H, d] bytes) with q_scale [n_q, H]
+  const float* q_scale;
 };
 cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s);
 bool score_select_supported(int h);

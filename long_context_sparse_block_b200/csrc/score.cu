@@ -66,14 +66,17 @@ struct Epi {
 };
 constexpr uint64_t kDrainNs = 2000000;  // 2 ms
 
-template <int D, int HT, bool FP8, bool SEL = false>
+// EB = bytes per operand element: 2 for bf16 operands, 1 when both Q and K are
+// e4m3 (kind::f8f6f4).
+template <int D, int HT, bool FP8, bool SEL = false, int EB = 2>
 struct ScoreLayout {
-  static constexpr int ROWB = D >= 64 ? 128 : 64;  // bytes per row of one swizzle chunk
-  static constexpr int KCH = D * 2 / ROWB;         // swizzle chunks along d
+  static_assert(D * EB >= 64, "operand rows of at least 64 bytes");
+  static constexpr int ROWB = D * EB >= 128 ? 128 : 64;  // bytes per row of one swizzle chunk
+  static constexpr int KCH = D * EB / ROWB;              // swizzle chunks along d
   static constexpr int A_CHUNK = kTileKeys * ROWB;
-  static constexpr int A_BYTES = kTileKeys * D * 2;
+  static constexpr int A_BYTES = kTileKeys * D * EB;
   static constexpr int B_CHUNK = kCols * ROWB;
-  static constexpr int B_BYTES = kCols * D * 2;
+  static constexpr int B_BYTES = kCols * D * EB;
   // fused logits of a tile are staged in shared memory ([QG queries][128 keys]
   // fp32, double-buffered) and written by one TMA store (h >= 4)
   static constexpr bool TMA_STORE = HT >= 4 && !SEL;
@@ -87,7 +90,7 @@ struct ScoreLayout {
       !FP8 ? 0 : ((SMEM_BUDGET - B_BYTES - 2 * STG_BYTES - 2 * RAW_TILE) / A_BYTES >= 2 ? 2 : 1);
   static constexpr int STAGES_FIT =
       (SMEM_BUDGET - B_BYTES - 2 * STG_BYTES - NRAW * RAW_TILE) / A_BYTES;
-  static constexpr int STAGES_MAX = D == 128 ? 4 : 8;
+  static constexpr int STAGES_MAX = D * EB == 256 ? 4 : 8;
   static constexpr int STAGES = STAGES_FIT < STAGES_MAX ? STAGES_FIT : STAGES_MAX;
   static_assert(STAGES >= 2, "key ring needs two stages");
   static constexpr int OFF_A = 0;
@@ -125,6 +128,7 @@ struct ScoreParams {
   // repair launch: nothing unless gate[0] != 0, then only the query groups
   // holding a row t with gate[1 + t] != 0
   const int* gate;
+  const float* q_scale;  // e4m3 queries only: [n_q, H] per (query, head) row
 };
 
 // Flattened schedule over (group g, key tile kt): each role of a CTA walks the
@@ -194,14 +198,18 @@ struct Sched {
 
 // Key modes: KM 0 = bf16 keys; KM 1 = FP8 E4M3 keys decoded by converter
 // warps in the kernel; KM 2 = FP8 keys already decoded to bf16 (exact) by the
-// caller.  KM 1 and 2 multiply each logit by the key's scale.
+// caller; KM 3 = E4M3 queries and keys multiplied as they are (kind::f8f6f4),
+// each (query, head) row's scale folded into its head weight.  KM 1, 2 and 3
+// multiply each logit by the key's scale.
 template <int D, int HT, int KM, bool SEL>
 __global__ void __maxnreg__((Epi<HT, KM == 1>::MAXREG))
 score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap lmap,
                     const ScoreParams p) {
   constexpr bool FP8 = KM == 1;  // converter warps
   constexpr bool KSC = KM != 0;  // per-key scale
-  using L = ScoreLayout<D, HT, FP8, SEL>;
+  constexpr bool QK8 = KM == 3;  // e4m3 operands
+  constexpr int EB = QK8 ? 1 : 2;
+  using L = ScoreLayout<D, HT, FP8, SEL, EB>;
   static_assert(!SEL || HT >= 4, "select mode needs h >= 4");
   if (p.gate && *p.gate == 0) return;  // repair launch with nothing to repair
   constexpr int EW = Epi<HT, FP8>::WARPS;
@@ -276,13 +284,14 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           hs[n] = j;
         }
         __syncwarp();
-        constexpr int UPR = D / 8;             // 16-byte units per row
+        constexpr int UPR = D * EB / 16;       // 16-byte units per row
         constexpr int UPC = L::ROWB / 16;      // units per swizzle chunk row
+        const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.Q);
         for (int x = lane; x < kCols * UPR; x += 32) {
           const int n = x / UPR, u = x % UPR;
           const int j = hs[n];
           const int t = it.g * QG + n / HT;
-          const uint16_t* src = j >= 0 ? p.Q + (static_cast<int64_t>(t) * p.H + j) * D + u * 8 : p.Q;
+          const uint8_t* src = j >= 0 ? qb + (static_cast<int64_t>(t) * p.H + j) * (D * EB) + u * 16 : qb;
           const uint32_t off = (u / UPC) * L::B_CHUNK + swz_offset(n, u % UPC, L::ROWB);
           cp_async16(sB + off, src, j >= 0 ? 16u : 0u);
         }
@@ -301,7 +310,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
 #pragma unroll
           for (int c = 0; c < L::KCH; ++c)
             tma_load_2d(sA + stage * L::A_BYTES + c * L::A_CHUNK, &kmap, bar(FULL + stage),
-                        c * (L::ROWB / 2), static_cast<int>(it.kt * kTileKeys));
+                        c * (L::ROWB / EB), static_cast<int>(it.kt * kTileKeys));
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -317,7 +326,8 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
     int stage = 0, acc = 0;
     uint32_t phase = 0, accph = 0, gcount = 0;
     int prev_g = -1;
-    constexpr uint32_t idesc = umma_idesc_bf16_f32(kTileKeys, kCols);
+    constexpr uint32_t idesc =
+        QK8 ? umma_idesc_e4m3_f32(kTileKeys, kCols) : umma_idesc_bf16_f32(kTileKeys, kCols);
     for (; it.left > 0; it.next(p)) {
       const bool new_group = it.g != prev_g;
       bool ok = true;
@@ -328,13 +338,17 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
         if (ok) {
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kCols);
+          // one instruction per 32 bytes of the rows (16 bf16 or 32 e4m3 elements)
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < D * EB / 32; ++kk) {
             const int c = (kk * 32) / L::ROWB, within = (kk * 32) % L::ROWB;
             const uint64_t ad =
                 umma_desc_kmajor(sA + stage * L::A_BYTES + c * L::A_CHUNK + within, L::ROWB);
             const uint64_t bd = umma_desc_kmajor(sB + c * L::B_CHUNK + within, L::ROWB);
-            tc_mma_bf16(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            if constexpr (QK8)
+              tc_mma_e4m3(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            else
+              tc_mma_bf16(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
           tc_commit(bar(EMPTY + stage));
           tc_commit(bar(ACCFULL + acc));
@@ -478,6 +492,8 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
             int j = p.heads ? __ldg(p.heads + static_cast<int64_t>(t) * HT + col % HT) : col % HT;
             if (j < 0 || j >= p.H) j = 0;
             wv = __ldg(p.w + static_cast<int64_t>(t) * p.H + j);
+            // e4m3 queries: the row's scale > 0 commutes with the ReLU
+            if constexpr (QK8) wv *= __ldg(p.q_scale + static_cast<int64_t>(t) * p.H + j);
           }
           w_s[i] = wv;
         }
@@ -644,7 +660,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
 template <int D, int HT, int KM, bool SEL>
 cudaError_t launch_dhs(const ScoreParams& p, const CUtensorMap& map, cudaStream_t s) {
   constexpr bool FP8 = KM == 1;
-  using L = ScoreLayout<D, HT, FP8, SEL>;
+  using L = ScoreLayout<D, HT, FP8, SEL, KM == 3 ? 1 : 2>;
   // fused-logit store map: [n_q rows][n_k keys] fp32 with row pitch ld, box 128 keys x QG queries
   CUtensorMap lmap;
   std::memset(&lmap, 0, sizeof lmap);
@@ -708,9 +724,20 @@ cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s
   }
   ScoreParams p{a.Q, a.w, a.heads, a.k_scale, static_cast<const uint8_t*>(a.K), a.logits, a.ld,
                 a.n_q, a.q_pos0, a.n_k, a.H, total, ctl, a.tau, a.mask, a.mask_ld,
-                a.gate};
+                a.gate, a.q_scale};
   CUtensorMap map;
   std::memset(&map, 0, sizeof map);
+  if (a.q8) {  // e4m3 queries and keys: one-byte key tiles by TMA, kind::f8f6f4
+    if (!a.fp8 || a.k_bf16 || (a.d != 64 && a.d != 128)) return cudaErrorNotSupported;
+    const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.n_k)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(a.d)};
+    const uint32_t box[2] = {static_cast<uint32_t>(a.d), static_cast<uint32_t>(kTileKeys)};
+    if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.K, dims, strides, box,
+                          a.d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    return a.d == 128 ? launch_d<128, 3>(p, a.h, sel, map, s) : launch_d<64, 3>(p, a.h, sel, map, s);
+  }
   if (a.fp8 && !a.k_bf16) {  // converter warps read the e4m3 keys; no key tensor map
     switch (a.d) {
       case 32: return launch_d<32, 1>(p, a.h, sel, map, s);

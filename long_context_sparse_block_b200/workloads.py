@@ -163,6 +163,19 @@ def e4m3_quantize_keys(k_values: np.ndarray):
     return codes, scale
 
 
+def e4m3_quantize_queries(q_values: np.ndarray):
+    """Per (query, head) row of [n_q, H, d]: the per-row rule of e4m3_quantize_keys.
+    Returns codes [n_q, H, d] and fp32 scales [n_q, H]."""
+    n_q, H, d = q_values.shape
+    flat = q_values.reshape(n_q * H, d)
+    codes = np.empty((n_q * H, d), dtype=np.uint8)
+    scale = np.empty(n_q * H, dtype=np.float32)
+    for r0 in range(0, n_q * H, _CHUNK_ROWS):
+        r1 = min(n_q * H, r0 + _CHUNK_ROWS)
+        codes[r0:r1], scale[r0:r1] = e4m3_quantize_keys(flat[r0:r1])
+    return codes.reshape(n_q, H, d), scale.reshape(n_q, H)
+
+
 # ---------------------------------------------------------------------------
 # generators
 # ---------------------------------------------------------------------------
@@ -175,7 +188,7 @@ def _normal_rows(rng, n_rows, n_cols, scale):
     return out
 
 
-def generate(wl: Workload, fp8_keys: bool = False) -> dict:
+def generate(wl: Workload, fp8_keys: bool = False, fp8_queries: bool = False) -> dict:
     """Draw the inputs of workload `wl`.
 
     Returns a dict with
@@ -184,6 +197,7 @@ def generate(wl: Workload, fp8_keys: bool = False) -> dict:
       w      float32 [n_q, H]
       needles int64 [n_needles]  positions of planted needle keys (may be empty)
       K8, k_scale                e4m3 codes [n_k, d] and fp32 [n_k] (fp8_keys only)
+      Q8, q_scale                e4m3 codes [n_q, H, d] and fp32 [n_q, H] (fp8_queries only)
     """
     rng = np.random.Generator(np.random.PCG64(wl.seed))
     d, H, n_q, n_k = wl.d, wl.H, wl.n_q, wl.n_k
@@ -227,6 +241,8 @@ def generate(wl: Workload, fp8_keys: bool = False) -> dict:
            "w": np.ascontiguousarray(w, dtype=np.float32), "needles": needles}
     if fp8_keys:
         out["K8"], out["k_scale"] = e4m3_quantize_keys(bf16_values(K).astype(np.float64))
+    if fp8_queries:
+        out["Q8"], out["q_scale"] = e4m3_quantize_queries(bf16_values(Q).astype(np.float64))
     return out
 
 

@@ -222,9 +222,15 @@ def select_candidates(vals, cand, q_pos0: int, n_k: int, k: int) -> np.ndarray:
 
 # ---- whole-path helpers over stored inputs -----------------------------------
 
-def decode_inputs(inp: dict, fp8_keys: bool = False):
-    """fp64 views of the stored inputs: (Q [n_q,H,d], K [n_k,d], w [n_q,H])."""
-    Q = bf16_to_f64(inp["Q"])
+def decode_inputs(inp: dict, fp8_keys: bool = False, fp8_queries: bool = False):
+    """fp64 views of the stored inputs: (Q [n_q,H,d], K [n_k,d], w [n_q,H]).
+    fp8_queries: Q from its e4m3 codes times the per-(query, head) scales."""
+    if fp8_queries:
+        n_q, H, d = inp["Q8"].shape
+        Q = e4m3_keys_to_f64(inp["Q8"].reshape(n_q * H, d),
+                             inp["q_scale"].reshape(n_q * H)).reshape(n_q, H, d)
+    else:
+        Q = bf16_to_f64(inp["Q"])
     K = e4m3_keys_to_f64(inp["K8"], inp["k_scale"]) if fp8_keys else bf16_to_f64(inp["K"])
     w = np.asarray(inp["w"], dtype=np.float64)
     return Q, K, w

@@ -95,6 +95,16 @@ def test_invalid_arguments_rejected_before_launch(lib):
     assert so.misa_score_tokens(p, p, p, p, None, 0, 10, 0, 100, 64, 128, 6, p, 100, None) == UNS
     assert so.misa_score_tokens(odd, p, p, p, None, 0, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
     assert so.misa_score_tokens(p, p, p, p, None, 0, 10, 0, 101, 64, 128, 8, p, 101, None) == INV
+    # FP8 queries and keys: d = 32 unsupported, missing scales, misaligned codes,
+    # ld < n_k, dense with h != H
+    f8 = so.misa_score_tokens_fp8
+    assert f8(p, p, p, p, p, p, 10, 0, 100, 64, 32, 8, p, 100, None) == UNS
+    assert f8(p, None, p, p, p, p, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    assert f8(p, p, p, p, p, None, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    assert f8(odd, p, p, p, p, p, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    assert f8(p, p, p, p, p, p, 10, 0, 100, 64, 128, 8, p, 99, None) == INV
+    assert f8(p, p, p, None, p, p, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    assert f8(p, p, p, p, p, p, 0, 0, 100, 64, 128, 8, p, 100, None) == 0
     # fused score + top-k: ld not a multiple of 4, k too large, missing workspace
     # where the sizes need one, d unsupported
     assert so.misa_score_topk(p, p, p, p, None, 0, 10, 8000, 9000, 64, 128, 8, 64, p, p, 9001,

@@ -140,6 +140,79 @@ def test_score_fp8_keys_matches_oracle(lib, n_q, q_pos0, n_k, H, d, h):
         assert_logits_close(out[t], ref[t, :pos + 1], mag, what=f"fp8 row {t}")
 
 
+FP8_QK_CASES = [
+    (70, 300, 517, 64, 128, 8, False),
+    (40, 1000, 1100, 32, 64, 16, False),
+    (9, 200, 250, 64, 128, 64, False),
+    (100, 0, 100, 64, 128, 4, False),
+    (257, 3, 300, 8, 64, 2, False),
+    (50, 10, 300, 16, 128, 1, False),
+    (33, 90, 200, 8, 64, 8, True),
+    (5, 130, 140, 128, 128, 128, True),
+]
+
+
+@pytest.mark.parametrize("n_q,q_pos0,n_k,H,d,h,dense", FP8_QK_CASES)
+def test_score_fp8_queries_and_keys_matches_oracle(lib, n_q, q_pos0, n_k, H, d, h, dense):
+    # queries and keys both e4m3 (a scale per (query, head) row and per key),
+    # multiplied as e4m3 on the tensor cores
+    wl = _wl(n_q, q_pos0, n_k, H, d, 64, h, 8, seed=13 * n_q + h)
+    inp = W.generate(wl, fp8_keys=True, fp8_queries=True)
+    Qd, Kd, wd = oracle.decode_inputs(inp, fp8_keys=True, fp8_queries=True)
+    rng = np.random.default_rng(n_q + 2)
+    if dense:
+        heads = np.tile(np.arange(H, dtype=np.int32), (n_q, 1))
+    else:
+        heads = np.sort(np.stack([rng.choice(H, size=h, replace=False) for _ in range(n_q)]),
+                        axis=1).astype(np.int32)
+    ref = oracle.score(Qd, wd, heads, Kd, q_pos0)
+    ld = (n_k + 3) // 4 * 4 + 4
+    logits = torch.full((n_q, ld), float("nan"), device="cuda")
+    lib.misa_score_tokens_fp8(dev(inp["Q8"]), dev(inp["q_scale"]), dev(inp["w"]),
+                              None if dense else dev(heads), dev(inp["K8"]), dev(inp["k_scale"]),
+                              q_pos0, logits=logits, h=h)
+    assert lib.misa_last_device_status() == 0
+    out = logits.cpu().numpy()
+    n4 = (n_k + 3) // 4 * 4
+    for t in range(n_q):
+        pos = q_pos0 + t
+        mag = logit_magnitude(Qd, wd, Kd, heads, t, q_pos0)
+        assert_logits_close(out[t], ref[t, :pos + 1], mag, what=f"fp8 q+k row {t}")
+        tail = out[t, pos + 1:n4]
+        assert np.all(np.isnan(tail) | np.isneginf(tail))
+        assert np.all(np.isnan(out[t, n4:]))
+    # top-k on those logits: bit-exact against the oracle's selection of them
+    k = min(64, n_k)
+    idx = lib.misa_topk(logits[:, :n_k], q_pos0, n_k, k)
+    assert np.array_equal(idx.cpu().numpy(), oracle.topk(out[:, :n_k], q_pos0, n_k, k))
+
+
+def test_fp8_queries_and_keys_exact_arithmetic_is_bitwise(lib):
+    # small-integer e4m3 codes with power-of-two scales and weights: every
+    # product and sum is exact, so the logits and the top-k match exactly
+    n_q, q_pos0, n_k, H, d, h, k = 150, 200, 520, 8, 128, 4, 40
+    rng = np.random.default_rng(21)
+    Q8 = W.e4m3_encode(rng.integers(-3, 4, size=(n_q, H, d)).astype(np.float64))
+    K8 = W.e4m3_encode(rng.integers(-3, 4, size=(n_k, d)).astype(np.float64))
+    q_scale = np.ldexp(1.0, rng.integers(-3, 2, size=(n_q, H))).astype(np.float32)
+    k_scale = np.ldexp(1.0, rng.integers(-3, 2, size=n_k)).astype(np.float32)
+    sign = np.where(rng.integers(0, 4, size=(n_q, H)) == 0, -1.0, 1.0)
+    w = (sign * np.ldexp(1.0, rng.integers(-3, 2, size=(n_q, H)))).astype(np.float32)
+    heads = np.sort(np.stack([rng.choice(H, size=h, replace=False) for _ in range(n_q)]),
+                    axis=1).astype(np.int32)
+    inp = {"Q8": Q8, "q_scale": q_scale, "K8": K8, "k_scale": k_scale, "w": w}
+    Qd, Kd, wd = oracle.decode_inputs(inp, fp8_keys=True, fp8_queries=True)
+    ref = oracle.score(Qd, wd, heads, Kd, q_pos0)
+    logits = lib.misa_score_tokens_fp8(dev(Q8), dev(q_scale), dev(w), dev(heads), dev(K8),
+                                       dev(k_scale), q_pos0)
+    idx = lib.misa_topk(logits, q_pos0, n_k, k)
+    assert lib.misa_last_device_status() == 0
+    out = logits.cpu().numpy().astype(np.float64)
+    for t in range(n_q):
+        assert np.array_equal(out[t, :q_pos0 + t + 1], ref[t, :q_pos0 + t + 1])
+    assert np.array_equal(idx.cpu().numpy(), oracle.topk(ref, q_pos0, n_k, k))
+
+
 def test_exact_arithmetic_is_bitwise(lib):
     # small integers and power-of-two weights: every product and sum is exact in
     # fp32, so pool, router scores, heads, logits and top-k must match exactly.

@@ -88,6 +88,31 @@ def test_e4m3_keys_dequantise_per_token():
     assert np.array_equal(K, [[0.5, -0.5], [896.0, 2.0 ** -8]])
 
 
+def test_e4m3_queries_quantise_per_query_head_row():
+    # each (query, head) row gets its own scale amax/448 (1 for a zero row); the
+    # row maximum maps to the largest code, and decoding through the oracle
+    # recovers every value within half an e4m3 step
+    rng = np.random.default_rng(3)
+    Q = rng.standard_normal((3, 2, 16)) * np.array([1.0, 1e-3])[None, :, None]
+    Q[2, 1] = 0.0
+    codes, scale = wlmod.e4m3_quantize_queries(Q)
+    assert codes.shape == (3, 2, 16) and scale.shape == (3, 2)
+    assert scale[2, 1] == 1.0 and not codes[2, 1].any()
+    for t in range(3):
+        for j in range(2):
+            if not Q[t, j].any():
+                continue
+            assert scale[t, j] == np.float32(np.abs(Q[t, j]).max() / 448.0)
+            assert (codes[t, j] & 0x7F).max() == 0x7E
+    inp = {"Q8": codes, "q_scale": scale, "K": np.zeros((1, 16), np.uint16),
+           "w": np.zeros((3, 2), np.float32)}
+    Qd, _, _ = oracle.decode_inputs(inp, fp8_queries=True)
+    y = Q / scale.astype(np.float64)[..., None]
+    step = np.where(np.abs(y) >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(np.abs(y), 1e-300))) - 3),
+                    2.0 ** -9)
+    assert np.all(np.abs(Qd / scale.astype(np.float64)[..., None] - y) <= step / 2 + 1e-12)
+
+
 # ---------------------------------------------------------------- worked example
 
 def test_worked_example_every_stage():
