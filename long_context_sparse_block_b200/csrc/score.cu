@@ -214,7 +214,6 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
   if (p.gate && *p.gate == 0) return;  // repair launch with nothing to repair
   constexpr int EW = Epi<HT, FP8>::WARPS;
   constexpr int EC = Epi<HT, FP8>::COLS;
-  constexpr int CONV = Epi<HT, FP8>::CONV;
   constexpr int QG = kCols / HT;  // queries per group
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
