@@ -13,6 +13,8 @@
  * Shapes and layouts (all row-major, all pointers are DEVICE pointers owned by
  * the caller unless stated otherwise):
  *   Q       [n_q, H, d]  bf16 (uint16 codes)  index queries, H = H_I heads
+ *   Q8      [n_q, H, d]  FP8 E4M3 codes with q_scale [n_q, H] fp32 (the FP8
+ *                        scoring call only; value = e4m3(code) * q_scale[t, j])
  *   K       [n_k, d]     bf16 codes, or FP8 E4M3 codes with k_scale [n_k] fp32
  *                        (value = e4m3(code) * k_scale[s])
  *   w       [n_q, H]     fp32 per-query head weights
