@@ -64,9 +64,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait that may suspend the thread (up to `hint_ns`) until the phase
-// completes instead of returning at once: keeps waiting warps off the issue slots.
-
 // Waits for the phase of parity `parity` of barrier `bar`.  Gives up (returns
 // false) when another role of the CTA has raised `*abort`, or when the wait
 // budget runs out, in which case it raises `*abort` and reports DEV_TIMEOUT.
