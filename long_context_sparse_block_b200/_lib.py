@@ -98,6 +98,19 @@ def _ptr(t, dtypes=None, name="tensor"):
 _BF16_CODES = (torch.bfloat16, torch.int16, torch.uint16)
 
 
+def _need(t, n: int, name: str):
+    """The kernels read or write `n` elements of `t` (which the C ABI cannot see):
+    refuse a smaller tensor before anything is launched."""
+    if t is not None and t.numel() < n:
+        raise ValueError(f"{name} holds {t.numel()} elements, the call needs {n}")
+
+
+def _need_rows(t, rows: int, cols: int, name: str):
+    """A 2-D (possibly row-padded) buffer with at least `rows` rows of `cols` entries."""
+    if t.dim() != 2 or t.shape[0] < rows or t.shape[1] < cols:
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, the call needs [>= {rows}, >= {cols}]")
+
+
 def _kdtype(K):
     return MISA_K_FP8E4M3 if K.dtype in (torch.uint8, torch.float8_e4m3fn) else MISA_K_BF16
 
@@ -112,6 +125,9 @@ def misa_pool_keys(K, B: int, k_scale=None, kbar=None, kbar_hl=None, want_kbar: 
         kbar = torch.empty((M, d), dtype=torch.float32, device=K.device)
     if kbar_hl is None:
         kbar_hl = torch.empty((2, M, d), dtype=torch.int16, device=K.device)
+    _need(k_scale, n_k, "k_scale")
+    _need(kbar, M * d, "kbar")
+    _need(kbar_hl, 2 * M * d, "kbar_hl")
     st = _lib.misa_pool_keys(_ptr(K, name="K"), _ptr(k_scale, (torch.float32,), "k_scale"),
                              _kdtype(K), n_k, d, B, _ptr(kbar, (torch.float32,), "kbar"),
                              _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), _stream())
@@ -126,6 +142,11 @@ def misa_pool_keys_range(K, B: int, m0: int, m1: int, kbar=None, kbar_hl=None, k
     if n_k is None:
         n_k = K.shape[0]
     d = K.shape[1]
+    M = -(-n_k // B) if B > 0 else 0
+    _need(K, n_k * d, "K")
+    _need(k_scale, n_k, "k_scale")
+    _need(kbar, M * d, "kbar")
+    _need(kbar_hl, 2 * M * d, "kbar_hl")
     st = _lib.misa_pool_keys_range(_ptr(K, name="K"), _ptr(k_scale, (torch.float32,), "k_scale"),
                                    _kdtype(K), n_k, d, B, m0, m1,
                                    _ptr(kbar, (torch.float32,), "kbar"),
@@ -141,6 +162,10 @@ def misa_route_heads(Q, w, kbar_hl, q_pos0: int, n_k: int, B: int, h: int, heads
     if heads is None:
         heads = torch.empty((n_q, h), dtype=torch.int32, device=Q.device)
     r = torch.empty((n_q, H), dtype=torch.float32, device=Q.device) if want_r else None
+    M = -(-n_k // B) if B > 0 else 0
+    _need(w, n_q * H, "w")
+    _need(kbar_hl, 2 * M * d, "kbar_hl")
+    _need(heads, n_q * h, "heads")
     st = _lib.misa_route_heads(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
                                _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), n_q, q_pos0, n_k, H, d, B, h,
                                _ptr(heads, (torch.int32,), "heads"), _ptr(r, (torch.float32,), "r"),
@@ -158,6 +183,13 @@ def misa_score_tokens(Q, w, heads, K, q_pos0: int, k_scale=None, logits=None, h:
     if logits is None:  # rows padded to 16 bytes (the kernel stores tiles by TMA)
         logits = torch.empty((n_q, (n_k + 3) // 4 * 4), dtype=torch.float32, device=Q.device)[:, :n_k]
     ld = logits.stride(0) if logits.dim() == 2 else n_k
+    _need(w, n_q * H, "w")
+    _need(heads, n_q * h, "heads")
+    _need(k_scale, n_k, "k_scale")
+    if logits.dim() == 2:
+        _need_rows(logits, n_q, n_k, "logits")
+    else:
+        _need(logits, n_q * n_k, "logits")
     st = _lib.misa_score_tokens(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
                                 _ptr(heads, (torch.int32,), "heads"), _ptr(K, name="K"),
                                 _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K), n_q, q_pos0,
@@ -180,6 +212,14 @@ def misa_score_tokens_fp8(Q8, q_scale, w, heads, K8, k_scale, q_pos0: int, logit
     if logits is None:
         logits = torch.empty((n_q, (n_k + 3) // 4 * 4), dtype=torch.float32, device=Q8.device)[:, :n_k]
     ld = logits.stride(0) if logits.dim() == 2 else n_k
+    _need(q_scale, n_q * H, "q_scale")
+    _need(w, n_q * H, "w")
+    _need(heads, n_q * h, "heads")
+    _need(k_scale, n_k, "k_scale")
+    if logits.dim() == 2:
+        _need_rows(logits, n_q, n_k, "logits")
+    else:
+        _need(logits, n_q * n_k, "logits")
     st = _lib.misa_score_tokens_fp8(_ptr(Q8, _E4M3_CODES, "Q8"), _ptr(q_scale, (torch.float32,), "q_scale"),
                                     _ptr(w, (torch.float32,), "w"), _ptr(heads, (torch.int32,), "heads"),
                                     _ptr(K8, _E4M3_CODES, "K8"), _ptr(k_scale, (torch.float32,), "k_scale"),
@@ -195,6 +235,8 @@ def misa_topk(logits, q_pos0: int, n_k: int, k: int, idx=None, n_q: int | None =
         n_q = logits.shape[0]
     if idx is None:
         idx = torch.empty((n_q, k), dtype=torch.int32, device=logits.device)
+    _need_rows(logits, n_q, min(n_k, q_pos0 + n_q), "logits")
+    _need(idx, n_q * k, "idx")
     st = _lib.misa_topk(ctypes.c_void_p(logits.data_ptr()), logits.stride(0), n_q, q_pos0, n_k, k,
                         _ptr(idx, (torch.int32,), "idx"), None, 0, _stream())
     _check("misa_topk", st)
@@ -217,6 +259,11 @@ def misa_score_topk(Q, w, heads, K, q_pos0: int, k: int, k_scale=None, h: int | 
         logits = torch.empty((n_q, (n_k + 3) // 4 * 4), dtype=torch.float32, device=Q.device)
     if logits.dim() != 2 or logits.stride(1) != 1 or logits.shape[0] < n_q:
         raise ValueError("logits must be a row-major [n_q, >= n_k] fp32 buffer")
+    _need(w, n_q * H, "w")
+    _need(heads, n_q * h, "heads")
+    _need(k_scale, n_k, "k_scale")
+    _need(idx, n_q * k, "idx")
+    _need_rows(logits, n_q, n_k, "logits")
     ws_bytes = misa_workspace_size("score_topk", n_q, n_k, k, 0)
     if ws_bytes and (ws is None or ws.numel() * ws.element_size() < ws_bytes):
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
@@ -243,6 +290,10 @@ def misa_rerank(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, want_full: boo
     if idx is None:
         idx = torch.empty((n_q, k), dtype=torch.int32, device=Q.device)
     full = torch.empty((n_q, kp), dtype=torch.float32, device=Q.device) if want_full else None
+    _need(w, n_q * H, "w")
+    _need(k_scale, n_k, "k_scale")
+    _need(cand, n_q * kp, "cand")
+    _need(idx, n_q * k, "idx")
     ws_bytes = 0
     if full is None:
         ws_bytes = misa_workspace_size("rerank", n_q, n_k, k, kp)
@@ -264,6 +315,10 @@ def misa_rerank_noalloc(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, idx=No
     kp = cand.shape[1]
     if idx is None:
         idx = torch.empty((n_q, k), dtype=torch.int32, device=Q.device)
+    _need(w, n_q * H, "w")
+    _need(k_scale, K.shape[0], "k_scale")
+    _need(cand, n_q * kp, "cand")
+    _need(idx, n_q * k, "idx")
     st = _lib.misa_rerank_noalloc(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
                                   _ptr(K, name="K"), _ptr(k_scale, (torch.float32,), "k_scale"),
                                   _kdtype(K), _ptr(cand, (torch.int32,), "cand"), kp, n_q, q_pos0,

@@ -146,3 +146,42 @@ def test_host_pipeline_pieces(lib):
         assert len(b) <= pieces
     sizes = [y - x for x, y in _piece_bounds(8192, 4)]
     assert sizes == [1024, 3072, 3072, 1024]
+
+
+def test_binding_refuses_undersized_buffers(lib):
+    # the C ABI sees pointers only: the binding checks the element counts the
+    # kernels will touch before anything is launched (CPU tensors: the size
+    # check comes first, the device check after it)
+    import torch
+    n_q, H, d, n_k, h, k = 4, 8, 64, 256, 2, 16
+    Q = torch.zeros((n_q, H, d), dtype=torch.int16)
+    K = torch.zeros((n_k, d), dtype=torch.int16)
+    w = torch.zeros((n_q, H), dtype=torch.float32)
+    heads = torch.zeros((n_q, h), dtype=torch.int32)
+
+    def size_error(fn, *a, **kw):
+        with pytest.raises(ValueError, match="the call needs"):
+            fn(*a, **kw)
+
+    def device_error(fn, *a, **kw):
+        with pytest.raises(ValueError, match="must be a CUDA tensor"):
+            fn(*a, **kw)
+
+    lg = torch.zeros((n_q, n_k), dtype=torch.float32)
+    device_error(lib.misa_score_tokens, Q, w, heads, K, 0, logits=lg, h=h)
+    size_error(lib.misa_score_tokens, Q, w[:3], heads, K, 0, logits=lg, h=h)
+    size_error(lib.misa_score_tokens, Q, w, heads[:, :1], K, 0, logits=lg, h=h)
+    size_error(lib.misa_score_tokens, Q, w, heads, K, 0, logits=lg[:, :n_k - 1], h=h)
+    size_error(lib.misa_score_tokens, Q, w, heads, K.to(torch.uint8), 0,
+               k_scale=torch.ones(n_k - 1), logits=lg, h=h)
+    size_error(lib.misa_score_tokens_fp8, Q.to(torch.uint8), torch.ones((n_q, H - 1)), w, heads,
+               K.to(torch.uint8), torch.ones(n_k), 0, logits=lg, h=h)
+    size_error(lib.misa_topk, lg[:, :2], 0, n_k, k)                # rows see up to n_q keys
+    device_error(lib.misa_topk, lg[:, :n_q], 0, n_k, k)
+    size_error(lib.misa_topk, lg, 0, n_k, k, idx=torch.zeros((n_q, k - 1), dtype=torch.int32))
+    size_error(lib.misa_route_heads, Q, w, torch.zeros((2, 3, d), dtype=torch.int16), 0, n_k, 64, h)
+    size_error(lib.misa_pool_keys, K, 64, kbar=torch.zeros((3, d)))
+    size_error(lib.misa_pool_keys_range, K[:100], 64, 0, 2, n_k=200)
+    size_error(lib.misa_rerank, Q, w, K, torch.zeros((n_q - 1, 32), dtype=torch.int32), 0, k)
+    size_error(lib.misa_score_topk, Q, w, heads, K, 0, k, h=h,
+               idx=torch.zeros((n_q, k - 1), dtype=torch.int32), logits=lg)
