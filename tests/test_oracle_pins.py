@@ -439,3 +439,45 @@ def test_select_candidates_agrees_with_rerank_on_exact_scores():
     idx, full = oracle.rerank(Q, w, K, cand, pos0, 5, want_logits=True)
     sel = oracle.select_candidates(full.astype(np.float32), cand, pos0, n_k, 5)
     assert np.array_equal(sel, idx)      # integer-valued scores: exact in fp32
+
+
+# ---------------------------------------------------------------- homogeneity
+
+@pytest.mark.parametrize("seed", range(3))
+def test_positive_scaling_of_keys_weights_and_queries(seed):
+    # ReLU is positively homogeneous and the scores are linear in w: scaling K,
+    # Q or w by a power of two c > 0 scales every router score and logit by c
+    # (exactly) and changes no selection; c < 0 on the keys flips which dot
+    # products the ReLU keeps, so the logits are NOT -c times the originals
+    Q, K, w, q_pos0 = _rand_case(seed, n_q=6, q_pos0=9, n_k=15, H=6, d=4)
+    B, h, k = 3, 3, 5
+    n_k = K.shape[0]
+    kbar = oracle.pool_keys(K, B)
+    r, heads = oracle.route(Q, w, kbar, q_pos0, n_k, B, h)
+    lg = oracle.score(Q, w, heads, K, q_pos0)
+    sel = oracle.topk(lg, q_pos0, n_k, k)
+    for c in (0.25, 4.0):
+        for which in ("K", "Q", "w"):
+            Q2, K2, w2 = (Q * c if which == "Q" else Q), (K * c if which == "K" else K), \
+                (w * c if which == "w" else w)
+            r2, heads2 = oracle.route(Q2, w2, oracle.pool_keys(K2, B), q_pos0, n_k, B, h)
+            assert np.array_equal(r2, r * c) and np.array_equal(heads2, heads)
+            lg2 = oracle.score(Q2, w2, heads, K2, q_pos0)
+            fin = np.isfinite(lg)
+            assert np.array_equal(lg2[fin], lg[fin] * c)
+            assert np.array_equal(oracle.topk(lg2, q_pos0, n_k, k), sel)
+    lg_neg = oracle.score(Q, w, heads, -K, q_pos0)
+    fin = np.isfinite(lg)
+    assert not np.allclose(lg_neg[fin], -lg[fin])
+
+
+def test_scores_are_linear_in_the_head_weights():
+    Q, K, w, q_pos0 = _rand_case(11, n_q=5, q_pos0=6, n_k=12, H=4, d=3)
+    heads = np.tile(np.array([0, 2, 3], dtype=np.int32), (5, 1))
+    rng = np.random.default_rng(12)
+    w2 = rng.standard_normal(w.shape)
+    a = oracle.score(Q, w, heads, K, q_pos0)
+    b = oracle.score(Q, w2, heads, K, q_pos0)
+    ab = oracle.score(Q, w + w2, heads, K, q_pos0)
+    fin = np.isfinite(a)
+    assert np.allclose(ab[fin], a[fin] + b[fin], rtol=1e-12, atol=1e-12)
