@@ -47,7 +47,7 @@ METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor 
 # queries of chunk_128k: the ncu capture of queries 0..1023 summarised in
 # profiles/score_select_chunk_128k.md, scaled by the query count; valid only for
 # the kernel sources it was taken on (null otherwise).
-SCORE_TRAFFIC = {"sources_sha256_16": "e5f68628459107c9", "bytes_per_launch": 8 * (168.861440e6 + 121.014528e6),
+SCORE_TRAFFIC = {"sources_sha256_16": "96ea2c45fccba3ae", "bytes_per_launch": 8 * (168.861440e6 + 121.014528e6),
                  "queries": 8192}
 
 

@@ -39,6 +39,11 @@
 //                        flagged by the fused top-k (nothing when none is).
 // Work is the flattened list of (query group, key tile) pairs, split evenly
 // over the CTAs, so causal triangles stay balanced.
+//
+// With e4m3 queries and keys (a scale per (query, head) row and per key) the
+// same roles run on one-byte operands: key tiles of 128 x d bytes, gathered
+// rows of d bytes, tcgen05.mma.kind::f8f6f4; the row scale is folded into the
+// head weight and the key scale multiplies the head-sum.
 #include <cstring>
 
 #include "internal.h"
