@@ -185,3 +185,33 @@ def test_binding_refuses_undersized_buffers(lib):
     size_error(lib.misa_rerank, Q, w, K, torch.zeros((n_q - 1, 32), dtype=torch.int32), 0, k)
     size_error(lib.misa_score_topk, Q, w, heads, K, 0, k, h=h,
                idx=torch.zeros((n_q, k - 1), dtype=torch.int32), logits=lg)
+
+
+def test_binding_checks_pass_for_well_sized_buffers(lib):
+    # every wrapper runs all of its size checks on correctly sized (CPU) tensors
+    # and stops only at the device check
+    import torch
+    n_q, H, d, n_k, h, k, kp, B = 4, 8, 64, 256, 2, 16, 32, 64
+    M = n_k // B
+    Q = torch.zeros((n_q, H, d), dtype=torch.int16)
+    K = torch.zeros((n_k, d), dtype=torch.int16)
+    K8 = torch.zeros((n_k, d), dtype=torch.uint8)
+    w = torch.zeros((n_q, H), dtype=torch.float32)
+    heads = torch.zeros((n_q, h), dtype=torch.int32)
+    lg = torch.zeros((n_q, n_k), dtype=torch.float32)
+    hl = torch.zeros((2, M, d), dtype=torch.int16)
+    calls = [
+        lambda: lib.misa_pool_keys(K, B, kbar=torch.zeros((M, d)), kbar_hl=hl),
+        lambda: lib.misa_pool_keys_range(K, B, 0, M, kbar_hl=hl),
+        lambda: lib.misa_route_heads(Q, w, hl, 0, n_k, B, h),
+        lambda: lib.misa_score_tokens(Q, w, heads, K, 0, logits=lg, h=h),
+        lambda: lib.misa_score_tokens_fp8(Q.to(torch.uint8), torch.ones((n_q, H)), w, heads, K8,
+                                          torch.ones(n_k), 0, logits=lg, h=h),
+        lambda: lib.misa_topk(lg, 0, n_k, k),
+        lambda: lib.misa_score_topk(Q, w, heads, K, 0, k, h=h, logits=lg),
+        lambda: lib.misa_rerank(Q, w, K, torch.zeros((n_q, kp), dtype=torch.int32), 0, k),
+        lambda: lib.misa_rerank_noalloc(Q, w, K, torch.zeros((n_q, kp), dtype=torch.int32), 0, k),
+    ]
+    for fn in calls:
+        with pytest.raises(ValueError, match="must be a CUDA tensor"):
+            fn()
