@@ -43,24 +43,6 @@ from long_context_sparse_block_b200 import workloads as W  # noqa: E402
 
 METRIC = "MISA indexer ms per 8192x131072 chunk; scoring TFLOP/s vs B200 tensor peak"
 
-# DRAM bytes (read + write) of one select-mode scoring launch over all 8192
-# queries of chunk_128k: the ncu capture of queries 0..1023 summarised in
-# profiles/score_select_chunk_128k.md, scaled by the query count; valid only for
-# the kernel sources it was taken on (null otherwise).
-SCORE_TRAFFIC = {"sources_sha256_16": "96ea2c45fccba3ae", "bytes_per_launch": 8 * (168.861440e6 + 121.014528e6),
-                 "queries": 8192}
-
-
-def _score_sources_digest():
-    import hashlib
-    h = hashlib.sha256()
-    for f in ("long_context_sparse_block_b200/csrc/score.cu",
-              "long_context_sparse_block_b200/csrc/common.cuh"):
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
-    return h.hexdigest()[:16]
-
-
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -161,31 +143,43 @@ def _oracle_worker(rows):
     return time.perf_counter() - t0, len(rows)
 
 
-def cpu_baseline(wl: W.Workload, h: int, inp: dict, budget_s: float = 15.0) -> dict:
-    """Times the oracle as it stands (route + score + top-k per query; keys pooled
-    once) on a seeded sample of query rows, one single-threaded oracle process per
-    core, and extrapolates to milliseconds per chunk.  Must run before any CUDA
-    call: the worker processes are forked."""
+def _oracle_setup(wl: W.Workload, h: int, inp: dict) -> int:
+    """Builds the oracle, pools the keys once and returns the worker count (one
+    single-threaded oracle process per host core, at most 32)."""
     import oracle
     oracle.build()
     try:
         cores = len(os.sched_getaffinity(0))
     except AttributeError:
         cores = os.cpu_count() or 1
-    workers = max(1, min(cores, 32))
     Kd = oracle.bf16_to_f64(inp["K"])
     _SHARED.update(wl=wl, h=h, inp=inp, Kd=Kd, kbar=oracle.pool_keys(Kd, wl.B))
+    return max(1, min(cores, 32))
+
+
+def _oracle_step(pool, workers: int, rows) -> tuple:
+    """One sample: the rows split over the worker processes.  Returns (wall s,
+    summed single-thread s, rows)."""
+    parts = [rows[i::workers].tolist() for i in range(workers)]
+    t0 = time.perf_counter()
+    res = pool.map(_oracle_worker, [p for p in parts if p])
+    return time.perf_counter() - t0, sum(t for t, _ in res), sum(n for _, n in res)
+
+
+def cpu_baseline(wl: W.Workload, h: int, inp: dict, budget_s: float = 15.0) -> dict:
+    """Times the oracle as it stands (route + score + top-k per query; keys pooled
+    once) on a seeded sample of query rows, one single-threaded oracle process per
+    core, and extrapolates to milliseconds per chunk.  Must run before any CUDA
+    call: the worker processes are forked."""
+    workers = _oracle_setup(wl, h, inp)
     rng = np.random.default_rng(12345)
     cal_t, _ = _oracle_worker([wl.n_q - 1])
     per_worker = max(1, min(64, int(budget_s / max(cal_t, 1e-3))))
     n_rows = min(wl.n_q, per_worker * workers)
     rows = np.sort(rng.choice(wl.n_q, size=n_rows, replace=False))
-    parts = [rows[i::workers].tolist() for i in range(workers)]
-    t0 = time.perf_counter()
     with mp.get_context("fork").Pool(workers) as pool:
-        res = pool.map(_oracle_worker, [p for p in parts if p])
-    wall = time.perf_counter() - t0
-    per_query = sum(t for t, _ in res) / sum(n for _, n in res)   # single-thread s/query
+        wall, busy, done = _oracle_step(pool, workers, rows)
+    per_query = busy / done   # single-thread s/query
     ms_chunk = per_query * wl.n_q / workers * 1e3
     return {"value": round(ms_chunk, 1), "unit": "ms", "cores": workers, "kind": "oracle",
             "sample": f"{n_rows} of {wl.n_q} query rows of {wl.name} (route + score + top-k "
@@ -357,18 +351,16 @@ def run_ours(args, rank, world, local_rank, inp):
 
     peaks = _peaks()
     pairs = wl.causal_pairs()
-    traffic = (SCORE_TRAFFIC["bytes_per_launch"]
-               if h == 8 and wl.name == "chunk_128k" and ix.sub == SCORE_TRAFFIC["queries"]
-               and _score_sources_digest() == SCORE_TRAFFIC["sources_sha256_16"] else None)
     score_flops = 2.0 * h * wl.d * pairs
     score_key = "select_score" if "select_score" in stage_ms else "score_topk"
     score_ms = stage_ms[score_key]
     tflops = score_flops / (score_ms * 1e-3) / 1e12
     pool_gbs = (wl.n_k * wl.d * 2 + 2 * wl.M * wl.d * 2) / (stage_ms["pool"] * 1e-3) / 1e9
-    # router: H_I * d multiply-adds per (query, complete causal block), done twice
-    # (hi and lo halves of the pooled keys)
+    # router: the method's work is H_I * d multiply-adds per (query, complete
+    # causal block); the kernel runs that contraction twice (the hi and lo bf16
+    # halves of the pooled keys), reported separately
     blocks = sum(min((p + 1) // wl.B, wl.n_k // wl.B) for p in wl.positions().tolist())
-    route_flops = 2.0 * 2.0 * wl.H * wl.d * blocks
+    route_flops = 2.0 * wl.H * wl.d * blocks
     route_tflops = route_flops / (stage_ms["route"] * 1e-3) / 1e12
     h2d = inp["Q"].nbytes + inp["K"].nbytes + inp["w"].nbytes
     d2h = idx_h.numel() * 4
@@ -402,15 +394,16 @@ def run_ours(args, rank, world, local_rank, inp):
             "unit": "TFLOP/s",
             "frac": round(tflops / peaks["bf16_tflops"], 4),
             "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
-            "traffic": traffic,
-            "traffic_unit": "bytes per launch (ncu dram read+write)",
+            "traffic": None,
             "algorithmic": f"2*h*d*pairs = {score_flops:.4g} flop per step, {pairs} causal pairs",
             "launches_per_step": math.ceil(wl.n_q / ix.sub),
         },
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "stage_rates": {
             "score_tflops": round(tflops, 1),
-            "route_tflops_hi_lo": round(route_tflops, 1),
+            "route_tflops": round(route_tflops, 1),
+            "route_frac": round(route_tflops / peaks["bf16_tflops"], 4),
+            "route_tflops_issued_hi_lo": round(2.0 * route_tflops, 1),
             "pool_gbs": round(pool_gbs, 1),
             "hbm_peak_gbs": peaks["hbm_gbs"],
             "pairs_per_s": round(pairs / (ms * 1e-3), 1),
@@ -577,23 +570,47 @@ def run_variants(wl, inp, stream, flush):
 
 
 def run_reference(args, rank):
+    """The oracle arm: W warm-up and K timed steps, each step the oracle over a
+    fresh seeded sample of query rows (one single-threaded process per host
+    core, about --ref-step-s seconds of wall time); a step's time is its wall
+    time, and the value is each step's time per row scaled to the whole chunk,
+    averaged over the timed steps."""
     if rank != 0:
         return None
     wl = W.WORKLOADS[args.workload]
     h = args.h or wl.h
-    t0 = time.perf_counter()
-    cb = cpu_baseline(wl, h, W.generate(wl), budget_s=args.cpu_budget)
+    t_start = time.perf_counter()
+    workers = _oracle_setup(wl, h, W.generate(wl))
+    cal_t, _ = _oracle_worker([wl.n_q - 1])
+    rows_per_step = min(wl.n_q, workers * max(1, int(args.ref_step_s / max(cal_t, 1e-3))))
+    rng = np.random.default_rng(54321)
+    walls, chunk_ms = [], []
+    with mp.get_context("fork").Pool(workers) as pool:
+        for i in range(args.warmup + args.steps):
+            rows = np.sort(rng.choice(wl.n_q, size=rows_per_step, replace=False))
+            wall, _, done = _oracle_step(pool, workers, rows)
+            if i >= args.warmup:
+                walls.append(wall)
+                chunk_ms.append(wall * wl.n_q / done * 1e3)
+    value = statistics.mean(chunk_ms)
     world = int(os.environ.get("WORLD_SIZE", 1))
-    return {"metric": METRIC, "value": cb["value"], "unit": "ms", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["value"],
+    return {"metric": METRIC, "value": round(value, 1), "unit": "ms", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(statistics.mean(walls) * 1e3, 1),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
+            "extrapolated": True,
             "config": {"workload": _workload_name(wl, h),
-                       "parallelism": "one host process pool (the oracle arm)"},
-            "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": "ms", "h2d_bytes_per_step": 0,
+                       "sample_rows_per_step": rows_per_step,
+                       "parallelism": f"{workers} single-threaded oracle processes on the host"},
+            "cpu_baseline": {"value": round(value, 1), "unit": "ms", "cores": workers,
+                             "kind": "oracle",
+                             "sample": f"each step: {rows_per_step} seeded query rows of "
+                                       f"{wl.n_q} (route + score + top-k each); the step's wall "
+                                       f"time scaled by {wl.n_q}/{rows_per_step}"},
+            "e2e": {"value": round(value, 1), "unit": "ms", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
-            "wall_s": round(time.perf_counter() - t0, 1)}
+            "wall_s": round(time.perf_counter() - t_start, 1)}
 
 
 def main():
@@ -606,6 +623,8 @@ def main():
     ap.add_argument("--h", type=int, default=0)
     ap.add_argument("--sub-chunk", type=int, default=8192)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-step-s", type=float, default=1.0,
+                    help="oracle arm: wall seconds per step (each step a sample of rows)")
     ap.add_argument("--queries", type=int, default=0,
                     help="index only the first N queries of the chunk (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -154,9 +154,12 @@ int misa_topk(const float* logits, int64_t ld, int n_q, int64_t q_pos0, int64_t 
  *   full[t, i] = sum_{j < H} w[t, j] * ReLU(q[t, j] . k_{c}),  c = cand[t, i]
  * Entries c outside 0..pos(t) (including the -1 padding) are ignored.  The k
  * candidates of largest full score, ties to the lower token index, are written
- * ascending to idx[t, :], -1 padded.  full_logits (nullable, [n_q, kp]) receives
- * full, -inf where ignored.  Candidates must be distinct.  H <= 128 and a
- * multiple of 16; 1 <= kp <= 16384; 0 <= k <= kp.
+ * ascending to idx[t, :], -1 padded, whatever order a row's candidates come in
+ * (rows whose valid candidates ascend, as the coarse selection emits them,
+ * take a faster path).  full_logits (nullable, [n_q, kp]) receives full, -inf
+ * where ignored.  The valid candidates of a row must be distinct: a token kept
+ * twice records MISA_ERR_DEVICE in the device status.  H <= 128; 1 <= kp <=
+ * 16384; 0 <= k <= kp.
  * ws/ws_bytes: workspace, size from misa_workspace_size("rerank", ...).
  */
 int misa_rerank(const uint16_t* Q, const float* w, const void* K, const float* k_scale, int kdtype,

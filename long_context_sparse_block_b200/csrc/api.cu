@@ -290,7 +290,7 @@ int misa_topk(const float* logits, int64_t ld, int n_q, int64_t q_pos0, int64_t 
   DevCtl ctl;
   if (!make_ctl(ctl)) return MISA_ERR_CUDA;
   return cuda_status(
-      launch_topk(logits, ld, n_q, q_pos0, n_k, 0, nullptr, k, idx, ctl, as_stream(stream)));
+      launch_topk(logits, ld, n_q, q_pos0, n_k, k, idx, ctl, as_stream(stream)));
 }
 
 int misa_rerank(const uint16_t* Q, const float* w, const void* K, const float* k_scale, int kdtype,
@@ -320,7 +320,7 @@ int misa_rerank(const uint16_t* Q, const float* w, const void* K, const float* k
                                        q_pos0, n_k, H, d, full, kp, ctl, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   if (k == 0) return MISA_OK;
-  return cuda_status(launch_topk(full, kp, n_q, q_pos0, n_k, kp, cand, k, idx, ctl, s));
+  return cuda_status(launch_select_candidates(full, kp, cand, kp, n_q, q_pos0, n_k, k, idx, ctl, s));
 }
 
 int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
@@ -365,7 +365,7 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
   if (!fused) {  // unfused: every logit, then the selection
     cudaError_t e = launch_score(a, ctl, s);
     if (e != cudaSuccess) return MISA_ERR_CUDA;
-    return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, 0, nullptr, k, idx, ctl, s));
+    return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, k, idx, ctl, s));
   }
   const FusedLayout L(n_q, n_k);
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -430,7 +430,7 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
   }
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   StageMark m(6, s);
-  return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, 0, nullptr, k, idx, ctl, s, gate));
+  return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, k, idx, ctl, s, gate));
 }
 
 int misa_profile_start(void) {

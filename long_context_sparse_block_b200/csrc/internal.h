@@ -58,13 +58,18 @@ cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t
                                 int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
                                 int64_t ld, const DevCtl& ctl, cudaStream_t s);
 
-// Top-k over rows.  Token mode (cand == nullptr): row t is logits[t*ld ..] with
-// min(pos(t)+1, n_k) visible entries; writes token indices.  Candidate mode:
-// row t is vals[t*ld .. t*ld+row_len); -inf entries are absent; writes
-// cand[t*row_len + i] for the selected positions i.
+// Top-k over token rows: row t is vals[t*ld ..] with min(pos(t)+1, n_k)
+// visible entries; writes token indices.
 cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k,
-                        int row_len, const int32_t* cand, int k, int32_t* idx,
-                        const DevCtl& ctl, cudaStream_t s, const int* gate = nullptr);
+                        int k, int32_t* idx, const DevCtl& ctl, cudaStream_t s,
+                        const int* gate = nullptr);
+
+// Top-k over candidate rows: row t holds the scores vals[t*ldv + i] of tokens
+// cand[t*kp + i] (absent: token outside 0..pos(t), or -inf); ties to the lower
+// token; tokens written ascending whatever the candidate order (kp <= 16384).
+cudaError_t launch_select_candidates(const float* vals, int64_t ldv, const int32_t* cand, int kp,
+                                     int n_q, int64_t q_pos0, int64_t n_k, int k, int32_t* idx,
+                                     const DevCtl& ctl, cudaStream_t s);
 
 // Exact decode of FP8 E4M3 key codes to bf16 codes (pool.cu); n multiple of 16.
 cudaError_t launch_e4m3_to_bf16(const uint8_t* src, uint16_t* dst, int64_t n, cudaStream_t s);

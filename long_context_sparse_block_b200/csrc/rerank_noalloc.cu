@@ -84,7 +84,8 @@ extern "C" int misa_rerank_noalloc(const uint16_t* Q, const float* w, const void
                            H, d, scratch, kp, ctl, s) != cudaSuccess)
     return MISA_ERR_CUDA;
   if (k == 0) return MISA_OK;
-  return launch_topk(scratch, kp, n_q, q_pos0, n_k, kp, cand, k, idx, ctl, s) == cudaSuccess
+  return launch_select_candidates(scratch, kp, cand, kp, n_q, q_pos0, n_k, k, idx, ctl, s) ==
+                     cudaSuccess
              ? MISA_OK
              : MISA_ERR_CUDA;
 }

@@ -3,10 +3,10 @@
 // For each row keep the k largest values, ties to the lower position, and
 // write the kept positions in ascending order, padded with -1 ("MISA"
 // technical summary, Metodologia step 2: the final top-k tokens are chosen from
-// the routed scores).  Two row kinds share the kernel:
-//   token rows      logits[t, 0 .. min(pos(t), n_k-1)]; output = token index;
-//   candidate rows  full[t, 0 .. kp-1] (-inf = absent); output = cand[t, i]
-//                   (MISA-dagger: final top-k among the re-scored candidates).
+// the routed scores).  Token rows are logits[t, 0 .. min(pos(t), n_k-1)] and
+// the output is the token index.  Candidate rows (MISA-dagger, Variante
+// Hierarquica: the final top-k among the re-scored candidates) have a kernel of
+// their own at the end of this file.
 //
 // Values are mapped to order-preserving 32-bit keys (-0.0 folded onto +0.0,
 // -inf and padding to the reserved key 0).  One CTA per row.
@@ -58,8 +58,6 @@ struct TopkParams {
   int n_q;
   int64_t q_pos0;
   int64_t n_k;
-  int row_len;           // candidate rows only
-  const int32_t* cand;   // nullptr: token rows
   int k;
   int32_t* idx;
   int cap;               // shared-memory list capacity (entries)
@@ -177,12 +175,12 @@ struct ListEmit {
   }
 };
 
+// Writes the position (a token index) of a kept entry to its output slot.
 struct OutEmit {
   int32_t* out;           // idx row
-  const int32_t* cand;    // candidate row or nullptr
   uint32_t k;
   __device__ __forceinline__ void operator()(uint32_t slot, uint32_t, uint32_t pos) const {
-    if (slot < k) out[slot] = cand ? __ldg(cand + pos) : static_cast<int32_t>(pos);
+    if (slot < k) out[slot] = static_cast<int32_t>(pos);
   }
 };
 
@@ -539,17 +537,10 @@ topk_kernel(const TopkParams p) {
 
   const int t = blockIdx.x;
   const uint32_t k = static_cast<uint32_t>(p.k);
-  int64_t n;
-  const int32_t* cand_row = nullptr;
-  if (p.cand) {
-    n = p.row_len;
-    cand_row = p.cand + static_cast<int64_t>(t) * p.row_len;
-  } else {
-    n = min(p.q_pos0 + t + 1, p.n_k);
-  }
+  const int64_t n = min(p.q_pos0 + t + 1, p.n_k);
   const float* row = p.vals + static_cast<int64_t>(t) * p.ld;
   const RowSrc src{row, n, (reinterpret_cast<uintptr_t>(row) & 15u) == 0u};
-  const OutEmit out{p.idx + static_cast<int64_t>(t) * p.k, cand_row, k};
+  const OutEmit out{p.idx + static_cast<int64_t>(t) * p.k, k};
   if (k == 0) return;
   if (k <= static_cast<uint32_t>(kFastMaxK) && n <= 32 * kBins1 &&
       topk_fast(p, src, out, hist, lkeys, lposs, sel, counts, sc))
@@ -749,7 +740,7 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
   }
   __syncthreads();
   const ListSrc ls{keys, poss, static_cast<int64_t>(total)};
-  const OutEmit out{idx + static_cast<int64_t>(t) * k, nullptr, static_cast<uint32_t>(k)};
+  const OutEmit out{idx + static_cast<int64_t>(t) * k, static_cast<uint32_t>(k)};
   uint32_t T = 0u, need = 0u;
   if (total > static_cast<uint32_t>(k)) T = kth_largest(ls, static_cast<uint32_t>(k), hist, sc, need);
   const uint32_t kept = ordered_select(ls, T, need, static_cast<uint32_t>(k), out, sc);
@@ -758,11 +749,107 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
     out.out[i] = -1;
 }
 
+// ---------------------------------------------------------------- candidate rows
+// MISA-dagger final selection (Variante Hierarquica: the top-k among the
+// re-scored candidates).  Row t holds the all-head scores vals[t*ldv + i] of
+// the candidate tokens cand[t*kp + i]; a candidate is absent when its token
+// lies outside 0..pos(t) (the -1 padding included) or its score is -inf.  The
+// k present candidates of largest score are kept, ties to the lower TOKEN, and
+// their tokens written ascending, -1 padded, whatever order the candidates
+// come in.  The row (scores as order-preserving keys, and tokens) is staged in
+// shared memory; three radix rounds over it give the exact k-th key T.
+//   ascending rows (present tokens strictly increasing, absent entries only at
+//   the end, which is what the coarse selection emits): one ordered pass, since
+//   position order is token order;
+//   any other row: the tokens tied at T are sorted and the lowest kept, then
+//   the kept tokens are sorted and written.  Two kept entries with the same
+//   token break the contract (distinct candidates) and are reported.
+__global__ void __launch_bounds__(kTopkThreads)
+select_candidates_kernel(const float* __restrict__ vals, int64_t ldv,
+                         const int32_t* __restrict__ cand, int kp, int64_t q_pos0, int64_t n_k,
+                         int k, int32_t* __restrict__ idx, int tmp_cap, DevCtl ctl) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
+  uint32_t* toks = keys + kp;
+  uint32_t* tmp = toks + kp;  // tmp_cap entries: the next power of two >= kp
+  const int t = blockIdx.x;
+  const int64_t pos = q_pos0 + t;
+  const float* vrow = vals + static_cast<int64_t>(t) * ldv;
+  const int32_t* crow = cand + static_cast<int64_t>(t) * kp;
+  int32_t* out = idx + static_cast<int64_t>(t) * k;
+  const uint32_t kk = static_cast<uint32_t>(k);
+
+  auto stage = [&](int i, float v, int32_t tok) {
+    const bool valid = tok >= 0 && tok <= pos && tok < n_k;
+    const uint32_t key = valid ? f2key(v) : 0u;
+    keys[i] = key;
+    toks[i] = static_cast<uint32_t>(tok);
+    return key != 0u ? 1u : 0u;
+  };
+  uint32_t c = 0;
+  const bool vec = (kp & 3) == 0 && (reinterpret_cast<uintptr_t>(vrow) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(crow) & 15u) == 0;
+  if (vec) {
+    for (int i = threadIdx.x * 4; i < kp; i += kTopkThreads * 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(vrow + i));
+      const int4 tk = __ldg(reinterpret_cast<const int4*>(crow + i));
+      c += stage(i, v.x, tk.x) + stage(i + 1, v.y, tk.y) + stage(i + 2, v.z, tk.z) +
+           stage(i + 3, v.w, tk.w);
+    }
+  } else {
+    for (int i = threadIdx.x; i < kp; i += kTopkThreads) c += stage(i, __ldg(vrow + i), __ldg(crow + i));
+  }
+  uint32_t present;
+  block_excl_scan(c, sc, present);  // (also orders the stores above before the reads below)
+  bool unordered = false;
+  for (int i = threadIdx.x; i + 1 < kp; i += kTopkThreads)
+    if (keys[i + 1] != 0u && (keys[i] == 0u || toks[i] >= toks[i + 1])) unordered = true;
+  unordered = __syncthreads_or(unordered) != 0;
+
+  const ListSrc ls{keys, toks, static_cast<int64_t>(kp)};
+  uint32_t T = 0u, need = 0u;  // present <= k: every present entry (key > 0)
+  if (present > kk) T = kth_largest(ls, kk, hist, sc, need);
+  if (!unordered) {
+    const uint32_t kept = ordered_select(ls, T, need, kk, OutEmit{out, kk}, sc);
+    for (uint32_t i = min(kept, kk) + threadIdx.x; i < kk; i += kTopkThreads) out[i] = -1;
+    return;
+  }
+  // tokens tied at T: keep the `need` lowest (those <= cut)
+  uint32_t cut = 0xFFFFFFFFu;
+  if (present > kk) {
+    if (threadIdx.x == 0) sc.res[2] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < kp; i += kTopkThreads)
+      if (keys[i] == T) tmp[atomicAdd(&sc.res[2], 1u)] = toks[i];
+    __syncthreads();
+    const uint32_t n_eq = sc.res[2];
+    if (n_eq > need) {
+      bitonic_sort_asc(tmp, n_eq);
+      cut = tmp[need - 1];
+    }
+  }
+  if (threadIdx.x == 0) sc.res[3] = 0u;
+  __syncthreads();  // every thread has read cut before tmp is refilled
+  for (int i = threadIdx.x; i < kp; i += kTopkThreads) {
+    const uint32_t key = keys[i];
+    if (key > T || (key == T && key != 0u && toks[i] <= cut)) tmp[atomicAdd(&sc.res[3], 1u)] = toks[i];
+  }
+  __syncthreads();
+  const uint32_t n_win = min(sc.res[3], static_cast<uint32_t>(tmp_cap));
+  bitonic_sort_asc(tmp, n_win);
+  bool dup = false;
+  for (uint32_t i = threadIdx.x; i + 1 < n_win; i += kTopkThreads) dup |= tmp[i] == tmp[i + 1];
+  if (__syncthreads_or(dup) && threadIdx.x == 0) report(ctl, DEV_BAD_INPUT);
+  for (uint32_t i = threadIdx.x; i < kk; i += kTopkThreads)
+    out[i] = i < n_win ? static_cast<int32_t>(tmp[i]) : -1;
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k,
-                        int row_len, const int32_t* cand, int k, int32_t* idx,
-                        const DevCtl& ctl, cudaStream_t s, const int* gate) {
+                        int k, int32_t* idx, const DevCtl& ctl, cudaStream_t s, const int* gate) {
   if (n_q <= 0 || k <= 0) return cudaSuccess;
   // list capacity: kFastCap for k <= 4096 (three CTAs per SM); larger k need
   // room for ~1.4 k sampled-threshold entries (fast path) or for the entries in
@@ -773,7 +860,7 @@ cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, 
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  TopkParams p{vals, ld, n_q, q_pos0, n_k, row_len, cand, k, idx, cap, ctl, gate};
+  TopkParams p{vals, ld, n_q, q_pos0, n_k, k, idx, cap, ctl, gate};
   topk_kernel<<<n_q, kTopkThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
@@ -793,6 +880,22 @@ cudaError_t launch_fused_tau(const float* sample, int64_t lds, int n_s, int n_q,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   fused_tau_kernel<<<n_q, kTopkThreads, smem, s>>>(sample, lds, n_s, q_pos0, n_k, k, tau, gate);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_candidates(const float* vals, int64_t ldv, const int32_t* cand, int kp,
+                                     int n_q, int64_t q_pos0, int64_t n_k, int k, int32_t* idx,
+                                     const DevCtl& ctl, cudaStream_t s) {
+  if (n_q <= 0 || k <= 0 || kp <= 0) return cudaSuccess;
+  int cap = 1;
+  while (cap < kp) cap <<= 1;
+  const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + (2 * static_cast<size_t>(kp) + cap) * 4;
+  cudaError_t e = cudaFuncSetAttribute(select_candidates_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  select_candidates_kernel<<<n_q, kTopkThreads, smem, s>>>(vals, ldv, cand, kp, q_pos0, n_k, k,
+                                                           idx, cap, ctl);
   return cudaGetLastError();
 }
 

@@ -68,8 +68,15 @@ def test_full_size_sampled_rows(name):
 
 @pytest.mark.parametrize("fp8", [False, True])
 def test_full_size_dagger_sampled_rows(fp8):
-    # MISA-dagger on the 8192 x 131072 chunk; fp8=True stores the keys as e4m3
-    # with a per-token scale for every stage (pool, route, score, rerank)
+    # MISA-dagger on the 8192 x 131072 chunk (k' = 8192 -> k = 2048); fp8=True
+    # stores the keys as e4m3 with a per-token scale for every stage (pool,
+    # route, score, rerank).  Per sampled row: the routed heads against the
+    # oracle's, the routed logits against the oracle's where the heads agree,
+    # the coarse candidates bit-exact against the oracle's top-k' of the GPU's
+    # own logits, the all-head scores of those candidates against the oracle's,
+    # and the final selection bit-exact against the oracle's rule on the GPU's
+    # own scores (the launch configuration of the benchmark's MISA-dagger run).
+    from long_context_sparse_block_b200 import _lib
     from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
     wl = W.WORKLOADS["dagger_128k"]
     inp = W.generate(wl, fp8_keys=fp8)
@@ -78,23 +85,59 @@ def test_full_size_dagger_sampled_rows(fp8):
     ix = MisaIndexer(IndexerShape(wl.n_q, wl.q_pos0, wl.n_k, wl.H, wl.d, wl.B, wl.h, wl.k,
                                   kp=wl.kp, sub_chunk=1024))
     K = g["K8"] if fp8 else g["K"]
-    fin = ix.run(g["Q"], K, g["w"], k_scale=g.get("k_scale")).cpu().numpy()
+    ksc = g.get("k_scale")
+    dumps = {}
+
+    def grab(c0, c1, lg):
+        for t in rows:
+            if c0 <= t < c1:
+                dumps[t] = lg[t - c0].cpu().numpy()
+
+    fin = ix.run(g["Q"], K, g["w"], k_scale=ksc, on_subchunk=grab).cpu().numpy()
     cand = ix.sel.cpu().numpy()
     heads = ix.heads.cpu().numpy()
+    # the fused coarse pass (the product path) selects the same candidates
+    fused = ix.run(g["Q"], K, g["w"], k_scale=ksc).cpu().numpy()
+    assert np.array_equal(ix.sel.cpu().numpy(), cand)
+    assert np.array_equal(fused, fin)
+    assert _lib.misa_last_device_status() == 0
     Kd = oracle.e4m3_keys_to_f64(inp["K8"], inp["k_scale"]) if fp8 else oracle.bf16_to_f64(inp["K"])
     kbar = oracle.pool_keys(Kd, wl.B)
     sel = np.array(rows)
     Qd = oracle.bf16_to_f64(inp["Q"][sel])
     wd = inp["w"][sel].astype(np.float64)
+    matched = 0
     for i, t in enumerate(rows):
         pos = wl.q_pos0 + t
-        _, h_o = oracle.route(Qd[i:i + 1], wd[i:i + 1], kbar, pos, wl.n_k, wl.B, wl.h)
-        if not np.array_equal(heads[t], h_o[0]):
-            continue
-        # the fine stage on the GPU's own candidates, in fp64
-        ref = oracle.rerank(Qd[i:i + 1], wd[i:i + 1], Kd, cand[t:t + 1], pos, wl.k)
-        assert recall(fin[t:t + 1], ref) >= 0.999
+        r_o, h_o = oracle.route(Qd[i:i + 1], wd[i:i + 1], kbar, pos, wl.n_k, wl.B, wl.h)
+        check_heads(heads[t:t + 1], r_o, h_o, wl.h)
+        lg_gpu = dumps[t]
+        # coarse stage: bit-exact on the GPU's own routed logits
+        assert np.array_equal(cand[t], oracle.topk(lg_gpu[None, :], pos, wl.n_k, wl.kp)[0])
+        if np.array_equal(heads[t], h_o[0]):
+            matched += 1
+            ref_lg = oracle.score(Qd[i:i + 1], wd[i:i + 1], h_o, Kd, pos)[0]
+            hs = h_o[0]
+            mag = (np.abs(wd[i, hs])[:, None] * np.maximum(Qd[i, hs] @ Kd[:pos + 1].T, 0)).sum(0)
+            assert_logits_close(lg_gpu, ref_lg[:pos + 1], mag, what=f"dagger row {t}")
+        # fine stage: the GPU's all-head scores of this row's candidates (the
+        # kernel scores each candidate the same way whatever the batch)
+        idx1, full1 = _lib.misa_rerank(g["Q"][t:t + 1], g["w"][t:t + 1], K,
+                                        ix.sel[t:t + 1].contiguous(), pos, wl.k, k_scale=ksc,
+                                        want_full=True)
+        idx1, full1 = idx1.cpu().numpy(), full1.cpu().numpy()
+        assert np.array_equal(idx1[0], fin[t])
+        assert np.array_equal(fin[t], oracle.select_candidates(full1, cand[t:t + 1], pos,
+                                                               wl.n_k, wl.k)[0])
+        ref_idx, ref_full = oracle.rerank(Qd[i:i + 1], wd[i:i + 1], Kd, cand[t:t + 1], pos, wl.k,
+                                          want_logits=True)
+        valid = cand[t] >= 0
+        dots = Qd[i] @ Kd[cand[t, valid]].T
+        mag = (np.abs(wd[i])[:, None] * np.maximum(dots, 0.0)).sum(axis=0)
+        assert np.all(np.abs(full1[0, valid] - ref_full[0, valid]) <= 2e-3 * mag + 1e-5)
+        assert recall(fin[t:t + 1], ref_idx) >= 0.999
         assert np.all(np.diff(fin[t][fin[t] >= 0]) > 0)
+    assert matched >= len(rows) - 2
 
 
 @pytest.mark.parametrize("name,sub", [("chunk_128k", 8192), ("chunk_128k_h4", 8192),

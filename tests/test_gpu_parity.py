@@ -301,8 +301,10 @@ def test_topk_fewer_tokens_than_k(lib):
 # ------------------------------------------------------------------ MISA-dagger rerank
 
 @pytest.mark.parametrize("fp8,H,d,kp,k", [(False, 64, 128, 256, 64), (True, 64, 128, 256, 64),
-                                          (False, 8, 32, 100, 30), (False, 32, 64, 384, 128)])
+                                          (False, 8, 32, 100, 30), (False, 32, 64, 384, 128),
+                                          (False, 64, 128, 256, 256), (True, 16, 64, 128, 128)])
 def test_rerank_matches_oracle(lib, fp8, H, d, kp, k):
+    # k == kp (the last two cases): every valid candidate is kept
     n_q, q_pos0, n_k, B, h = 40, 500, 600, 64, 4 if H > 8 else 2
     wl = _wl(n_q, q_pos0, n_k, H, d, B, h, k, seed=kp + H, kp=kp)
     inp = W.generate(wl, fp8_keys=fp8)
@@ -340,9 +342,84 @@ def test_rerank_whole_prefix_is_dense_topk(lib):
     cand = np.full((n_q, kp), -1, dtype=np.int32)
     for t in range(n_q):
         cand[t, :q_pos0 + t + 1] = np.arange(q_pos0 + t + 1)
-    idx = lib.misa_rerank(g["Q"], g["w"], g["K"], dev(cand), q_pos0, k).cpu().numpy()
+    idx, full = lib.misa_rerank(g["Q"], g["w"], g["K"], dev(cand), q_pos0, k, want_full=True)
+    idx, full = idx.cpu().numpy(), full.cpu().numpy()
+    # bit-exact against the oracle's rule on the GPU's own scores
+    assert np.array_equal(idx, oracle.select_candidates(full, cand, q_pos0, n_k, k))
+    # and the GPU's scores of the whole prefix, selected with the plain token
+    # top-k, give the same tokens
+    rows = np.full((n_q, n_k), -np.inf, dtype=np.float32)
+    for t in range(n_q):
+        rows[t, :q_pos0 + t + 1] = full[t, :q_pos0 + t + 1]
+    assert np.array_equal(idx, oracle.topk(rows, q_pos0, n_k, k))
     dense_ref = oracle.topk(oracle.dense_logits(Qd, wd, Kd, q_pos0), q_pos0, n_k, k)
     assert recall(idx, dense_ref) >= 0.999
+
+
+def _rerank_case(lib, seed, n_q=40, q_pos0=500, n_k=600, H=64, d=128, kp=256, k=64):
+    inp = W.generate(_wl(n_q, q_pos0, n_k, H, d, 64, 8, k, seed=seed, kp=kp))
+    g = inputs_to_device(inp)
+    _, hl = lib.misa_pool_keys(g["K"], 64)
+    heads, _ = lib.misa_route_heads(g["Q"], g["w"], hl, q_pos0, n_k, 64, 8)
+    logits = lib.misa_score_tokens(g["Q"], g["w"], heads, g["K"], q_pos0)
+    cand = lib.misa_topk(logits, q_pos0, n_k, kp)
+    return g, cand
+
+
+@pytest.mark.parametrize("k", [64, 256])
+def test_rerank_any_candidate_order(lib, k):
+    # candidates in a shuffled order (the -1 padding spread through the row,
+    # some rows reversed): ties still go to the lower token and the tokens come
+    # out ascending, equal to the selection from the ascending candidates
+    n_q, q_pos0, n_k, kp = 40, 150, 600, 256     # rows 0..105 see fewer than kp tokens
+    g, cand = _rerank_case(lib, seed=91, n_q=n_q, q_pos0=q_pos0, n_k=n_k, kp=kp, k=k)
+    want, full_sorted = lib.misa_rerank(g["Q"], g["w"], g["K"], cand, q_pos0, k, want_full=True)
+    rng = np.random.default_rng(92)
+    c = cand.cpu().numpy()
+    shuf = np.stack([c[t, ::-1] if t % 3 == 0 else c[t, rng.permutation(kp)] for t in range(n_q)])
+    shuf = np.ascontiguousarray(shuf)
+    got, full = lib.misa_rerank(g["Q"], g["w"], g["K"], dev(shuf), q_pos0, k, want_full=True)
+    assert lib.misa_last_device_status() == lib.MISA_OK
+    got, full = got.cpu().numpy(), full.cpu().numpy()
+    assert np.array_equal(got, oracle.select_candidates(full, shuf, q_pos0, n_k, k))
+    assert np.array_equal(got, want.cpu().numpy())
+    # a candidate's score does not depend on where it sits in the row
+    fs = full_sorted.cpu().numpy()
+    for t in range(n_q):
+        by_tok = dict(zip(c[t].tolist(), fs[t].tolist()))
+        for tok, v in zip(shuf[t].tolist(), full[t].tolist()):
+            assert v == by_tok[tok] or (tok < 0 and v == -np.inf)
+
+
+def test_rerank_ties_in_any_order(lib):
+    # every candidate of a row scores the same (identical keys): the k lowest
+    # tokens are kept whatever the candidate order
+    n_q, q_pos0, n_k, H, d, kp, k = 16, 900, 1000, 64, 128, 300, 100
+    inp = W.generate(_wl(n_q, q_pos0, n_k, H, d, 64, 8, k, seed=93, kp=kp))
+    g = inputs_to_device(inp)
+    K = g["K"][:1].expand(n_k, d).contiguous()
+    rng = np.random.default_rng(94)
+    cand = np.stack([rng.choice(q_pos0 + t + 1, size=kp, replace=False)
+                     for t in range(n_q)]).astype(np.int32)
+    got, full = lib.misa_rerank(g["Q"], g["w"], K, dev(cand), q_pos0, k, want_full=True)
+    assert lib.misa_last_device_status() == lib.MISA_OK
+    got, full = got.cpu().numpy(), full.cpu().numpy()
+    for t in range(n_q):
+        assert np.all(full[t] == full[t, 0])
+        assert np.array_equal(got[t], np.sort(cand[t])[:k])
+    assert np.array_equal(got, oracle.select_candidates(full, cand, q_pos0, n_k, k))
+
+
+def test_rerank_reports_repeated_candidates(lib):
+    # a token listed twice breaks the contract: the kernel reports it in the
+    # device status (all candidates kept, so the repeat is among the kept)
+    g, cand = _rerank_case(lib, seed=95, kp=128, k=128)
+    c = cand.cpu().numpy().copy()
+    c[3, 7] = c[3, 11]
+    lib.misa_rerank(g["Q"], g["w"], g["K"], dev(c), 500, 128)
+    assert lib.misa_last_device_status() == lib.MISA_ERR_DEVICE
+    lib.misa_rerank(g["Q"], g["w"], g["K"], cand, 500, 128)
+    assert lib.misa_last_device_status() == lib.MISA_OK
 
 
 # ------------------------------------------------------------------ whole path
