@@ -493,6 +493,28 @@ def run_variants(wl, inp, stream, flush):
     out["dagger_fp8_recall_vs_dense_bf16"] = round(_recall(fin8, dense_bf.run(Q, K, w), wl.n_k), 4)
     del dense_bf, dg8, fin8, ref8, K8, ks     # (K8c, sc stay on the host)
 
+    # the same chunk with its keys in a paged cache (pages of 64 keys in a
+    # seeded random order in a larger pool, unused rows filled with +inf codes):
+    # the indices must equal the contiguous ones
+    from long_context_sparse_block_b200 import _lib as L
+    ps = 64
+    table, n_pages = Wm.page_table(wl.n_k, ps, seed=64)
+    pages = torch.full((n_pages, ps, wl.d), 0x7F80, dtype=torch.int16, device="cuda")
+    bt = torch.from_numpy(table).cuda()
+    n_blocks = len(table)
+    flat = torch.full((n_blocks * ps, wl.d), 0x7F80, dtype=torch.int16, device="cuda")
+    flat[:wl.n_k] = K
+    pages[bt.long()] = flat.view(n_blocks, ps, wl.d)
+    del flat
+    pk = L.PagedKeys(pages, bt, wl.n_k)
+    ixp = MisaIndexer(IndexerShape(h=wl.h, **base))
+    out["paged_chunk_ms"] = round(_time_ms(lambda: ixp.run(Q, pk, w), stream, flush), 4)
+    sel_p = ixp.run(Q, pk, w).clone()
+    sel_c = ixp.run(Q, K, w)
+    out["paged_chunk_equal_contiguous"] = bool(torch.equal(sel_p, sel_c))
+    out["paged_page_size"] = ps
+    del ixp, pk, pages, bt, sel_p, sel_c
+
     # the unfused sequence on the chunk: every logit written (store mode), then
     # the standalone top-k reading them once (HBM-bound: 4 bytes per causal pair)
     from long_context_sparse_block_b200 import _lib
@@ -540,6 +562,45 @@ def run_variants(wl, inp, stream, flush):
         _lib.misa_topk(lg1, wl.n_k - 1, wl.n_k, wl.k, idx=idx1)
 
     out["decode_step_ms"] = round(_time_ms(decode_step, stream, flush), 4)
+
+    # batched decode: 64 sequences of 131072 keys each in one page pool (every
+    # sequence its own copy of the chunk's keys in its own seeded page order),
+    # one new query each (rows of the chunk's queries): re-pool each
+    # sequence's last block, route, score and select, three launches plus the
+    # top-k
+    n_seq, ps = 64, 64
+    nb = wl.n_k // ps
+    table, n_pages = Wm.page_table(n_seq * wl.n_k, ps, seed=65)
+    pages = torch.empty((n_pages, ps, wl.d), dtype=torch.int16, device="cuda")
+    bts = torch.from_numpy(table.reshape(n_seq, nb).copy()).cuda()
+    Kp = K.view(nb, ps, wl.d)
+    for b in range(n_seq):
+        pages[bts[b].long()] = Kp
+    del Kp
+    seq_lens = torch.full((n_seq,), wl.n_k, dtype=torch.int32, device="cuda")
+    Qd = Q[-n_seq:].contiguous()
+    wd = w[-n_seq:].contiguous()
+    M_max = -(-wl.n_k // wl.B)
+    _, hl_d = _lib.misa_decode_pool_keys(pages, bts, seq_lens, wl.B, M_max, M_max)
+    heads_d = torch.empty((n_seq, wl.h), dtype=torch.int32, device="cuda")
+    idx_d = torch.empty((n_seq, wl.k), dtype=torch.int32, device="cuda")
+    lg_d = torch.empty((n_seq, wl.n_k), dtype=torch.float32, device="cuda")
+
+    def decode_batch():
+        _lib.misa_decode_pool_keys(pages, bts, seq_lens, wl.B, M_max, 1, kbar_hl=hl_d)
+        _lib.misa_decode_route_heads(Qd, wd, hl_d, seq_lens, wl.B, wl.h, heads=heads_d)
+        _lib.misa_decode_score_topk(Qd, wd, heads_d, pages, bts, seq_lens, wl.k, idx=idx_d,
+                                    logits=lg_d)
+
+    t_db = _time_ms(decode_batch, stream, flush)
+    t_ds = _time_ms(lambda: _lib.misa_decode_score_topk(Qd, wd, heads_d, pages, bts, seq_lens,
+                                                         wl.k, idx=idx_d, logits=lg_d),
+                    stream, flush)
+    key_bytes = n_seq * wl.n_k * wl.d * 2
+    out["decode_batch64_ms"] = round(t_db, 4)
+    out["decode_batch64_score_topk_ms"] = round(t_ds, 4)
+    out["decode_batch64_key_gbs"] = round(key_bytes / (t_ds * 1e-3) / 1e9, 1)
+    del pages, bts, seq_lens, Qd, wd, hl_d, heads_d, idx_d, lg_d
     del ixu, lg, Q, K, w
 
     # the prefill configurations (whole-sequence prefill, the fused path per

@@ -213,6 +213,94 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
                     size_t ws_bytes, void* stream);
 
 /*
+ * Paged key caches.  The integration issue ("Clarification on the Figure 3
+ * baseline...", measurement table and the use_misa call path) measures the
+ * indexer at the vLLM boundary, where the index keys live in a paged cache and
+ * the indexer's time includes the cache handling.  These entry points take the
+ * keys in that form instead of as one contiguous [n_k, d] array:
+ *   pages        [n_pages, page_size, d] key rows (bf16 codes, or e4m3 codes
+ *                with k_scale [n_pages, page_size] fp32: a scale per row),
+ *                16-byte aligned; n_pages * page_size < 2^31
+ *   block_table  [ceil(n_k / page_size)] int32: logical key s of the sequence
+ *                is row s % page_size of page block_table[s / page_size]
+ *   page_size    16, 32, 64 or 128 (else MISA_ERR_UNSUPPORTED)
+ * Every other argument, and the result, is that of the contiguous entry point
+ * of the same name: the result equals the contiguous call on the keys gathered
+ * in logical order, bit for bit (the same arithmetic on the same values).  A
+ * block-table entry outside 0..n_pages-1 is reported as MISA_ERR_DEVICE and
+ * read as page 0.  Table entries are read only for keys below n_k.
+ */
+int misa_pool_keys_paged(const void* pages, const float* k_scale, int kdtype,
+                         const int32_t* block_table, int page_size, int64_t n_pages, int64_t n_k,
+                         int d, int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
+                         void* stream);  /* misa_pool_keys_range over a paged cache */
+int misa_score_tokens_paged(const uint16_t* Q, const float* w, const int32_t* heads,
+                            const void* pages, const float* k_scale, int kdtype,
+                            const int32_t* block_table, int page_size, int64_t n_pages, int n_q,
+                            int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
+                            int64_t ld, void* stream);
+int misa_score_topk_paged(const uint16_t* Q, const float* w, const int32_t* heads,
+                          const void* pages, const float* k_scale, int kdtype,
+                          const int32_t* block_table, int page_size, int64_t n_pages, int n_q,
+                          int64_t q_pos0, int64_t n_k, int H, int d, int h, int k, int32_t* idx,
+                          float* logits, int64_t ld, void* ws, size_t ws_bytes, void* stream);
+int misa_rerank_paged(const uint16_t* Q, const float* w, const void* pages, const float* k_scale,
+                      int kdtype, const int32_t* block_table, int page_size, int64_t n_pages,
+                      const int32_t* cand, int kp, int n_q, int64_t q_pos0, int64_t n_k, int H,
+                      int d, int k, int32_t* idx, float* full_logits, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * Decode over paged caches: n_seq sequences, each with one new query at the
+ * last of its own seq_lens[b] keys (the pages evaluate prefill only; this is
+ * stages 1-5 for the token-by-token generation that follows it, batched over
+ * sequences the way a serving engine calls the indexer).  Layouts:
+ *   Q            [n_seq, H, d] bf16: the new query of each sequence
+ *   w            [n_seq, H] fp32
+ *   pages, k_scale, page_size, n_pages: one shared page pool, as above
+ *   block_tables [n_seq, max_blocks] int32: row b is sequence b's block table
+ *   seq_lens     [n_seq] int32 (device): keys of sequence b, 0..max_blocks *
+ *                page_size (a longer length is reported as MISA_ERR_DEVICE and
+ *                clamped); query b sits at position seq_lens[b] - 1
+ *   kbar, kbar_hl per-sequence pooled keys: [n_seq, M_max, d] fp32 and
+ *                [n_seq, 2, M_max, d] bf16 hi/lo (sequence b's slice in the
+ *                layout misa_pool_keys writes for M = M_max)
+ * n_seq <= 65535 for the pooling call.
+ */
+/* Stage 1: re-pools the last n_last blocks of every sequence (blocks
+ * M_b - n_last .. M_b - 1, M_b = ceil(seq_lens[b] / B)): n_last = 1 after one
+ * key was appended, n_last = M_max for a whole cache.  M_max >=
+ * ceil(max_blocks * page_size / B).  Each block's arithmetic is that of
+ * misa_pool_keys. */
+int misa_decode_pool_keys(const void* pages, const float* k_scale, int kdtype,
+                          const int32_t* block_tables, int max_blocks, int page_size,
+                          int64_t n_pages, const int32_t* seq_lens, int n_seq, int d, int B,
+                          int64_t M_max, int64_t n_last, float* kbar, uint16_t* kbar_hl,
+                          void* stream);
+/* Stages 2-3 for each sequence's query against its own pooled keys: the router
+ * of misa_route_heads with C(b) = the complete blocks of sequence b
+ * (floor(seq_lens[b] / B), at most M_max).  heads [n_seq, h], r_out [n_seq, H]
+ * (nullable).  H a power of two <= 128. */
+int misa_decode_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
+                            int64_t M_max, const int32_t* seq_lens, int n_seq, int H, int d, int B,
+                            int h, int32_t* heads, float* r_out, void* stream);
+/* Stages 4-5 for each sequence's query over all its keys:
+ *   logits[b, s] = sum_{i<h} w[b, j_i] * ReLU(q[b, j_i] . k_{b,s}),  s < seq_lens[b]
+ * (heads [n_seq, h], NULL = all H heads with h == H), then idx[b, :] = the k
+ * keys of largest logit, ties to the lower index, ascending, -1 padded.  A
+ * scoring pass shaped for one query per sequence: 128-key tiles against the
+ * query's h head rows padded to 16, 32 or 64 MMA columns, so the keys are read
+ * once and the MMA stays small.  bf16 pages only (FP8 pages:
+ * MISA_ERR_UNSUPPORTED); h a power of two <= 64.  logits [n_seq, ld] fp32
+ * scratch (ld >= max_blocks * page_size; entries s < seq_lens[b] hold the
+ * logits afterwards). */
+int misa_decode_score_topk(const uint16_t* Q, const float* w, const int32_t* heads,
+                           const void* pages, const float* k_scale, int kdtype,
+                           const int32_t* block_tables, int max_blocks, int page_size,
+                           int64_t n_pages, const int32_t* seq_lens, int n_seq, int H, int d,
+                           int h, int k, int32_t* idx, float* logits, int64_t ld, void* stream);
+
+/*
  * Stage timing of misa_score_topk (diagnostic; not a step of the method).
  * Between misa_profile_start() and misa_profile_stop(), each launch of the fused
  * sequence is bracketed by CUDA events on the call's stream.  misa_profile_stop

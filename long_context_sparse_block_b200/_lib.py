@@ -49,6 +49,20 @@ _SIGS = {
                                    _int, _int, _vp, _vp]),
     "misa_score_topk": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _int, _int, _int,
                                _int, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "misa_pool_keys_paged": (_int, [_vp, _vp, _int, _vp, _int, _i64, _i64, _int, _int, _i64, _i64,
+                                    _vp, _vp, _vp]),
+    "misa_score_tokens_paged": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _vp, _int, _i64, _int, _i64,
+                                       _i64, _int, _int, _int, _vp, _i64, _vp]),
+    "misa_score_topk_paged": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _vp, _int, _i64, _int, _i64,
+                                     _i64, _int, _int, _int, _int, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "misa_rerank_paged": (_int, [_vp, _vp, _vp, _vp, _int, _vp, _int, _i64, _vp, _int, _int, _i64,
+                                 _i64, _int, _int, _int, _vp, _vp, _vp, _sz, _vp]),
+    "misa_decode_pool_keys": (_int, [_vp, _vp, _int, _vp, _int, _int, _i64, _vp, _int, _int, _int,
+                                     _i64, _i64, _vp, _vp, _vp]),
+    "misa_decode_route_heads": (_int, [_vp, _vp, _vp, _i64, _vp, _int, _int, _int, _int, _int, _vp,
+                                       _vp, _vp]),
+    "misa_decode_score_topk": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _vp, _int, _int, _i64, _vp,
+                                      _int, _int, _int, _int, _int, _vp, _vp, _i64, _vp]),
     "misa_profile_start": (_int, []),
     "misa_profile_stop": (_int, [_vp, _vp, _int]),
     "misa_profile_stage_name": (ctypes.c_char_p, [_int]),
@@ -112,19 +126,51 @@ def _need_rows(t, rows: int, cols: int, name: str):
 
 
 def _kdtype(K):
+    K = K.pages if isinstance(K, PagedKeys) else K
     return MISA_K_FP8E4M3 if K.dtype in (torch.uint8, torch.float8_e4m3fn) else MISA_K_BF16
+
+
+class PagedKeys:
+    """A paged key cache: `pages` [n_pages, page_size, d] (bf16 codes, or e4m3 codes
+    with `k_scale` [n_pages, page_size] fp32), `block_table` int32 with at least
+    ceil(n_k / page_size) entries (logical key s is row s % page_size of page
+    block_table[s // page_size]), and the sequence's `n_k` logical keys.  Every
+    stage call below accepts one in place of a contiguous K [n_k, d]."""
+
+    def __init__(self, pages, block_table, n_k: int, k_scale=None):
+        if pages.dim() != 3:
+            raise ValueError("pages must be [n_pages, page_size, d]")
+        self.pages, self.block_table, self.n_k, self.k_scale = pages, block_table, int(n_k), k_scale
+        self.n_pages, self.page_size, self.d = (int(x) for x in pages.shape)
+        _need(block_table, -(-self.n_k // self.page_size), "block_table")
+        _need(k_scale, self.n_pages * self.page_size, "k_scale")
+
+    @property
+    def shape(self):
+        """The logical [n_k, d] shape of the keys."""
+        return (self.n_k, self.d)
+
+    def paged_args(self):
+        """(pages, k_scale, kdtype, block_table, page_size, n_pages) of the C calls."""
+        return (_ptr(self.pages, name="pages"), _ptr(self.k_scale, (torch.float32,), "k_scale"),
+                _kdtype(self.pages), _ptr(self.block_table, (torch.int32,), "block_table"),
+                self.page_size, self.n_pages)
 
 
 # ---------------------------------------------------------------- stage calls
 
 def misa_pool_keys(K, B: int, k_scale=None, kbar=None, kbar_hl=None, want_kbar: bool = True):
-    """K [n_k, d] bf16 codes (or e4m3 codes + k_scale) -> (kbar [M,d] f32, kbar_hl [2,M,d])."""
+    """K [n_k, d] bf16 codes (or e4m3 codes + k_scale), or a PagedKeys cache
+    -> (kbar [M,d] f32, kbar_hl [2,M,d])."""
     n_k, d = K.shape
     M = -(-n_k // B)
+    dev = K.pages.device if isinstance(K, PagedKeys) else K.device
     if kbar is None and want_kbar:
-        kbar = torch.empty((M, d), dtype=torch.float32, device=K.device)
+        kbar = torch.empty((M, d), dtype=torch.float32, device=dev)
     if kbar_hl is None:
-        kbar_hl = torch.empty((2, M, d), dtype=torch.int16, device=K.device)
+        kbar_hl = torch.empty((2, M, d), dtype=torch.int16, device=dev)
+    if isinstance(K, PagedKeys):
+        return misa_pool_keys_range(K, B, 0, M, kbar=kbar, kbar_hl=kbar_hl)
     _need(k_scale, n_k, "k_scale")
     _need(kbar, M * d, "kbar")
     _need(kbar_hl, 2 * M * d, "kbar_hl")
@@ -143,10 +189,18 @@ def misa_pool_keys_range(K, B: int, m0: int, m1: int, kbar=None, kbar_hl=None, k
         n_k = K.shape[0]
     d = K.shape[1]
     M = -(-n_k // B) if B > 0 else 0
-    _need(K, n_k * d, "K")
-    _need(k_scale, n_k, "k_scale")
     _need(kbar, M * d, "kbar")
     _need(kbar_hl, 2 * M * d, "kbar_hl")
+    if isinstance(K, PagedKeys):
+        if n_k > K.n_k:
+            raise ValueError(f"n_k={n_k} exceeds the cache's {K.n_k} keys")
+        st = _lib.misa_pool_keys_paged(*K.paged_args(), n_k, d, B, m0, m1,
+                                       _ptr(kbar, (torch.float32,), "kbar"),
+                                       _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), _stream())
+        _check("misa_pool_keys_paged", st)
+        return kbar, kbar_hl
+    _need(K, n_k * d, "K")
+    _need(k_scale, n_k, "k_scale")
     st = _lib.misa_pool_keys_range(_ptr(K, name="K"), _ptr(k_scale, (torch.float32,), "k_scale"),
                                    _kdtype(K), n_k, d, B, m0, m1,
                                    _ptr(kbar, (torch.float32,), "kbar"),
@@ -185,11 +239,18 @@ def misa_score_tokens(Q, w, heads, K, q_pos0: int, k_scale=None, logits=None, h:
     ld = logits.stride(0) if logits.dim() == 2 else n_k
     _need(w, n_q * H, "w")
     _need(heads, n_q * h, "heads")
-    _need(k_scale, n_k, "k_scale")
     if logits.dim() == 2:
         _need_rows(logits, n_q, n_k, "logits")
     else:
         _need(logits, n_q * n_k, "logits")
+    if isinstance(K, PagedKeys):
+        st = _lib.misa_score_tokens_paged(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                                          _ptr(heads, (torch.int32,), "heads"), *K.paged_args(),
+                                          n_q, q_pos0, n_k, H, d, h,
+                                          ctypes.c_void_p(logits.data_ptr()), ld, _stream())
+        _check("misa_score_tokens_paged", st)
+        return logits
+    _need(k_scale, n_k, "k_scale")
     st = _lib.misa_score_tokens(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
                                 _ptr(heads, (torch.int32,), "heads"), _ptr(K, name="K"),
                                 _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K), n_q, q_pos0,
@@ -261,12 +322,21 @@ def misa_score_topk(Q, w, heads, K, q_pos0: int, k: int, k_scale=None, h: int | 
         raise ValueError("logits must be a row-major [n_q, >= n_k] fp32 buffer")
     _need(w, n_q * H, "w")
     _need(heads, n_q * h, "heads")
-    _need(k_scale, n_k, "k_scale")
     _need(idx, n_q * k, "idx")
     _need_rows(logits, n_q, n_k, "logits")
     ws_bytes = misa_workspace_size("score_topk", n_q, n_k, k, 0)
     if ws_bytes and (ws is None or ws.numel() * ws.element_size() < ws_bytes):
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    if isinstance(K, PagedKeys):
+        st = _lib.misa_score_topk_paged(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                                        _ptr(heads, (torch.int32,), "heads"), *K.paged_args(), n_q,
+                                        q_pos0, n_k, H, d, h, k, _ptr(idx, (torch.int32,), "idx"),
+                                        ctypes.c_void_p(logits.data_ptr()), logits.stride(0),
+                                        _ptr(ws, name="ws") if ws_bytes else None, ws_bytes,
+                                        _stream())
+        _check("misa_score_topk_paged", st)
+        return idx
+    _need(k_scale, n_k, "k_scale")
     st = _lib.misa_score_topk(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
                               _ptr(heads, (torch.int32,), "heads"), _ptr(K, name="K"),
                               _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K), n_q, q_pos0,
@@ -291,7 +361,6 @@ def misa_rerank(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, want_full: boo
         idx = torch.empty((n_q, k), dtype=torch.int32, device=Q.device)
     full = torch.empty((n_q, kp), dtype=torch.float32, device=Q.device) if want_full else None
     _need(w, n_q * H, "w")
-    _need(k_scale, n_k, "k_scale")
     _need(cand, n_q * kp, "cand")
     _need(idx, n_q * k, "idx")
     ws_bytes = 0
@@ -299,6 +368,16 @@ def misa_rerank(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, want_full: boo
         ws_bytes = misa_workspace_size("rerank", n_q, n_k, k, kp)
         if ws is None or ws.numel() * ws.element_size() < ws_bytes:
             ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=Q.device)
+    if isinstance(K, PagedKeys):
+        st = _lib.misa_rerank_paged(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                                    *K.paged_args(), _ptr(cand, (torch.int32,), "cand"), kp, n_q,
+                                    q_pos0, n_k, H, d, k, _ptr(idx, (torch.int32,), "idx"),
+                                    _ptr(full, (torch.float32,), "full"),
+                                    _ptr(ws, name="ws") if full is None else None, ws_bytes,
+                                    _stream())
+        _check("misa_rerank_paged", st)
+        return (idx, full) if want_full else idx
+    _need(k_scale, n_k, "k_scale")
     st = _lib.misa_rerank(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"), _ptr(K, name="K"),
                           _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K),
                           _ptr(cand, (torch.int32,), "cand"), kp, n_q, q_pos0, n_k, H, d, k,
@@ -325,6 +404,86 @@ def misa_rerank_noalloc(Q, w, K, cand, q_pos0: int, k: int, k_scale=None, idx=No
                                   K.shape[0], H, d, k, _ptr(idx, (torch.int32,), "idx"), _stream())
     _check("misa_rerank_noalloc", st)
     return idx
+
+
+# ---------------------------------------------------------------- decode (many sequences)
+
+def _decode_cache(pages, block_tables, seq_lens, k_scale):
+    if pages.dim() != 3 or block_tables.dim() != 2:
+        raise ValueError("pages [n_pages, page_size, d] and block_tables [n_seq, max_blocks]")
+    n_pages, ps, d = (int(x) for x in pages.shape)
+    n_seq, max_blocks = (int(x) for x in block_tables.shape)
+    _need(seq_lens, n_seq, "seq_lens")
+    _need(k_scale, n_pages * ps, "k_scale")
+    args = (_ptr(pages, name="pages"), _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(pages),
+            _ptr(block_tables, (torch.int32,), "block_tables"), max_blocks, ps, n_pages)
+    return args, n_seq, d, max_blocks * ps
+
+
+def misa_decode_pool_keys(pages, block_tables, seq_lens, B: int, M_max: int, n_last: int,
+                          kbar=None, kbar_hl=None, k_scale=None, want_kbar: bool = False):
+    """Re-pool the last n_last blocks of every sequence into per-sequence pooled
+    keys kbar [n_seq, M_max, d] f32 (optional) and kbar_hl [n_seq, 2, M_max, d]."""
+    args, n_seq, d, _ = _decode_cache(pages, block_tables, seq_lens, k_scale)
+    if kbar is None and want_kbar:
+        kbar = torch.empty((n_seq, M_max, d), dtype=torch.float32, device=pages.device)
+    if kbar_hl is None:
+        kbar_hl = torch.empty((n_seq, 2, M_max, d), dtype=torch.int16, device=pages.device)
+    _need(kbar, n_seq * M_max * d, "kbar")
+    _need(kbar_hl, n_seq * 2 * M_max * d, "kbar_hl")
+    st = _lib.misa_decode_pool_keys(*args, _ptr(seq_lens, (torch.int32,), "seq_lens"), n_seq, d, B,
+                                    M_max, n_last, _ptr(kbar, (torch.float32,), "kbar"),
+                                    _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), _stream())
+    _check("misa_decode_pool_keys", st)
+    return kbar, kbar_hl
+
+
+def misa_decode_route_heads(Q, w, kbar_hl, seq_lens, B: int, h: int, heads=None,
+                            want_r: bool = False):
+    """Q [n_seq, H, d], w [n_seq, H], kbar_hl [n_seq, 2, M_max, d] -> (heads [n_seq, h], r)."""
+    n_seq, H, d = Q.shape
+    M_max = int(kbar_hl.shape[-2])
+    if heads is None:
+        heads = torch.empty((n_seq, h), dtype=torch.int32, device=Q.device)
+    r = torch.empty((n_seq, H), dtype=torch.float32, device=Q.device) if want_r else None
+    _need(w, n_seq * H, "w")
+    _need(kbar_hl, n_seq * 2 * M_max * d, "kbar_hl")
+    _need(seq_lens, n_seq, "seq_lens")
+    _need(heads, n_seq * h, "heads")
+    st = _lib.misa_decode_route_heads(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                                      _ptr(kbar_hl, _BF16_CODES, "kbar_hl"), M_max,
+                                      _ptr(seq_lens, (torch.int32,), "seq_lens"), n_seq, H, d, B, h,
+                                      _ptr(heads, (torch.int32,), "heads"),
+                                      _ptr(r, (torch.float32,), "r"), _stream())
+    _check("misa_decode_route_heads", st)
+    return heads, r
+
+
+def misa_decode_score_topk(Q, w, heads, pages, block_tables, seq_lens, k: int, k_scale=None,
+                           h: int | None = None, idx=None, logits=None):
+    """Per sequence b: the top-k keys (ascending, -1 padded) of its new query's
+    routed logits over its seq_lens[b] keys -> (idx [n_seq, k], logits [n_seq, ld])."""
+    n_seq, H, d = Q.shape
+    args, n_seq2, d2, max_len = _decode_cache(pages, block_tables, seq_lens, k_scale)
+    if n_seq2 != n_seq or d2 != d:
+        raise ValueError("block_tables / pages do not match Q")
+    if h is None:
+        h = heads.shape[1] if heads is not None else H
+    if idx is None:
+        idx = torch.empty((n_seq, k), dtype=torch.int32, device=Q.device)
+    if logits is None:
+        logits = torch.empty((n_seq, max_len), dtype=torch.float32, device=Q.device)
+    _need(w, n_seq * H, "w")
+    _need(heads, n_seq * h, "heads")
+    _need(idx, n_seq * k, "idx")
+    _need_rows(logits, n_seq, max_len, "logits")
+    st = _lib.misa_decode_score_topk(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
+                                     _ptr(heads, (torch.int32,), "heads"), *args,
+                                     _ptr(seq_lens, (torch.int32,), "seq_lens"), n_seq, H, d, h, k,
+                                     _ptr(idx, (torch.int32,), "idx"),
+                                     ctypes.c_void_p(logits.data_ptr()), logits.stride(0), _stream())
+    _check("misa_decode_score_topk", st)
+    return idx, logits
 
 
 def misa_profile_start() -> None:

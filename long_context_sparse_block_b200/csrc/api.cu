@@ -70,6 +70,45 @@ constexpr int kFusedMaxK = 8192;                    // the finish kernel's list 
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
+// The key cache of an entry point: contiguous ([n_k, d] rows) or paged (pages
+// of page_size rows in a pool of n_pages pages, logical block b of the
+// sequence in page block_table[b]); FP8 scales follow the physical rows.
+struct KeyArg {
+  const void* K;
+  const float* k_scale;
+  int kdtype;
+  KeyPages kpg;
+  bool fp8() const { return kdtype == MISA_K_FP8E4M3; }
+};
+
+KeyArg contiguous_keys(const void* K, const float* k_scale, int kdtype) {
+  return KeyArg{K, k_scale, kdtype, KeyPages{nullptr, 0, 0}};
+}
+
+// page_size must be 16, 32, 64 or 128 (a 128-key tile holds whole pages); an
+// unsupported size leaves page_shift at -1 for check_keys to refuse.
+KeyArg paged_keys(const void* pages, const float* k_scale, int kdtype, const int32_t* block_table,
+                  int page_size, int64_t n_pages) {
+  int shift = -1;
+  for (int sh = 4; sh <= 7; ++sh)
+    if (page_size == (1 << sh)) shift = sh;
+  return KeyArg{pages, k_scale, kdtype, KeyPages{block_table, shift, n_pages}};
+}
+
+int check_keys(const KeyArg& k, int64_t n_k) {
+  if (!k.K || !aligned16(k.K)) return MISA_ERR_INVALID_ARG;
+  if (k.kdtype != MISA_K_BF16 && k.kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
+  if (k.fp8() && (!k.k_scale || !aligned4(k.k_scale))) return MISA_ERR_INVALID_ARG;
+  if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
+  if (k.kpg.bt) {
+    if (!aligned4(k.kpg.bt)) return MISA_ERR_INVALID_ARG;
+    if (k.kpg.page_shift < 0) return MISA_ERR_UNSUPPORTED;
+    if (k.kpg.n_pages < 1 || (k.kpg.n_pages << k.kpg.page_shift) > 0x7fffffffLL)
+      return MISA_ERR_INVALID_ARG;
+  }
+  return MISA_OK;
+}
+
 // Optional per-stage timing of misa_score_topk: while enabled, every launch of
 // the fused sequence is bracketed by a pair of CUDA events on its stream.
 constexpr int kStages = 7;
@@ -107,7 +146,7 @@ struct StageMark {
 int64_t mask_words(int64_t n_k) { return ((n_k + 31) / 32 + 3) / 4 * 4; }
 
 struct FusedLayout {
-  size_t gate, tau, ks, ks_scale, sample, mask, kbf, total;
+  size_t gate, tau, ks, ks_scale, sample, mask, kbf, kbf_scale, total;
   FusedLayout(int n_q, int64_t n_k) {
     const size_t nq = static_cast<size_t>(n_q);
     size_t o = 0;
@@ -123,8 +162,10 @@ struct FusedLayout {
     o += round256(nq * kSampleKeys * 4);
     mask = o;
     o += round256(nq * static_cast<size_t>(mask_words(n_k)) * 4);
-    kbf = o;  // FP8 keys decoded to bf16 (d <= 128)
+    kbf = o;  // FP8 keys decoded to bf16 (d <= 128), in logical order
     o += round256(static_cast<size_t>(n_k) * 256);
+    kbf_scale = o;  // their scales, in logical order (paged caches)
+    o += round256(static_cast<size_t>(n_k) * 4);
     total = o;
   }
 };
@@ -175,22 +216,222 @@ CUresult encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank
 
 using namespace misa;
 
-extern "C" {
+namespace {
 
-int misa_pool_keys_range(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d,
-                         int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
-                         void* stream) {
-  if (!K || !aligned16(K) || n_k < 1 || !good_d(d) || B < 1 || B > 4096) return MISA_ERR_INVALID_ARG;
-  if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
-  if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
+int pool_impl(const KeyArg& key, int64_t n_k, int d, int B, int64_t m0, int64_t m1, float* kbar,
+              uint16_t* kbar_hl, void* stream) {
+  if (n_k < 1 || !good_d(d) || B < 1 || B > 4096) return MISA_ERR_INVALID_ARG;
+  if (const int st = check_keys(key, n_k)) return st;
   if (!kbar && !kbar_hl) return MISA_ERR_INVALID_ARG;
   if ((kbar && !aligned4(kbar)) || (kbar_hl && (reinterpret_cast<uintptr_t>(kbar_hl) & 1u)))
     return MISA_ERR_INVALID_ARG;
   const int64_t M = (n_k + B - 1) / B;
   if (M > 0x7fffffff || m0 < 0 || m1 < m0 || m1 > M) return MISA_ERR_INVALID_ARG;
   if (m0 == m1) return MISA_OK;
-  return cuda_status(launch_pool_keys(K, k_scale, kdtype == MISA_K_FP8E4M3, n_k, d, B, m0, m1,
-                                      kbar, kbar_hl, as_stream(stream)));
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  return cuda_status(launch_pool_keys(key.K, key.k_scale, key.kpg, key.fp8(), n_k, d, B, m0, m1,
+                                      kbar, kbar_hl, ctl, as_stream(stream)));
+}
+
+}  // namespace
+
+namespace {
+
+int score_impl(const uint16_t* Q, const float* w, const int32_t* heads, const KeyArg& key, int n_q,
+               int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits, int64_t ld,
+               void* stream) {
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !logits || !aligned16(logits))
+    return MISA_ERR_INVALID_ARG;
+  if (heads && !aligned4(heads)) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || H < 1 || h < 1 || h > H ||
+      ld < n_k || ld % 4 != 0)
+    return MISA_ERR_INVALID_ARG;
+  if (!heads && h != H) return MISA_ERR_INVALID_ARG;
+  if (const int st = check_keys(key, n_k)) return st;
+  if (!good_d(d) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
+  if (n_q == 0) return MISA_OK;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  ScoreLaunch a{};
+  a.Q = Q;
+  a.w = w;
+  a.heads = heads;
+  a.K = key.K;
+  a.k_scale = key.k_scale;
+  a.fp8 = key.fp8();
+  a.kpg = key.kpg;
+  a.n_q = n_q;
+  a.q_pos0 = q_pos0;
+  a.n_k = n_k;
+  a.H = H;
+  a.d = d;
+  a.h = h;
+  a.logits = logits;
+  a.ld = ld;
+  return cuda_status(launch_score(a, ctl, as_stream(stream)));
+}
+
+}  // namespace
+
+namespace {
+
+int rerank_impl(const uint16_t* Q, const float* w, const KeyArg& key, const int32_t* cand, int kp,
+                int n_q, int64_t q_pos0, int64_t n_k, int H, int d, int k, int32_t* idx,
+                float* full_logits, void* ws, size_t ws_bytes, void* stream) {
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !cand || !aligned4(cand) ||
+      (k > 0 && (!idx || !aligned4(idx))))
+    return MISA_ERR_INVALID_ARG;
+  if (full_logits && !aligned4(full_logits)) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || kp < 1 || kp > 16384 || k < 0 ||
+      k > kp || H < 1)
+    return MISA_ERR_INVALID_ARG;
+  if (const int st = check_keys(key, n_k)) return st;
+  if (!good_d(d) || H > 128) return MISA_ERR_UNSUPPORTED;
+  if (n_q == 0) return MISA_OK;
+  float* full = full_logits;
+  if (!full) {
+    const size_t need = misa_workspace_size("rerank", n_q, n_k, k, kp);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return MISA_ERR_WORKSPACE;
+    full = static_cast<float*>(ws);
+  }
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  const cudaStream_t s = as_stream(stream);
+  cudaError_t e = launch_rerank_scores(Q, w, key.K, key.k_scale, key.kpg, key.fp8(), cand, kp, n_q,
+                                       q_pos0, n_k, H, d, full, kp, ctl, s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  if (k == 0) return MISA_OK;
+  return cuda_status(launch_select_candidates(full, kp, cand, kp, n_q, q_pos0, n_k, k, idx, ctl, s));
+}
+
+}  // namespace
+
+namespace {
+
+int score_topk_impl(const uint16_t* Q, const float* w, const int32_t* heads, const KeyArg& key,
+                    int n_q, int64_t q_pos0, int64_t n_k, int H, int d, int h, int k, int32_t* idx,
+                    float* logits, int64_t ld, void* ws, size_t ws_bytes, void* stream) {
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !logits || !aligned16(logits) ||
+      (k > 0 && (!idx || !aligned4(idx))))
+    return MISA_ERR_INVALID_ARG;
+  if (heads && !aligned4(heads)) return MISA_ERR_INVALID_ARG;
+  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || H < 1 || h < 1 || h > H ||
+      ld < n_k || ld % 4 != 0 || k < 0 || k > 16384)
+    return MISA_ERR_INVALID_ARG;
+  if (!heads && h != H) return MISA_ERR_INVALID_ARG;
+  if (const int st = check_keys(key, n_k)) return st;
+  if (!good_d(d) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
+  if (n_q == 0 || k == 0) return MISA_OK;
+  const size_t need = misa_workspace_size("score_topk", n_q, n_k, k, 0);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return MISA_ERR_WORKSPACE;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  const cudaStream_t s = as_stream(stream);
+  const bool fp8 = key.fp8();
+  ScoreLaunch a{};
+  a.Q = Q;
+  a.w = w;
+  a.heads = heads;
+  a.K = key.K;
+  a.k_scale = key.k_scale;
+  a.fp8 = fp8;
+  a.kpg = key.kpg;
+  a.n_q = n_q;
+  a.q_pos0 = q_pos0;
+  a.n_k = n_k;
+  a.H = H;
+  a.d = d;
+  a.h = h;
+  a.logits = logits;
+  a.ld = ld;
+  const bool fused = need > 0 && q_pos0 + 1 >= kSampleKeys && score_select_supported(h);
+  if (!fused) {  // unfused: every logit, then the selection
+    cudaError_t e = launch_score(a, ctl, s);
+    if (e != cudaSuccess) return MISA_ERR_CUDA;
+    return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, k, idx, ctl, s));
+  }
+  const FusedLayout L(n_q, n_k);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* gate = reinterpret_cast<int*>(base + L.gate);
+  float* tau = reinterpret_cast<float*>(base + L.tau);
+  void* Ks = base + L.ks;
+  float* ks_scale = reinterpret_cast<float*>(base + L.ks_scale);
+  float* sample = reinterpret_cast<float*>(base + L.sample);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(base + L.mask);
+  const int64_t mld = mask_words(n_k);
+  cudaError_t e;
+  {
+    StageMark m(0, s);
+    if (fp8) {
+      // decode the keys once, in logical order (with their scales when paged);
+      // every scoring pass then reads contiguous bf16 codes
+      uint16_t* kbf = reinterpret_cast<uint16_t*>(base + L.kbf);
+      float* kbf_scale = key.kpg.paged() ? reinterpret_cast<float*>(base + L.kbf_scale) : nullptr;
+      e = launch_e4m3_rows_to_bf16(static_cast<const uint8_t*>(key.K), key.k_scale, key.kpg, n_k, d,
+                                   kbf, kbf_scale, ctl, s);
+      if (e != cudaSuccess) return MISA_ERR_CUDA;
+      a.K = kbf;
+      a.k_bf16 = true;
+      if (kbf_scale) a.k_scale = kbf_scale;
+      a.kpg = KeyPages{nullptr, 0, 0};
+    }
+    e = launch_gather_sample(a.K, fp8 ? a.k_scale : nullptr, a.kpg, 2 * d, q_pos0 + 1,
+                             kSampleBlocks, Ks, fp8 ? ks_scale : nullptr, ctl, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  ScoreLaunch sa = a;  // the sample: every sampled key is visible to every query
+  sa.K = Ks;
+  sa.k_scale = fp8 ? ks_scale : nullptr;
+  sa.kpg = KeyPages{nullptr, 0, 0};
+  sa.q_pos0 = kSampleKeys - 1;
+  sa.n_k = kSampleKeys;
+  sa.logits = sample;
+  sa.ld = kSampleKeys;
+  {
+    StageMark m(1, s);
+    e = launch_score(sa, ctl, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  {
+    StageMark m(2, s);
+    e = launch_fused_tau(sample, kSampleKeys, kSampleKeys, n_q, q_pos0, n_k, k, tau, gate, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  ScoreLaunch se = a;  // select mode
+  se.tau = tau;
+  se.mask = mask;
+  se.mask_ld = mld;
+  {
+    StageMark m(3, s);
+    e = launch_score(se, ctl, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  {
+    StageMark m(4, s);
+    e = launch_fused_finish(logits, ld, mask, mld, n_q, q_pos0, n_k, k, idx, gate, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  // exact fallback for the rows the thresholds missed (a no-op launch when none)
+  ScoreLaunch ra = a;
+  ra.gate = gate;
+  {
+    StageMark m(5, s);
+    e = launch_score(ra, ctl, s);
+  }
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  StageMark m(6, s);
+  return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, k, idx, ctl, s, gate));
+}
+
+}  // namespace
+
+extern "C" {
+
+int misa_pool_keys_range(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d,
+                         int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
+                         void* stream) {
+  return pool_impl(contiguous_keys(K, k_scale, kdtype), n_k, d, B, m0, m1, kbar, kbar_hl, stream);
 }
 
 int misa_pool_keys(const void* K, const float* k_scale, int kdtype, int64_t n_k, int d, int B,
@@ -198,6 +439,15 @@ int misa_pool_keys(const void* K, const float* k_scale, int kdtype, int64_t n_k,
   if (B < 1) return MISA_ERR_INVALID_ARG;
   return misa_pool_keys_range(K, k_scale, kdtype, n_k, d, B, 0, (n_k + B - 1) / B, kbar, kbar_hl,
                               stream);
+}
+
+int misa_pool_keys_paged(const void* pages, const float* k_scale, int kdtype,
+                         const int32_t* block_table, int page_size, int64_t n_pages, int64_t n_k,
+                         int d, int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
+                         void* stream) {
+  if (!block_table) return MISA_ERR_INVALID_ARG;
+  return pool_impl(paged_keys(pages, k_scale, kdtype, block_table, page_size, n_pages), n_k, d, B,
+                   m0, m1, kbar, kbar_hl, stream);
 }
 
 int misa_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl, int n_q,
@@ -221,23 +471,18 @@ int misa_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
 int misa_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
                       const float* k_scale, int kdtype, int n_q, int64_t q_pos0, int64_t n_k, int H,
                       int d, int h, float* logits, int64_t ld, void* stream) {
-  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !K || !aligned16(K) || !logits ||
-      !aligned4(logits))
-    return MISA_ERR_INVALID_ARG;
-  if (heads && !aligned4(heads)) return MISA_ERR_INVALID_ARG;
-  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || H < 1 || h < 1 || h > H ||
-      ld < n_k || ld % 4 != 0 || !aligned16(logits))
-    return MISA_ERR_INVALID_ARG;
-  if (!heads && h != H) return MISA_ERR_INVALID_ARG;
-  if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
-  if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
-  if (!good_d(d) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
-  if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
-  if (n_q == 0) return MISA_OK;
-  DevCtl ctl;
-  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
-  return cuda_status(launch_score_tokens(Q, w, heads, K, k_scale, kdtype == MISA_K_FP8E4M3, n_q,
-                                         q_pos0, n_k, H, d, h, logits, ld, ctl, as_stream(stream)));
+  return score_impl(Q, w, heads, contiguous_keys(K, k_scale, kdtype), n_q, q_pos0, n_k, H, d, h,
+                    logits, ld, stream);
+}
+
+int misa_score_tokens_paged(const uint16_t* Q, const float* w, const int32_t* heads,
+                            const void* pages, const float* k_scale, int kdtype,
+                            const int32_t* block_table, int page_size, int64_t n_pages, int n_q,
+                            int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
+                            int64_t ld, void* stream) {
+  if (!block_table) return MISA_ERR_INVALID_ARG;
+  return score_impl(Q, w, heads, paged_keys(pages, k_scale, kdtype, block_table, page_size, n_pages),
+                    n_q, q_pos0, n_k, H, d, h, logits, ld, stream);
 }
 
 int misa_score_tokens_fp8(const uint8_t* Q8, const float* q_scale, const float* w,
@@ -296,141 +541,108 @@ int misa_topk(const float* logits, int64_t ld, int n_q, int64_t q_pos0, int64_t 
 int misa_rerank(const uint16_t* Q, const float* w, const void* K, const float* k_scale, int kdtype,
                 const int32_t* cand, int kp, int n_q, int64_t q_pos0, int64_t n_k, int H, int d,
                 int k, int32_t* idx, float* full_logits, void* ws, size_t ws_bytes, void* stream) {
-  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !K || !aligned16(K) || !cand ||
-      !aligned4(cand) || (k > 0 && (!idx || !aligned4(idx))))
-    return MISA_ERR_INVALID_ARG;
-  if (full_logits && !aligned4(full_logits)) return MISA_ERR_INVALID_ARG;
-  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || kp < 1 || kp > 16384 || k < 0 ||
-      k > kp || H < 1)
-    return MISA_ERR_INVALID_ARG;
-  if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
-  if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
-  if (!good_d(d) || H > 128) return MISA_ERR_UNSUPPORTED;
-  if (n_q == 0) return MISA_OK;
-  float* full = full_logits;
-  if (!full) {
-    const size_t need = misa_workspace_size("rerank", n_q, n_k, k, kp);
-    if (!ws || ws_bytes < need || !aligned16(ws)) return MISA_ERR_WORKSPACE;
-    full = static_cast<float*>(ws);
-  }
-  DevCtl ctl;
-  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
-  const cudaStream_t s = as_stream(stream);
-  cudaError_t e = launch_rerank_scores(Q, w, K, k_scale, kdtype == MISA_K_FP8E4M3, cand, kp, n_q,
-                                       q_pos0, n_k, H, d, full, kp, ctl, s);
-  if (e != cudaSuccess) return MISA_ERR_CUDA;
-  if (k == 0) return MISA_OK;
-  return cuda_status(launch_select_candidates(full, kp, cand, kp, n_q, q_pos0, n_k, k, idx, ctl, s));
+  return rerank_impl(Q, w, contiguous_keys(K, k_scale, kdtype), cand, kp, n_q, q_pos0, n_k, H, d, k,
+                     idx, full_logits, ws, ws_bytes, stream);
+}
+
+int misa_rerank_paged(const uint16_t* Q, const float* w, const void* pages, const float* k_scale,
+                      int kdtype, const int32_t* block_table, int page_size, int64_t n_pages,
+                      const int32_t* cand, int kp, int n_q, int64_t q_pos0, int64_t n_k, int H,
+                      int d, int k, int32_t* idx, float* full_logits, void* ws, size_t ws_bytes,
+                      void* stream) {
+  if (!block_table) return MISA_ERR_INVALID_ARG;
+  return rerank_impl(Q, w, paged_keys(pages, k_scale, kdtype, block_table, page_size, n_pages), cand,
+                     kp, n_q, q_pos0, n_k, H, d, k, idx, full_logits, ws, ws_bytes, stream);
 }
 
 int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
                     const float* k_scale, int kdtype, int n_q, int64_t q_pos0, int64_t n_k, int H,
                     int d, int h, int k, int32_t* idx, float* logits, int64_t ld, void* ws,
                     size_t ws_bytes, void* stream) {
-  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !K || !aligned16(K) || !logits ||
-      !aligned16(logits) || (k > 0 && (!idx || !aligned4(idx))))
+  return score_topk_impl(Q, w, heads, contiguous_keys(K, k_scale, kdtype), n_q, q_pos0, n_k, H, d,
+                         h, k, idx, logits, ld, ws, ws_bytes, stream);
+}
+
+int misa_score_topk_paged(const uint16_t* Q, const float* w, const int32_t* heads,
+                          const void* pages, const float* k_scale, int kdtype,
+                          const int32_t* block_table, int page_size, int64_t n_pages, int n_q,
+                          int64_t q_pos0, int64_t n_k, int H, int d, int h, int k, int32_t* idx,
+                          float* logits, int64_t ld, void* ws, size_t ws_bytes, void* stream) {
+  if (!block_table) return MISA_ERR_INVALID_ARG;
+  return score_topk_impl(Q, w, heads,
+                         paged_keys(pages, k_scale, kdtype, block_table, page_size, n_pages), n_q,
+                         q_pos0, n_k, H, d, h, k, idx, logits, ld, ws, ws_bytes, stream);
+}
+
+int misa_decode_pool_keys(const void* pages, const float* k_scale, int kdtype,
+                          const int32_t* block_tables, int max_blocks, int page_size,
+                          int64_t n_pages, const int32_t* seq_lens, int n_seq, int d, int B,
+                          int64_t M_max, int64_t n_last, float* kbar, uint16_t* kbar_hl,
+                          void* stream) {
+  const KeyArg key = paged_keys(pages, k_scale, kdtype, block_tables, page_size, n_pages);
+  if (!block_tables || !seq_lens || !aligned4(seq_lens) || n_seq < 0 || n_seq > 65535 ||
+      max_blocks < 1 || !good_d(d) || B < 1 || B > 4096 || n_last < 0 || n_last > 0x7fffffffLL)
+    return MISA_ERR_INVALID_ARG;
+  const int64_t max_len = static_cast<int64_t>(max_blocks) * page_size;
+  if (const int st = check_keys(key, max_len)) return st;
+  if (M_max < (max_len + B - 1) / B || M_max > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
+  if (!kbar && !kbar_hl) return MISA_ERR_INVALID_ARG;
+  if ((kbar && !aligned4(kbar)) || (kbar_hl && (reinterpret_cast<uintptr_t>(kbar_hl) & 1u)))
+    return MISA_ERR_INVALID_ARG;
+  if (n_seq == 0 || n_last == 0) return MISA_OK;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  return cuda_status(launch_pool_keys_batch(pages, k_scale, key.fp8(), block_tables, max_blocks,
+                                            key.kpg.page_shift, n_pages, seq_lens, n_seq, d, B,
+                                            M_max, std::min<int64_t>(n_last, M_max), kbar, kbar_hl,
+                                            ctl, as_stream(stream)));
+}
+
+int misa_decode_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
+                            int64_t M_max, const int32_t* seq_lens, int n_seq, int H, int d, int B,
+                            int h, int32_t* heads, float* r_out, void* stream) {
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !kbar_hl || !aligned16(kbar_hl) || !heads ||
+      !aligned4(heads) || !seq_lens || !aligned4(seq_lens))
+    return MISA_ERR_INVALID_ARG;
+  if (r_out && !aligned4(r_out)) return MISA_ERR_INVALID_ARG;
+  if (n_seq < 0 || M_max < 1 || M_max > 0x7fffffffLL || B < 1 || h < 1 || h > H)
+    return MISA_ERR_INVALID_ARG;
+  if (!good_d(d) || !pow2(H) || H > 128) return MISA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(n_seq) * H > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
+  if (n_seq == 0) return MISA_OK;
+  DevCtl ctl;
+  if (!make_ctl(ctl)) return MISA_ERR_CUDA;
+  return cuda_status(launch_route_heads_decode(Q, w, kbar_hl, M_max, seq_lens, n_seq, H, d, B, h,
+                                               heads, r_out, ctl, as_stream(stream)));
+}
+
+int misa_decode_score_topk(const uint16_t* Q, const float* w, const int32_t* heads,
+                           const void* pages, const float* k_scale, int kdtype,
+                           const int32_t* block_tables, int max_blocks, int page_size,
+                           int64_t n_pages, const int32_t* seq_lens, int n_seq, int H, int d,
+                           int h, int k, int32_t* idx, float* logits, int64_t ld, void* stream) {
+  const KeyArg key = paged_keys(pages, k_scale, kdtype, block_tables, page_size, n_pages);
+  if (!Q || !aligned16(Q) || !w || !aligned4(w) || !block_tables || !seq_lens ||
+      !aligned4(seq_lens) || !logits || !aligned4(logits) || (k > 0 && (!idx || !aligned4(idx))))
     return MISA_ERR_INVALID_ARG;
   if (heads && !aligned4(heads)) return MISA_ERR_INVALID_ARG;
-  if (n_q < 0 || q_pos0 < 0 || n_k < 1 || q_pos0 + n_q > n_k || H < 1 || h < 1 || h > H ||
-      ld < n_k || ld % 4 != 0 || k < 0 || k > 16384)
+  if (n_seq < 0 || max_blocks < 1 || H < 1 || h < 1 || h > H || k < 0 || k > 16384)
     return MISA_ERR_INVALID_ARG;
   if (!heads && h != H) return MISA_ERR_INVALID_ARG;
-  if (kdtype != MISA_K_BF16 && kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
-  if (kdtype == MISA_K_FP8E4M3 && (!k_scale || !aligned4(k_scale))) return MISA_ERR_INVALID_ARG;
-  if (!good_d(d) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
-  if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
-  if (n_q == 0 || k == 0) return MISA_OK;
-  const size_t need = misa_workspace_size("score_topk", n_q, n_k, k, 0);
-  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return MISA_ERR_WORKSPACE;
+  const int64_t max_len = static_cast<int64_t>(max_blocks) * page_size;
+  if (const int st = check_keys(key, max_len)) return st;
+  if (ld < max_len) return MISA_ERR_INVALID_ARG;
+  if (key.fp8() || !good_d(d) || !pow2(h) || h > 64) return MISA_ERR_UNSUPPORTED;
+  if (n_seq == 0) return MISA_OK;
   DevCtl ctl;
   if (!make_ctl(ctl)) return MISA_ERR_CUDA;
   const cudaStream_t s = as_stream(stream);
-  const bool fp8 = kdtype == MISA_K_FP8E4M3;
-  ScoreLaunch a{};
-  a.Q = Q;
-  a.w = w;
-  a.heads = heads;
-  a.K = K;
-  a.k_scale = k_scale;
-  a.fp8 = fp8;
-  a.n_q = n_q;
-  a.q_pos0 = q_pos0;
-  a.n_k = n_k;
-  a.H = H;
-  a.d = d;
-  a.h = h;
-  a.logits = logits;
-  a.ld = ld;
-  const bool fused = need > 0 && q_pos0 + 1 >= kSampleKeys && score_select_supported(h);
-  if (!fused) {  // unfused: every logit, then the selection
-    cudaError_t e = launch_score(a, ctl, s);
-    if (e != cudaSuccess) return MISA_ERR_CUDA;
-    return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, k, idx, ctl, s));
-  }
-  const FusedLayout L(n_q, n_k);
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  int* gate = reinterpret_cast<int*>(base + L.gate);
-  float* tau = reinterpret_cast<float*>(base + L.tau);
-  void* Ks = base + L.ks;
-  float* ks_scale = reinterpret_cast<float*>(base + L.ks_scale);
-  float* sample = reinterpret_cast<float*>(base + L.sample);
-  uint32_t* mask = reinterpret_cast<uint32_t*>(base + L.mask);
-  const int64_t mld = mask_words(n_k);
-  cudaError_t e;
-  {
-    StageMark m(0, s);
-    if (fp8) {  // decode the keys once; every scoring pass then reads bf16 codes
-      uint16_t* kbf = reinterpret_cast<uint16_t*>(base + L.kbf);
-      e = launch_e4m3_to_bf16(static_cast<const uint8_t*>(K), kbf, n_k * d, s);
-      if (e != cudaSuccess) return MISA_ERR_CUDA;
-      a.K = kbf;
-      a.k_bf16 = true;
-    }
-    e = launch_gather_sample(a.K, fp8 ? k_scale : nullptr, 2 * d, q_pos0 + 1, kSampleBlocks, Ks,
-                             fp8 ? ks_scale : nullptr, s);
-  }
+  cudaError_t e = launch_decode_score(Q, w, heads, pages, block_tables, max_blocks,
+                                      key.kpg.page_shift, n_pages, seq_lens, n_seq, H, d, h, logits,
+                                      ld, ctl, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
-  ScoreLaunch sa = a;  // the sample: every sampled key is visible to every query
-  sa.K = Ks;
-  sa.k_scale = fp8 ? ks_scale : nullptr;
-  sa.q_pos0 = kSampleKeys - 1;
-  sa.n_k = kSampleKeys;
-  sa.logits = sample;
-  sa.ld = kSampleKeys;
-  {
-    StageMark m(1, s);
-    e = launch_score(sa, ctl, s);
-  }
-  if (e != cudaSuccess) return MISA_ERR_CUDA;
-  {
-    StageMark m(2, s);
-    e = launch_fused_tau(sample, kSampleKeys, kSampleKeys, n_q, q_pos0, n_k, k, tau, gate, s);
-  }
-  if (e != cudaSuccess) return MISA_ERR_CUDA;
-  ScoreLaunch se = a;  // select mode
-  se.tau = tau;
-  se.mask = mask;
-  se.mask_ld = mld;
-  {
-    StageMark m(3, s);
-    e = launch_score(se, ctl, s);
-  }
-  if (e != cudaSuccess) return MISA_ERR_CUDA;
-  {
-    StageMark m(4, s);
-    e = launch_fused_finish(logits, ld, mask, mld, n_q, q_pos0, n_k, k, idx, gate, s);
-  }
-  if (e != cudaSuccess) return MISA_ERR_CUDA;
-  // exact fallback for the rows the thresholds missed (a no-op launch when none)
-  ScoreLaunch ra = a;
-  ra.gate = gate;
-  {
-    StageMark m(5, s);
-    e = launch_score(ra, ctl, s);
-  }
-  if (e != cudaSuccess) return MISA_ERR_CUDA;
-  StageMark m(6, s);
-  return cuda_status(launch_topk(logits, ld, n_q, q_pos0, n_k, k, idx, ctl, s, gate));
+  if (k == 0) return MISA_OK;
+  return cuda_status(launch_topk(logits, ld, n_seq, 0, max_len, k, idx, ctl, s, nullptr, seq_lens));
 }
 
 int misa_profile_start(void) {

@@ -24,6 +24,29 @@ __device__ __forceinline__ void report(const DevCtl& ctl, int code) {
   atomicCAS(ctl.status, 0, code);
 }
 
+// ---- key cache addressing ------------------------------------------------------
+// Logical key row s lives at row s of a contiguous cache, or, in a paged cache
+// (pages of 2^page_shift rows in a pool of n_pages pages), at row s & (P - 1)
+// of page bt[s >> page_shift].  Per-token scales of FP8 keys follow the same
+// physical row layout.
+struct KeyPages {
+  const int32_t* bt;   // block table (nullptr: contiguous)
+  int page_shift;
+  int64_t n_pages;
+  __host__ __device__ bool paged() const { return bt != nullptr; }
+  // Physical row of logical row s (s inside the table).  A page id outside the
+  // pool is reported and replaced by page 0, so no access leaves the pool.
+  __device__ __forceinline__ int64_t row(int64_t s, const DevCtl& ctl) const {
+    if (!bt) return s;
+    int64_t pg = __ldg(bt + (s >> page_shift));
+    if (pg < 0 || pg >= n_pages) {
+      report(ctl, DEV_BAD_INPUT);
+      pg = 0;
+    }
+    return (pg << page_shift) | (s & ((int64_t(1) << page_shift) - 1));
+  }
+};
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -32,6 +55,30 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// The first 1024-byte-aligned byte at or after p (a dynamic shared-memory
+// base).  Pointer arithmetic on the shared array itself, not an integer round
+// trip, so the compiler still knows the result points into shared memory and
+// emits shared-space loads and stores (32-bit addresses) rather than generic
+// ones.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
+  return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
+}
+
+// Shared-space loads from 32-bit shared addresses.
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }

@@ -15,11 +15,23 @@ namespace {
 
 constexpr int kPoolThreads = 256;
 
+// Many sequences at once (decode): sequence blockIdx.y has lens[y] keys through
+// block table bts[y]; its pooled keys are kbar[y] ([M_max, d]) and kbar_hl[y]
+// ([2, M_max, d]); the CTA pools block M_y - n_last + blockIdx.x of it, where
+// M_y = ceil(lens[y] / B) (nothing when that block does not exist).
+struct PoolBatch {
+  const int32_t* bts;    // nullptr: one sequence (the kernel's own arguments)
+  int max_blocks;
+  const int32_t* lens;
+  int64_t M_max;
+  int64_t n_last;
+};
+
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kPoolThreads)
-pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scale, int64_t n_k,
-                 int B, int64_t M, int64_t m0, float* __restrict__ kbar,
-                 uint16_t* __restrict__ kbar_hl) {
+pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scale, KeyPages kpg,
+                 int64_t n_k, int B, int64_t M, int64_t m0, float* __restrict__ kbar,
+                 uint16_t* __restrict__ kbar_hl, DevCtl ctl, PoolBatch batch) {
   // elements per 16-byte unit and units per row
   constexpr int EPU = FP8 ? 16 : 8;
   constexpr int UPR = D / EPU;                 // column groups
@@ -27,7 +39,23 @@ pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scal
   static_assert(kPoolThreads % UPR == 0, "column groups must tile the block");
   __shared__ float part[PHASES][D];
 
-  const int64_t m = m0 + blockIdx.x;  // this CTA's block
+  int64_t m = m0 + blockIdx.x;  // this CTA's block
+  if (batch.bts) {
+    const int y = blockIdx.y;
+    kpg.bt = batch.bts + static_cast<int64_t>(y) * batch.max_blocks;
+    n_k = __ldg(batch.lens + y);
+    const int64_t cap = static_cast<int64_t>(batch.max_blocks) << kpg.page_shift;
+    if (n_k > cap) {
+      report(ctl, DEV_BAD_INPUT);
+      n_k = cap;
+    }
+    const int64_t My = (n_k + B - 1) / B;
+    m = My - batch.n_last + blockIdx.x;
+    if (n_k <= 0 || m < 0 || m >= My || My > batch.M_max) return;
+    M = batch.M_max;
+    if (kbar) kbar += static_cast<int64_t>(y) * batch.M_max * D;
+    if (kbar_hl) kbar_hl += static_cast<int64_t>(y) * 2 * batch.M_max * D;
+  }
   const int64_t first = m * B;
   const int n_m = static_cast<int>(n_k - first < B ? n_k - first : static_cast<int64_t>(B));
   const int u = threadIdx.x % UPR;
@@ -38,17 +66,20 @@ pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scal
 #pragma unroll
   for (int e = 0; e < EPU; ++e) acc[e] = 0.0f;
 
-  const uint8_t* base = K + first * ROW_BYTES + u * 16;
+  // physical row of the block's r-th key (contiguous or paged cache)
+  auto prow = [&](int r) { return kpg.row(first + r, ctl); };
+  const uint8_t* base = K + u * 16;
   int r = ph;
   // two rows in flight per iteration
   for (; r + PHASES < n_m; r += 2 * PHASES) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(r) * ROW_BYTES));
-    const uint4 b = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(r + PHASES) * ROW_BYTES));
+    const int64_t ra = prow(r), rb = prow(r + PHASES);
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(base + ra * ROW_BYTES));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(base + rb * ROW_BYTES));
     const uint4 ab[2] = {a, b};
     float sc[2] = {1.0f, 1.0f};
     if (FP8) {
-      sc[0] = __ldg(k_scale + first + r);
-      sc[1] = __ldg(k_scale + first + r + PHASES);
+      sc[0] = __ldg(k_scale + ra);
+      sc[1] = __ldg(k_scale + rb);
     }
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -72,10 +103,11 @@ pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scal
     }
   }
   for (; r < n_m; r += PHASES) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(r) * ROW_BYTES));
+    const int64_t ra = prow(r);
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(base + ra * ROW_BYTES));
     const uint32_t* wv = reinterpret_cast<const uint32_t*>(&a);
     if (FP8) {
-      const float sc = __ldg(k_scale + first + r);
+      const float sc = __ldg(k_scale + ra);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t bf2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(wv[i >> 1] >> ((i & 1) * 16)));
@@ -111,13 +143,26 @@ pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scal
 }
 
 template <int D, bool FP8>
-cudaError_t launch(const void* K, const float* k_scale, int64_t n_k, int B, int64_t m0,
-                   int64_t m1, float* kbar, uint16_t* kbar_hl, cudaStream_t s) {
+cudaError_t launch(const void* K, const float* k_scale, const KeyPages& kpg, int64_t n_k, int B,
+                   int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl, const DevCtl& ctl,
+                   cudaStream_t s) {
   const int64_t M = (n_k + B - 1) / B;
   if (m1 > M) m1 = M;
   if (m1 <= m0) return cudaSuccess;
   pool_keys_kernel<D, FP8><<<static_cast<unsigned>(m1 - m0), kPoolThreads, 0, s>>>(
-      static_cast<const uint8_t*>(K), k_scale, n_k, B, M, m0, kbar, kbar_hl);
+      static_cast<const uint8_t*>(K), k_scale, kpg, n_k, B, M, m0, kbar, kbar_hl, ctl,
+      PoolBatch{nullptr, 0, nullptr, 0, 0});
+  return cudaGetLastError();
+}
+
+template <int D, bool FP8>
+cudaError_t launch_batch(const void* K, const float* k_scale, const KeyPages& kpg, int B,
+                         const PoolBatch& batch, int n_seq, float* kbar, uint16_t* kbar_hl,
+                         const DevCtl& ctl, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(batch.n_last), static_cast<unsigned>(n_seq));
+  pool_keys_kernel<D, FP8><<<grid, kPoolThreads, 0, s>>>(static_cast<const uint8_t*>(K), k_scale,
+                                                        kpg, 0, B, batch.M_max, 0, kbar, kbar_hl,
+                                                        ctl, batch);
   return cudaGetLastError();
 }
 
@@ -140,7 +185,46 @@ e4m3_to_bf16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int6
   }
 }
 
+// Logical key rows 0..n_k-1 of an e4m3 cache (paged or contiguous) decoded to
+// bf16 codes (exact) in logical order, 16 codes per thread; with dst_scale the
+// rows' scales are gathered into logical order too.
+__global__ void __launch_bounds__(256)
+e4m3_rows_to_bf16_kernel(const uint8_t* __restrict__ src, const float* __restrict__ scale,
+                         KeyPages kpg, int64_t n_k, int d, uint4* __restrict__ dst,
+                         float* __restrict__ dst_scale, DevCtl ctl) {
+  const int upr = d / 16;  // 16-byte units of an e4m3 row
+  const int64_t n16 = n_k * upr;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t srow = i / upr;
+    const int u = static_cast<int>(i - srow * upr);
+    const int64_t prow = kpg.row(srow, ctl);
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + prow * d) + u);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      o[2 * j] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w[j] & 0xFFFF));
+      o[2 * j + 1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w[j] >> 16));
+    }
+    dst[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    if (dst_scale && u == 0) dst_scale[srow] = __ldg(scale + prow);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_e4m3_rows_to_bf16(const uint8_t* src, const float* scale, const KeyPages& kpg,
+                                     int64_t n_k, int d, uint16_t* dst, float* dst_scale,
+                                     const DevCtl& ctl, cudaStream_t s) {
+  const int64_t n16 = n_k * (d / 16);
+  if (n16 <= 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((n16 + 255) / 256, static_cast<int64_t>(sm_count()) * 8);
+  e4m3_rows_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      src, scale, kpg, n_k, d, reinterpret_cast<uint4*>(dst), dst_scale, ctl);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_e4m3_to_bf16(const uint8_t* src, uint16_t* dst, int64_t n, cudaStream_t s) {
   const int64_t n16 = n / 16;
@@ -151,20 +235,44 @@ cudaError_t launch_e4m3_to_bf16(const uint8_t* src, uint16_t* dst, int64_t n, cu
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool_keys(const void* K, const float* k_scale, bool fp8, int64_t n_k, int d,
-                             int B, int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl,
-                             cudaStream_t s) {
+cudaError_t launch_pool_keys_batch(const void* pages, const float* k_scale, bool fp8,
+                                   const int32_t* block_tables, int max_blocks, int page_shift,
+                                   int64_t n_pages, const int32_t* lens, int n_seq, int d, int B,
+                                   int64_t M_max, int64_t n_last, float* kbar, uint16_t* kbar_hl,
+                                   const DevCtl& ctl, cudaStream_t s) {
+  if (n_seq <= 0 || n_last <= 0) return cudaSuccess;
+  const KeyPages kpg{nullptr, page_shift, n_pages};  // the table is set per sequence
+  const PoolBatch batch{block_tables, max_blocks, lens, M_max, n_last};
   if (fp8) {
     switch (d) {
-      case 32: return launch<32, true>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
-      case 64: return launch<64, true>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
-      case 128: return launch<128, true>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
+      case 32: return launch_batch<32, true>(pages, k_scale, kpg, B, batch, n_seq, kbar, kbar_hl, ctl, s);
+      case 64: return launch_batch<64, true>(pages, k_scale, kpg, B, batch, n_seq, kbar, kbar_hl, ctl, s);
+      case 128: return launch_batch<128, true>(pages, k_scale, kpg, B, batch, n_seq, kbar, kbar_hl, ctl, s);
     }
   } else {
     switch (d) {
-      case 32: return launch<32, false>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
-      case 64: return launch<64, false>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
-      case 128: return launch<128, false>(K, k_scale, n_k, B, m0, m1, kbar, kbar_hl, s);
+      case 32: return launch_batch<32, false>(pages, k_scale, kpg, B, batch, n_seq, kbar, kbar_hl, ctl, s);
+      case 64: return launch_batch<64, false>(pages, k_scale, kpg, B, batch, n_seq, kbar, kbar_hl, ctl, s);
+      case 128: return launch_batch<128, false>(pages, k_scale, kpg, B, batch, n_seq, kbar, kbar_hl, ctl, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_pool_keys(const void* K, const float* k_scale, const KeyPages& kpg, bool fp8,
+                             int64_t n_k, int d, int B, int64_t m0, int64_t m1, float* kbar,
+                             uint16_t* kbar_hl, const DevCtl& ctl, cudaStream_t s) {
+  if (fp8) {
+    switch (d) {
+      case 32: return launch<32, true>(K, k_scale, kpg, n_k, B, m0, m1, kbar, kbar_hl, ctl, s);
+      case 64: return launch<64, true>(K, k_scale, kpg, n_k, B, m0, m1, kbar, kbar_hl, ctl, s);
+      case 128: return launch<128, true>(K, k_scale, kpg, n_k, B, m0, m1, kbar, kbar_hl, ctl, s);
+    }
+  } else {
+    switch (d) {
+      case 32: return launch<32, false>(K, k_scale, kpg, n_k, B, m0, m1, kbar, kbar_hl, ctl, s);
+      case 64: return launch<64, false>(K, k_scale, kpg, n_k, B, m0, m1, kbar, kbar_hl, ctl, s);
+      case 128: return launch<128, false>(K, k_scale, kpg, n_k, B, m0, m1, kbar, kbar_hl, ctl, s);
     }
   }
   return cudaErrorInvalidValue;

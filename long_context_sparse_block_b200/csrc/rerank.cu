@@ -60,6 +60,7 @@ struct RerankParams {
   float* full;
   int64_t ldf;
   DevCtl ctl;
+  KeyPages kpg;  // paged key cache (kpg.bt != nullptr) or contiguous
 };
 
 template <int D, int NB, bool FP8>
@@ -67,8 +68,7 @@ __global__ void __launch_bounds__(kRerankThreads, 1)
 rerank_scores_kernel(const RerankParams p) {
   using L = RerankLayout<D, NB>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const uint32_t sA = smem_u32(smem + L::OFF_A);
   const uint32_t sB = smem_u32(smem + L::OFF_B);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
@@ -136,10 +136,11 @@ rerank_scores_kernel(const RerankParams p) {
       // barrier when they land; FP8: each thread loads its own row's codes for
       // the next tile while decoding this tile's)
       const int32_t* crow = p.cand + static_cast<int64_t>(t) * p.kp;
+      // physical key row of this thread's candidate of a tile (-1: ignored)
       auto cand_of = [&](int tile) -> int64_t {
         const int i = tile * kCand + tid;
         int64_t c = i < p.kp ? static_cast<int64_t>(__ldg(crow + i)) : -1;
-        return (c >= 0 && c <= pos && c < p.n_k) ? c : -1;
+        return (c >= 0 && c <= pos && c < p.n_k) ? p.kpg.row(c, p.ctl) : -1;
       };
       constexpr int U8 = D / 16;  // 16-byte units of an e4m3 row
       int64_t c_next = tiles > 0 ? cand_of(0) : -1;
@@ -270,11 +271,14 @@ rerank_scores_kernel(const RerankParams p) {
       // ahead (and, for FP8 keys, its scale one tile ahead)
       const int first = static_cast<int>((grp - gtile % 2 + 2) % 2);
       const int32_t* crow = p.cand + static_cast<int64_t>(t) * p.kp;
+      // this lane's candidate of a tile: its physical key row (for the FP8
+      // scale), -1 when ignored
       auto cand_of = [&](int tile) -> int64_t {
         const int i = tile * kCand + quad * 32 + lane;
         if (tile >= tiles || i >= p.kp) return -1;
         const int64_t c = __ldg(crow + i);
-        return (c >= 0 && c <= pos && c < p.n_k) ? c : -1;
+        if (c < 0 || c > pos || c >= p.n_k) return -1;
+        return FP8 ? p.kpg.row(c, p.ctl) : c;
       };
       int64_t c_cur = cand_of(first), c_nxt = cand_of(first + 2);
       float ks_cur = (FP8 && c_cur >= 0) ? __ldg(p.k_scale + c_cur) : 1.0f;
@@ -364,12 +368,13 @@ cudaError_t launch2(const RerankParams& p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_rerank_scores(const uint16_t* Q, const float* w, const void* K,
-                                 const float* k_scale, bool fp8, const int32_t* cand, int kp,
-                                 int n_q, int64_t q_pos0, int64_t n_k, int H, int d, float* full,
-                                 int64_t ldf, const DevCtl& ctl, cudaStream_t s) {
+                                 const float* k_scale, const KeyPages& kpg, bool fp8,
+                                 const int32_t* cand, int kp, int n_q, int64_t q_pos0, int64_t n_k,
+                                 int H, int d, float* full, int64_t ldf, const DevCtl& ctl,
+                                 cudaStream_t s) {
   if (n_q <= 0 || kp <= 0) return cudaSuccess;
   RerankParams p{Q, w, static_cast<const uint8_t*>(K), k_scale, cand, kp, n_q, q_pos0, n_k, H, full,
-                 ldf, ctl};
+                 ldf, ctl, kpg};
   if (fp8) {
     switch (d) {
       case 32: return launch2<32, true>(p, s);

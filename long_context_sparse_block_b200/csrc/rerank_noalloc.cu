@@ -80,8 +80,8 @@ extern "C" int misa_rerank_noalloc(const uint16_t* Q, const float* w, const void
   if (!status) return MISA_ERR_CUDA;
   DevCtl ctl{status, wait_limit_ns()};
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (launch_rerank_scores(Q, w, K, k_scale, kdtype == MISA_K_FP8E4M3, cand, kp, n_q, q_pos0, n_k,
-                           H, d, scratch, kp, ctl, s) != cudaSuccess)
+  if (launch_rerank_scores(Q, w, K, k_scale, KeyPages{nullptr, 0, 0}, kdtype == MISA_K_FP8E4M3,
+                           cand, kp, n_q, q_pos0, n_k, H, d, scratch, kp, ctl, s) != cudaSuccess)
     return MISA_ERR_CUDA;
   if (k == 0) return MISA_OK;
   return launch_select_candidates(scratch, kp, cand, kp, n_q, q_pos0, n_k, k, idx, ctl, s) ==

@@ -67,17 +67,36 @@ struct RouteParams {
   int h;
   int row_tiles;
   DevCtl ctl;
+  // decode (lens != nullptr): query t is the last key of its own sequence of
+  // lens[t] keys, with its own pooled keys (slices 2t, 2t+1 of the pooled-key
+  // map, M = blocks per slice); each row tile holds one query's H rows
+  const int32_t* lens;
 };
 
 __device__ __forceinline__ int64_t causal_blocks(const RouteParams& p, int64_t pos) {
   return min((pos + 1) / p.B, p.n_k / p.B);
 }
 
+// Complete causal blocks of query t (decode: every complete block of its own
+// sequence, at most the slice's M).
+__device__ __forceinline__ int64_t query_blocks(const RouteParams& p, int t, int64_t M) {
+  if (p.lens) {
+    const int64_t len = __ldg(p.lens + t);
+    return len <= 0 ? 0 : min(len / p.B, M);
+  }
+  return causal_blocks(p, p.q_pos0 + t);
+}
+
+// Queries per row tile.
+__device__ __forceinline__ int queries_per_tile(const RouteParams& p) {
+  return p.lens ? 1 : kRows / p.H;
+}
+
 // Number of 128-block N tiles a row tile needs (its last query has the most).
-__device__ __forceinline__ int ntiles_of(const RouteParams& p, int rt) {
-  const int QT = kRows / p.H;
+__device__ __forceinline__ int ntiles_of(const RouteParams& p, int rt, int64_t M) {
+  const int QT = queries_per_tile(p);
   const int t_last = min((rt + 1) * QT, p.n_q) - 1;
-  const int64_t nc = causal_blocks(p, p.q_pos0 + t_last);
+  const int64_t nc = query_blocks(p, t_last, M);
   return static_cast<int>((nc + kBlkN - 1) / kBlkN);
 }
 
@@ -92,11 +111,10 @@ __device__ __forceinline__ void better(float& br, int& bj, float r, int j) {
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
-                   const __grid_constant__ CUtensorMap kbmap, const RouteParams p) {
+                   const __grid_constant__ CUtensorMap kbmap, const RouteParams p, int64_t M) {
   using L = RouteLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const uint32_t sA = smem_u32(smem + L::OFF_A);
   const uint32_t sB = smem_u32(smem + L::OFF_B);
   float* r_s = reinterpret_cast<float*>(smem + L::OFF_R);
@@ -143,14 +161,18 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
     uint32_t phase = 0, tcount = 0;
     bool ok = true;
     for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x) {
-      const int nN = ntiles_of(p, rt);
+      const int nN = ntiles_of(p, rt, M);
       if (nN == 0) continue;
+      // decode: the tile's rows start at query rt's first head row, and its
+      // pooled keys are slices 2rt (hi) and 2rt+1 (lo)
+      const int row0 = p.lens ? rt * p.H : rt * kRows;
+      const int z0 = p.lens ? 2 * rt : 0;
       if (lane == 0) {
         ok = mbar_wait(bar(AEMPTY), (tcount & 1) ^ 1, abort_flag, p.ctl);
         if (ok) {
           mbar_arrive_expect_tx(bar(AFULL), L::A_BYTES);
           for (int c = 0; c < L::KCH; ++c)
-            tma_load_2d(sA + c * L::A_CHUNK, &qmap, bar(AFULL), c * (L::ROWB / 2), rt * kRows);
+            tma_load_2d(sA + c * L::A_CHUNK, &qmap, bar(AFULL), c * (L::ROWB / 2), row0);
         }
         for (int nb = 0; nb < nN && ok; ++nb) {
           ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
@@ -160,7 +182,7 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
           for (int half = 0; half < 2; ++half)
             for (int c = 0; c < L::KCH; ++c)
               tma_load_3d(dst + half * L::B_HALF + c * L::B_CHUNK, &kbmap, bar(FULL + stage),
-                          c * (L::ROWB / 2), nb * kBlkN, half);
+                          c * (L::ROWB / 2), nb * kBlkN, z0 + half);
           if (++stage == kRouteStages) {
             stage = 0;
             phase ^= 1;
@@ -179,7 +201,7 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
     bool ok = true;
     constexpr uint32_t idesc = umma_idesc_bf16_f32(kRows, kBlkN);
     for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x) {
-      const int nN = ntiles_of(p, rt);
+      const int nN = ntiles_of(p, rt, M);
       if (nN == 0) continue;
       if (lane == 0) {
         ok = mbar_wait(bar(AFULL), tcount & 1, abort_flag, p.ctl);
@@ -223,7 +245,7 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
   } else {
     // ------------------------------------------------------------ epilogue / top-h
     const bool top_role = warp >= 2 + kRouteEpiWarps;
-    const int QT = kRows / p.H;
+    const int QT = queries_per_tile(p);
     uint32_t rcount = 0;  // row tiles handed over so far (buffer = rcount & 1)
     bool ok = true;
     if (!top_role) {
@@ -232,10 +254,10 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
       int acc = 0;
       uint32_t accph = 0;
       for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x, ++rcount) {
-        const int nN = ntiles_of(p, rt);
+        const int nN = ntiles_of(p, rt, M);
         const int t = rt * QT + row / p.H;
-        const bool valid = t < p.n_q;
-        const int64_t nc = valid ? causal_blocks(p, p.q_pos0 + t) : 0;
+        const bool valid = t < p.n_q && row / p.H < QT;
+        const int64_t nc = valid ? query_blocks(p, t, M) : 0;
         float sum = 0.0f;
         for (int nb = 0; nb < nN; ++nb) {
           if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
@@ -348,7 +370,7 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
 }
 
 template <int D>
-cudaError_t launch_d(const RouteParams& p, const CUtensorMap& qm, const CUtensorMap& km,
+cudaError_t launch_d(const RouteParams& p, const CUtensorMap& qm, const CUtensorMap& km, int64_t M,
                      cudaStream_t s) {
   using L = RouteLayout<D>;
   auto kern = route_heads_kernel<D>;
@@ -356,20 +378,15 @@ cudaError_t launch_d(const RouteParams& p, const CUtensorMap& qm, const CUtensor
   if (e != cudaSuccess) return e;
   const int grid = std::min(sm_count(), p.row_tiles);
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kRouteThreads, L::ALLOC, s>>>(qm, km, p);
+  kern<<<grid, kRouteThreads, L::ALLOC, s>>>(qm, km, p, M);
   return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
-                               int n_q, int64_t q_pos0, int64_t n_k, int H, int d, int B, int h,
-                               int32_t* heads, float* r_out, const DevCtl& ctl, cudaStream_t s) {
-  if (n_q <= 0) return cudaSuccess;
-  const int64_t M = (n_k + B - 1) / B;
-  const int64_t rows = static_cast<int64_t>(n_q) * H;
-  const int row_tiles = static_cast<int>((rows + kRows - 1) / kRows);
-  RouteParams p{w, heads, r_out, n_q, q_pos0, n_k, H, B, h, row_tiles, ctl};
+// Tensor maps and launch: Q as [n_q * H, d] rows; the pooled keys as [slices,
+// M, d] (slices = 2: hi, lo; decode: 2 per sequence).
+cudaError_t launch_route(const uint16_t* Q, const uint16_t* kbar_hl, const RouteParams& p, int d,
+                         int64_t M, int64_t slices, cudaStream_t s) {
+  const int64_t rows = static_cast<int64_t>(p.n_q) * p.H;
   const int rowb = d >= 64 ? 128 : 64;
   const CUtensorMapSwizzle swz = rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap qm, km;
@@ -382,7 +399,8 @@ cudaError_t launch_route_heads(const uint16_t* Q, const float* w, const uint16_t
       return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(M), 2};
+    const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(M),
+                              static_cast<uint64_t>(slices)};
     const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(M * d * 2)};
     const uint32_t box[3] = {static_cast<uint32_t>(rowb / 2), static_cast<uint32_t>(kBlkN), 1};
     if (encode_tensor_map(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, kbar_hl, dims, strides, box,
@@ -390,11 +408,34 @@ cudaError_t launch_route_heads(const uint16_t* Q, const float* w, const uint16_t
       return cudaErrorInvalidValue;
   }
   switch (d) {
-    case 32: return launch_d<32>(p, qm, km, s);
-    case 64: return launch_d<64>(p, qm, km, s);
-    case 128: return launch_d<128>(p, qm, km, s);
+    case 32: return launch_d<32>(p, qm, km, M, s);
+    case 64: return launch_d<64>(p, qm, km, M, s);
+    case 128: return launch_d<128>(p, qm, km, M, s);
   }
   return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_route_heads(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
+                               int n_q, int64_t q_pos0, int64_t n_k, int H, int d, int B, int h,
+                               int32_t* heads, float* r_out, const DevCtl& ctl, cudaStream_t s) {
+  if (n_q <= 0) return cudaSuccess;
+  const int64_t M = (n_k + B - 1) / B;
+  const int64_t rows = static_cast<int64_t>(n_q) * H;
+  const int row_tiles = static_cast<int>((rows + kRows - 1) / kRows);
+  const RouteParams p{w, heads, r_out, n_q, q_pos0, n_k, H, B, h, row_tiles, ctl, nullptr};
+  return launch_route(Q, kbar_hl, p, d, M, 2, s);
+}
+
+cudaError_t launch_route_heads_decode(const uint16_t* Q, const float* w, const uint16_t* kbar_hl,
+                                      int64_t M_max, const int32_t* lens, int n_seq, int H, int d,
+                                      int B, int h, int32_t* heads, float* r_out, const DevCtl& ctl,
+                                      cudaStream_t s) {
+  if (n_seq <= 0) return cudaSuccess;
+  // n_k only bounds the complete blocks in prefill mode; decode reads lens
+  const RouteParams p{w, heads, r_out, n_seq, 0, M_max * B, H, B, h, n_seq, ctl, lens};
+  return launch_route(Q, kbar_hl, p, d, M_max, 2 * static_cast<int64_t>(n_seq), s);
 }
 
 }  // namespace misa

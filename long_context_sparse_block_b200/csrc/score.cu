@@ -134,6 +134,8 @@ struct ScoreParams {
   // holding a row t with gate[1 + t] != 0
   const int* gate;
   const float* q_scale;  // e4m3 queries only: [n_q, H] per (query, head) row
+  KeyPages kpg;          // paged key cache (kpg.bt != nullptr) or contiguous
+  int64_t key_rows;      // rows of the key tensor map (n_k, or the page pool's rows)
 };
 
 // Flattened schedule over (group g, key tile kt): each role of a CTA walks the
@@ -221,8 +223,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
   constexpr int EC = Epi<HT, FP8>::COLS;
   constexpr int QG = kCols / HT;  // queries per group
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const uint32_t sA = smem_u32(smem + L::OFF_A);
   const uint32_t sB = smem_u32(smem + L::OFF_B);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
@@ -311,10 +312,24 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
         ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
         if (ok) {
           mbar_arrive_expect_tx(bar(FULL + stage), L::A_BYTES);
+          if (!p.kpg.paged()) {
 #pragma unroll
-          for (int c = 0; c < L::KCH; ++c)
-            tma_load_2d(sA + stage * L::A_BYTES + c * L::A_CHUNK, &kmap, bar(FULL + stage),
-                        c * (L::ROWB / EB), static_cast<int>(it.kt * kTileKeys));
+            for (int c = 0; c < L::KCH; ++c)
+              tma_load_2d(sA + stage * L::A_BYTES + c * L::A_CHUNK, &kmap, bar(FULL + stage),
+                          c * (L::ROWB / EB), static_cast<int>(it.kt * kTileKeys));
+          } else {
+            // one box per page of the tile; pages past the last key are read as
+            // fill (a box at the end of the pool), never through the table
+            const int ps = 1 << p.kpg.page_shift;
+            for (int j = 0; j < kTileKeys / ps; ++j) {
+              const int64_t s0 = it.kt * kTileKeys + j * ps;
+              const int y = static_cast<int>(s0 < p.n_k ? p.kpg.row(s0, p.ctl) : p.key_rows);
+#pragma unroll
+              for (int c = 0; c < L::KCH; ++c)
+                tma_load_2d(sA + stage * L::A_BYTES + c * L::A_CHUNK + j * ps * L::ROWB, &kmap,
+                            bar(FULL + stage), c * (L::ROWB / EB), y);
+            }
+          }
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -408,8 +423,8 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           const int r = x / U8, u = x % U8;
           const int64_t key = kt * kTileKeys + r;
           const bool in = key < p.n_k;
-          cp_async16(raw0 + rb * L::RAW_TILE + x * 16, p.K8 + (in ? key : 0) * D + u * 16,
-                     in ? 16u : 0u);
+          cp_async16(raw0 + rb * L::RAW_TILE + x * 16,
+                     p.K8 + (in ? p.kpg.row(key, p.ctl) : 0) * D + u * 16, in ? 16u : 0u);
         }
         cp_async_commit();
       };
@@ -485,7 +500,10 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
     uint32_t accph = 0, tcount = 0;
     int prev_g = -1;
     float* tau_s = reinterpret_cast<float*>(smem + L::OFF_TAU) + e * 16;  // select: thresholds
-    (void)tau_s;
+    // the per-tile reads of weights and thresholds: shared-space loads with
+    // 32-bit addresses (broadcasts: every lane reads the same word)
+    const uint32_t w_s32 = smem_u32(w_s), tau_s32 = smem_u32(tau_s);
+    (void)tau_s32;
     for (; it.left > 0; it.next(p), ++tcount) {
       if (it.g != prev_g) {
         for (int i = lane; i < EC; i += 32) {
@@ -523,7 +541,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
         float2 a2 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int j = 0; j < HT; j += 4) {
-          const float4 w4 = *reinterpret_cast<const float4*>(w_s + qq * HT + j);
+          const float4 w4 = lds_f32x4(w_s32 + static_cast<uint32_t>((qq * HT + j) * 4));
           const uint32_t* x = v + qq * HT + j;
           a2 = fma2(make_float2(w4.x, w4.y),
                     make_float2(relu(__uint_as_float(x[0])), relu(__uint_as_float(x[1]))), a2);
@@ -568,7 +586,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
         for (int qq = SPLIT ? QPW / 2 : 0; qq < QPW; ++qq) sums[qq] = qsum(qq);
         if constexpr (KSC) {
           // per-token scale > 0: w * ReLU(scale * dot) = scale * w * ReLU(dot)
-          const float ks = s_ok ? __ldg(p.k_scale + s) : 0.0f;
+          const float ks = s_ok ? __ldg(p.k_scale + p.kpg.row(s, p.ctl)) : 0.0f;
 #pragma unroll
           for (int qq = 0; qq < QPW; ++qq) sums[qq] *= ks;
         }
@@ -586,7 +604,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           if (full) {
 #pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
-              const bool pass = sums[qq] >= tau_s[qq];
+              const bool pass = sums[qq] >= lds_f32(tau_s32 + qq * 4);
               m[qq] = __ballot_sync(0xffffffffu, pass);
               if (pass) *dst = sums[qq];
               dst += p.ld;
@@ -597,7 +615,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
             const uint32_t valid = s_ok ? (((1u << q_end) - 1u) & ~((1u << cut) - 1u)) : 0u;
 #pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
-              const bool pass = ((valid >> qq) & 1u) && sums[qq] >= tau_s[qq];
+              const bool pass = ((valid >> qq) & 1u) && sums[qq] >= lds_f32(tau_s32 + qq * 4);
               m[qq] = __ballot_sync(0xffffffffu, pass);
               if (pass) *dst = sums[qq];
               dst += p.ld;
@@ -644,7 +662,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
             const float2 w2 = *reinterpret_cast<const float2*>(w_s + qq * 2);
             sum = fmaf(w2.y, relu(__uint_as_float(v[qq * 2 + 1])), w2.x * relu(__uint_as_float(v[qq * 2])));
           }
-          if constexpr (KSC) sum *= s_ok ? __ldg(p.k_scale + s) : 0.0f;
+          if constexpr (KSC) sum *= s_ok ? __ldg(p.k_scale + p.kpg.row(s, p.ctl)) : 0.0f;
           const int64_t t = tq0 + qq;
           if (t < p.n_q && s_ok) *dst = (s <= p.q_pos0 + t) ? sum : -INFINITY;
           dst += p.ld;
@@ -726,16 +744,21 @@ cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s
     const int t_last = std::min((g + 1) * QG, a.n_q) - 1;
     total += std::min<int64_t>(a.q_pos0 + t_last, a.n_k - 1) / kTileKeys + 1;
   }
+  // key tensor map: [key_rows, d] with one box per 128-key tile, or per page
+  const bool paged = a.kpg.paged();
+  const int64_t key_rows = paged ? (a.kpg.n_pages << a.kpg.page_shift) : a.n_k;
+  const uint32_t box_rows = paged ? (1u << a.kpg.page_shift) : static_cast<uint32_t>(kTileKeys);
+  if (paged && (box_rows > static_cast<uint32_t>(kTileKeys) || box_rows < 8)) return cudaErrorInvalidValue;
   ScoreParams p{a.Q, a.w, a.heads, a.k_scale, static_cast<const uint8_t*>(a.K), a.logits, a.ld,
                 a.n_q, a.q_pos0, a.n_k, a.H, total, ctl, a.tau, a.mask, a.mask_ld,
-                a.gate, a.q_scale};
+                a.gate, a.q_scale, a.kpg, key_rows};
   CUtensorMap map;
   std::memset(&map, 0, sizeof map);
   if (a.q8) {  // e4m3 queries and keys: one-byte key tiles by TMA, kind::f8f6f4
     if (!a.fp8 || a.k_bf16 || (a.d != 64 && a.d != 128)) return cudaErrorNotSupported;
-    const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.n_k)};
+    const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(key_rows)};
     const uint64_t strides[1] = {static_cast<uint64_t>(a.d)};
-    const uint32_t box[2] = {static_cast<uint32_t>(a.d), static_cast<uint32_t>(kTileKeys)};
+    const uint32_t box[2] = {static_cast<uint32_t>(a.d), box_rows};
     if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.K, dims, strides, box,
                           a.d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) !=
         CUDA_SUCCESS)
@@ -750,10 +773,10 @@ cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s
     }
     return cudaErrorInvalidValue;
   }
-  const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.n_k)};
+  const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(key_rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(a.d) * 2};
   const int rowb = a.d >= 64 ? 128 : 64;
-  const uint32_t box[2] = {static_cast<uint32_t>(rowb / 2), static_cast<uint32_t>(kTileKeys)};
+  const uint32_t box[2] = {static_cast<uint32_t>(rowb / 2), box_rows};
   if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.K, dims, strides, box,
                         rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) !=
       CUDA_SUCCESS)
@@ -772,28 +795,6 @@ cudaError_t launch_score(const ScoreLaunch& a, const DevCtl& ctl, cudaStream_t s
     case 128: return launch_d<128, 0>(p, a.h, sel, map, s);
   }
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_score_tokens(const uint16_t* Q, const float* w, const int32_t* heads,
-                                const void* K, const float* k_scale, bool fp8, int n_q,
-                                int64_t q_pos0, int64_t n_k, int H, int d, int h, float* logits,
-                                int64_t ld, const DevCtl& ctl, cudaStream_t s) {
-  ScoreLaunch a{};
-  a.Q = Q;
-  a.w = w;
-  a.heads = heads;
-  a.K = K;
-  a.k_scale = k_scale;
-  a.fp8 = fp8;
-  a.n_q = n_q;
-  a.q_pos0 = q_pos0;
-  a.n_k = n_k;
-  a.H = H;
-  a.d = d;
-  a.h = h;
-  a.logits = logits;
-  a.ld = ld;
-  return launch_score(a, ctl, s);
 }
 
 }  // namespace misa

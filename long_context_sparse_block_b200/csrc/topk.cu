@@ -63,6 +63,7 @@ struct TopkParams {
   int cap;               // shared-memory list capacity (entries)
   DevCtl ctl;
   const int* gate;       // nullable: row t is done unless gate[1 + t] != 0
+  const int32_t* row_len;  // nullable: row t has row_len[t] visible entries (else pos(t) + 1)
 };
 
 __device__ __forceinline__ uint32_t f2key(float f) {
@@ -280,26 +281,77 @@ struct RegionSrc {
   }
 };
 
-// Exact m-th largest key among the present entries of `src` (1 <= m <= present).
-// Returns T; `need` = how many entries equal to T belong to the m largest.
+// Exact m-th largest key T among the present entries of `src` (1 <= m <=
+// present); `need` = how many entries equal to T belong to the m largest.
+// A radix select with the digits placed where the keys differ: every
+// present key shares the bits above the highest bit in which the largest and
+// the smallest present key differ, and each round histograms the next (at
+// most) 12 bits below the bits already fixed, among the entries that still
+// agree with the answer on them.  The lists this selects from hold a narrow
+// band of values (the kept top few percent of a row), which a fixed top-bits
+// digit piles onto a few bins (and their shared-memory atomics onto a few
+// addresses); here they spread over up to 4096 bins.
 template <class Src>
-__device__ uint32_t kth_largest(const Src& src, uint32_t m, uint32_t* hist, SmemCtl& sc,
-                                uint32_t& need) {
-  for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) hist[i] = 0u;
-  __syncthreads();
+__device__ uint32_t kth_largest_spread(const Src& src, uint32_t m, uint32_t* hist, SmemCtl& sc,
+                                       uint32_t& need) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
   for (int64_t base = 0; base < src.n; base += kChunk) {
     uint32_t key[4], pos[4];
     src.load4(base + threadIdx.x * 4, key, pos);
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      if (key[e] != 0u) atomicAdd(&hist[key[e] >> 20], 1u);
+      if (key[e] != 0u) {
+        lo = min(lo, key[e]);
+        hi = max(hi, key[e]);
+      }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+  }
+  if (lane == 0) {
+    sc.scan[warp] = lo;
+    hist[warp] = hi;
   }
   __syncthreads();
-  find_bin<kBins1>(hist, m, sc);
-  const uint32_t b1 = sc.res[0], above1 = sc.res[1];
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    lo = min(lo, sc.scan[w]);
+    hi = max(hi, hist[w]);
+  }
   __syncthreads();
-  uint32_t T;
-  refine(src, b1, above1, m, hist, sc, T, need);
+  const uint32_t diff = hi ^ lo;
+  if (diff == 0u) {  // every present key equal
+    need = m;
+    return hi;
+  }
+  int hib = 31 - __clz(diff);  // bits above hib are common to every present key
+  uint32_t T = hib == 31 ? 0u : (hi >> (hib + 1)) << (hib + 1);
+  while (true) {
+    const int lob = hib >= 11 ? hib - 11 : 0;
+    const uint32_t dmask = (1u << (hib - lob + 1)) - 1u;
+    for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int64_t base = 0; base < src.n; base += kChunk) {
+      uint32_t key[4], pos[4];
+      src.load4(base + threadIdx.x * 4, key, pos);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool agree = hib == 31 || (key[e] >> (hib + 1)) == (T >> (hib + 1));
+        if (key[e] != 0u && agree) atomicAdd(&hist[(key[e] >> lob) & dmask], 1u);
+      }
+    }
+    __syncthreads();
+    find_bin<kBins1>(hist, m, sc);
+    T |= sc.res[0] << lob;
+    m -= sc.res[1];
+    __syncthreads();
+    if (lob == 0) break;
+    hib = lob - 1;
+  }
+  need = m;
   return T;
 }
 
@@ -492,7 +544,7 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   const RegionSrc rs{lkeys, lposs, counts, static_cast<int64_t>(kWarps) * region, region, inv};
   // ---- exact k-th key within the list
   uint32_t T = 0u, need = 0u;
-  if (total > k) T = kth_largest(rs, k, hist, sc, need);
+  if (total > k) T = kth_largest_spread(rs, k, hist, sc, need);
   // ---- kept positions: key > T, and the `need` lowest positions with key == T,
   // marked in a bitmap of the row (ascending output without a sort)
   uint32_t* bitmap = hist;                       // kBins1 words = 131072 positions
@@ -537,7 +589,8 @@ topk_kernel(const TopkParams p) {
 
   const int t = blockIdx.x;
   const uint32_t k = static_cast<uint32_t>(p.k);
-  const int64_t n = min(p.q_pos0 + t + 1, p.n_k);
+  const int64_t n = p.row_len ? max(int64_t(0), min(static_cast<int64_t>(__ldg(p.row_len + t)), p.n_k))
+                              : min(p.q_pos0 + t + 1, p.n_k);
   const float* row = p.vals + static_cast<int64_t>(t) * p.ld;
   const RowSrc src{row, n, (reinterpret_cast<uintptr_t>(row) & 15u) == 0u};
   const OutEmit out{p.idx + static_cast<int64_t>(t) * p.k, k};
@@ -607,20 +660,25 @@ constexpr double kFusedMargin = 1.6;  // ~1.6 k candidates expected above tau
 constexpr int kSampleBlock = 128;     // keys per contiguous sample block
 
 // Copies the keys of n_blocks contiguous 128-key blocks, evenly spaced over
-// [0, span), into a dense sample (and their FP8 scales when given).
+// [0, span), into a dense sample (and their FP8 scales when given); the keys
+// come from a contiguous or a paged cache.
 __global__ void __launch_bounds__(256)
-gather_sample_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scale,
+gather_sample_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scale, KeyPages kpg,
                      int row_bytes, int64_t span, int n_blocks, uint8_t* __restrict__ Ks,
-                     float* __restrict__ ks_scale) {
+                     float* __restrict__ ks_scale, DevCtl ctl) {
   const int b = blockIdx.x;
   const int64_t start = n_blocks > 1 ? (span - kSampleBlock) * b / (n_blocks - 1) : 0;
-  const int units = kSampleBlock * row_bytes / 16;
-  const uint4* src = reinterpret_cast<const uint4*>(K + start * row_bytes);
+  const int upr = row_bytes / 16;
+  const int units = kSampleBlock * upr;
   uint4* dst = reinterpret_cast<uint4*>(Ks + static_cast<int64_t>(b) * kSampleBlock * row_bytes);
-  for (int i = threadIdx.x; i < units; i += blockDim.x) dst[i] = __ldg(src + i);
+  for (int i = threadIdx.x; i < units; i += blockDim.x) {
+    const int r = i / upr;
+    const int64_t prow = kpg.row(start + r, ctl);
+    dst[i] = __ldg(reinterpret_cast<const uint4*>(K + prow * row_bytes) + (i - r * upr));
+  }
   if (k_scale)
     for (int i = threadIdx.x; i < kSampleBlock; i += blockDim.x)
-      ks_scale[b * kSampleBlock + i] = __ldg(k_scale + start + i);
+      ks_scale[b * kSampleBlock + i] = __ldg(k_scale + kpg.row(start + i, ctl));
 }
 
 // Per row: tau[t] = lower edge of the 22-bit key bin holding the m-th largest
@@ -742,7 +800,8 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
   const ListSrc ls{keys, poss, static_cast<int64_t>(total)};
   const OutEmit out{idx + static_cast<int64_t>(t) * k, static_cast<uint32_t>(k)};
   uint32_t T = 0u, need = 0u;
-  if (total > static_cast<uint32_t>(k)) T = kth_largest(ls, static_cast<uint32_t>(k), hist, sc, need);
+  if (total > static_cast<uint32_t>(k))
+    T = kth_largest_spread(ls, static_cast<uint32_t>(k), hist, sc, need);
   const uint32_t kept = ordered_select(ls, T, need, static_cast<uint32_t>(k), out, sc);
   for (uint32_t i = min(kept, static_cast<uint32_t>(k)) + threadIdx.x; i < static_cast<uint32_t>(k);
        i += kTopkThreads)
@@ -810,7 +869,7 @@ select_candidates_kernel(const float* __restrict__ vals, int64_t ldv,
 
   const ListSrc ls{keys, toks, static_cast<int64_t>(kp)};
   uint32_t T = 0u, need = 0u;  // present <= k: every present entry (key > 0)
-  if (present > kk) T = kth_largest(ls, kk, hist, sc, need);
+  if (present > kk) T = kth_largest_spread(ls, kk, hist, sc, need);
   if (!unordered) {
     const uint32_t kept = ordered_select(ls, T, need, kk, OutEmit{out, kk}, sc);
     for (uint32_t i = min(kept, kk) + threadIdx.x; i < kk; i += kTopkThreads) out[i] = -1;
@@ -849,7 +908,8 @@ select_candidates_kernel(const float* __restrict__ vals, int64_t ldv,
 }  // namespace
 
 cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k,
-                        int k, int32_t* idx, const DevCtl& ctl, cudaStream_t s, const int* gate) {
+                        int k, int32_t* idx, const DevCtl& ctl, cudaStream_t s, const int* gate,
+                        const int32_t* row_len) {
   if (n_q <= 0 || k <= 0) return cudaSuccess;
   // list capacity: kFastCap for k <= 4096 (three CTAs per SM); larger k need
   // room for ~1.4 k sampled-threshold entries (fast path) or for the entries in
@@ -860,15 +920,17 @@ cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, 
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  TopkParams p{vals, ld, n_q, q_pos0, n_k, k, idx, cap, ctl, gate};
+  TopkParams p{vals, ld, n_q, q_pos0, n_k, k, idx, cap, ctl, gate, row_len};
   topk_kernel<<<n_q, kTopkThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_sample(const void* K, const float* k_scale, int row_bytes, int64_t span,
-                                 int n_blocks, void* Ks, float* ks_scale, cudaStream_t s) {
-  gather_sample_kernel<<<n_blocks, 256, 0, s>>>(static_cast<const uint8_t*>(K), k_scale, row_bytes,
-                                                span, n_blocks, static_cast<uint8_t*>(Ks), ks_scale);
+cudaError_t launch_gather_sample(const void* K, const float* k_scale, const KeyPages& kpg,
+                                 int row_bytes, int64_t span, int n_blocks, void* Ks,
+                                 float* ks_scale, const DevCtl& ctl, cudaStream_t s) {
+  gather_sample_kernel<<<n_blocks, 256, 0, s>>>(static_cast<const uint8_t*>(K), k_scale, kpg,
+                                                row_bytes, span, n_blocks,
+                                                static_cast<uint8_t*>(Ks), ks_scale, ctl);
   return cudaGetLastError();
 }
 

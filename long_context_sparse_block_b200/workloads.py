@@ -246,6 +246,17 @@ def generate(wl: Workload, fp8_keys: bool = False, fp8_queries: bool = False) ->
     return out
 
 
+def page_table(n_k: int, page_size: int, seed: int, spare: int = 3) -> tuple:
+    """A paged layout for n_k keys: pages of `page_size` rows in a pool of
+    ceil(n_k / page_size) + `spare` pages, logical block b stored in page
+    table[b], the pages drawn in a seeded random order.  Returns (table int32,
+    n_pages).  (Storage layout only; the values stay those of the keys.)"""
+    n_blocks = -(-n_k // page_size)
+    n_pages = n_blocks + spare
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return rng.permutation(n_pages)[:n_blocks].astype(np.int32), n_pages
+
+
 def exact_arithmetic_inputs(n_q: int, q_pos0: int, n_k: int, H: int, d: int, seed: int,
                             qmax: int = 3, kmax: int = 3):
     """Small-integer Q and K with power-of-two w, so that every dot product, block

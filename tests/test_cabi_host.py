@@ -125,6 +125,41 @@ def test_invalid_arguments_rejected_before_launch(lib):
                           None) == lib.MISA_ERR_WORKSPACE
 
 
+def test_paged_arguments_rejected_before_launch(lib):
+    so = _so(lib)
+    p = ctypes.c_void_p(16 * 1024)
+    odd = ctypes.c_void_p(16 * 1024 + 2)
+    INV, UNS = lib.MISA_ERR_INVALID_ARG, lib.MISA_ERR_UNSUPPORTED
+    # (pages, scales, kdtype, block table, page size, pages in the pool)
+    good = (p, None, 0, p, 64, 100)
+    # pool: no table, page size not 16/32/64/128, empty pool, pool rows past 2^31,
+    # FP8 pages without scales, misaligned table
+    pool = so.misa_pool_keys_paged
+    assert pool(p, None, 0, None, 64, 100, 1000, 128, 64, 0, 16, p, p, None) == INV
+    assert pool(p, None, 0, p, 48, 100, 1000, 128, 64, 0, 16, p, p, None) == UNS
+    assert pool(p, None, 0, p, 8, 100, 1000, 128, 64, 0, 16, p, p, None) == UNS
+    assert pool(p, None, 0, p, 64, 0, 1000, 128, 64, 0, 16, p, p, None) == INV
+    assert pool(p, None, 0, p, 128, 1 << 24, 1000, 128, 64, 0, 16, p, p, None) == INV
+    assert pool(p, None, 1, p, 64, 100, 1000, 128, 64, 0, 16, p, p, None) == INV
+    assert pool(p, None, 0, odd, 64, 100, 1000, 128, 64, 0, 16, p, p, None) == INV
+    assert pool(*good, 1000, 128, 64, 3, 3, p, p, None) == 0          # empty range
+    # score, fused score + top-k and rerank refuse the same tables
+    sc = so.misa_score_tokens_paged
+    assert sc(p, p, p, p, None, 0, None, 64, 100, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    assert sc(p, p, p, p, None, 0, p, 24, 100, 10, 0, 100, 64, 128, 8, p, 100, None) == UNS
+    assert sc(p, p, p, *good, 10, 0, 100, 64, 128, 8, p, 99, None) == INV
+    assert sc(p, p, p, *good, 0, 0, 100, 64, 128, 8, p, 100, None) == 0
+    st = so.misa_score_topk_paged
+    assert st(p, p, p, p, None, 0, None, 64, 100, 10, 8000, 9000, 64, 128, 8, 64, p, p, 9000, p,
+              1 << 30, None) == INV
+    assert st(p, p, p, *good, 10, 8000, 9000, 64, 128, 8, 64, p, p, 9000, None, 0,
+              None) == lib.MISA_ERR_WORKSPACE
+    rr = so.misa_rerank_paged
+    assert rr(p, p, p, None, 0, None, 64, 100, p, 16, 4, 0, 100, 64, 128, 8, p, p, None, 0,
+              None) == INV
+    assert rr(p, p, *good, p, 16, 4, 0, 100, 64, 128, 32, p, p, None, 0, None) == INV
+
+
 def test_empty_work_is_a_no_op(lib):
     so = _so(lib)
     p = ctypes.c_void_p(16 * 1024)

@@ -80,3 +80,97 @@ def test_decode_step_matches_oracle(lib):
     if np.array_equal(heads.cpu().numpy(), h_o):
         ref = oracle.score(Qd, wd, h_o, Kd, n_k - 1)
         assert recall(idx, oracle.topk(ref, n_k - 1, n_k, k)) >= 0.999
+
+
+# ------------------------------------------------------------------ batched decode
+
+def _decode_batch(lens, H, d, B, h, k, ps, seed):
+    """One new query per sequence at the end of its own keys; all keys in one
+    page pool (pages of ps keys in a seeded random order, unused rows +inf)."""
+    seqs = []
+    for b, n in enumerate(lens):
+        wl = W.small_workload(f"dec{seed}_{b}", n_q=1, q_pos0=n - 1, n_k=n, H=H, d=d, B=B, h=h,
+                              k=k, seed=seed + b, generator="clustered")
+        seqs.append(W.generate(wl))
+    nb = [-(-n // ps) for n in lens]
+    max_blocks = max(nb)
+    table, n_pages = W.page_table(sum(nb) * ps, ps, seed=seed)
+    pages = np.full((n_pages, ps, d), 0x7F80, dtype=np.uint16)
+    bts = np.full((len(lens), max_blocks), -1, dtype=np.int32)
+    o = 0
+    for b, n in enumerate(lens):
+        flat = np.full((nb[b] * ps, d), 0x7F80, dtype=np.uint16)
+        flat[:n] = seqs[b]["K"]
+        bts[b, :nb[b]] = table[o:o + nb[b]]
+        pages[table[o:o + nb[b]]] = flat.reshape(nb[b], ps, d)
+        o += nb[b]
+    Q = np.concatenate([s["Q"] for s in seqs])
+    w = np.concatenate([s["w"] for s in seqs])
+    return seqs, Q, w, pages, bts
+
+
+@pytest.mark.parametrize("H,d,h,ps", [(64, 128, 8, 64), (64, 128, 64, 32), (32, 64, 4, 128)])
+def test_batched_decode_matches_oracle(lib, H, d, h, ps):
+    lens = [1, 100, 128, 3000, 7777, 20000]
+    B, k = 128, 256
+    seqs, Qn, wn, pages_n, bts_n = _decode_batch(lens, H, d, B, h, k, ps, seed=500 + h)
+    Q, w, pages, bts = dev(Qn), dev(wn), dev(pages_n), dev(bts_n)
+    seq_lens = dev(np.array(lens, dtype=np.int32))
+    M_max = -(-bts_n.shape[1] * ps // B)
+    _, hl = lib.misa_decode_pool_keys(pages, bts, seq_lens, B, M_max, M_max)
+    dense = h == H
+    heads, r = lib.misa_decode_route_heads(Q, w, hl, seq_lens, B, h, want_r=True)
+    idx, logits = lib.misa_decode_score_topk(Q, w, None if dense else heads, pages, bts, seq_lens,
+                                             k, h=h)
+    assert lib.misa_last_device_status() == lib.MISA_OK
+    hl_np, heads_np, r_np = hl.cpu().numpy(), heads.cpu().numpy(), r.cpu().numpy()
+    idx_np, lg_np = idx.cpu().numpy(), logits.cpu().numpy()
+    for b, n in enumerate(lens):
+        g = inputs_to_device(seqs[b])
+        M = -(-n // B)
+        # pooling and routing equal the single-sequence calls bit for bit
+        _, hl1 = lib.misa_pool_keys(g["K"], B)
+        hl1 = hl1.cpu().numpy()
+        assert np.array_equal(hl_np[b, 0, :M], hl1[0]) and np.array_equal(hl_np[b, 1, :M], hl1[1])
+        heads1, r1 = lib.misa_route_heads(g["Q"], g["w"], dev(hl1.view(np.int16)), n - 1, n, B, h,
+                                          want_r=True)
+        assert np.array_equal(r_np[b], r1.cpu().numpy()[0])
+        assert np.array_equal(heads_np[b], heads1.cpu().numpy()[0])
+        # against the oracle
+        Qd, Kd, wd = oracle.decode_inputs(seqs[b])
+        kb = oracle.pool_keys(Kd, B)
+        r_o, h_o = oracle.route(Qd, wd, kb, n - 1, n, B, h)
+        check_heads(heads_np[b:b + 1], r_o, h_o, h, r_gpu=r_np[b:b + 1])
+        hs = heads_np[b:b + 1] if not dense else np.arange(H, dtype=np.int32)[None, :]
+        ref = oracle.score(Qd, wd, hs, Kd, n - 1)[0]
+        mag = (np.abs(wd[0, hs[0]])[:, None] * np.maximum(Qd[0, hs[0]] @ Kd.T, 0)).sum(0)
+        row = lg_np[b, :n]
+        assert np.all(np.abs(row.astype(np.float64) - ref) <= 2e-3 * mag + 1e-5), f"seq {b}"
+        assert np.array_equal(idx_np[b], oracle.topk(row[None, :], n - 1, n, k)[0])
+        assert recall(idx_np[b:b + 1], oracle.topk(ref[None, :], n - 1, n, k)) >= 0.999
+        # and the prefill scoring kernel on the same query gives the same logits
+        lg1 = lib.misa_score_tokens(g["Q"], g["w"], None if dense else dev(heads_np[b:b + 1]),
+                                    g["K"], n - 1, h=h).cpu().numpy()[0, :n]
+        assert np.array_equal(lg1, row), f"seq {b}: decode and prefill logits differ"
+
+
+def test_batched_decode_appends_keys_incrementally(lib):
+    # keys appended one at a time to three sequences: re-pooling only each
+    # sequence's last block keeps the pooled keys equal to pooling from scratch
+    H, d, B, h, k, ps = 16, 64, 32, 4, 32, 16
+    lens0 = [31, 64, 200]
+    steps = 40
+    full = [n + steps for n in lens0]
+    seqs, Qn, wn, pages_n, bts_n = _decode_batch(full, H, d, B, h, k, ps, seed=600)
+    pages, bts = dev(pages_n), dev(bts_n)
+    M_max = -(-bts_n.shape[1] * ps // B)
+    lens = np.array(lens0, dtype=np.int32)
+    _, hl = lib.misa_decode_pool_keys(pages, bts, dev(lens), B, M_max, M_max)
+    for i in range(steps):
+        lens = lens + 1
+        lib.misa_decode_pool_keys(pages, bts, dev(lens), B, M_max, 1, kbar_hl=hl)
+    _, ref = lib.misa_decode_pool_keys(pages, bts, dev(lens), B, M_max, M_max)
+    assert lib.misa_last_device_status() == lib.MISA_OK
+    for b, n in enumerate(lens.tolist()):
+        M = -(-n // B)
+        assert torch.equal(hl[b, :, :M], ref[b, :, :M])

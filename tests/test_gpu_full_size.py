@@ -200,3 +200,49 @@ def test_full_size_fp8_queries_and_keys_sampled_rows():
         assert rec[-1] >= 0.99
     print(f"fp8 q+k chunk: max |gpu - oracle| / sum|w ReLU(q.k)| = {worst:.3e}; "
           f"min recall vs fp64 top-k = {min(rec):.4f}")
+
+
+@pytest.mark.parametrize("ps", [64])
+def test_full_size_paged_chunk(ps):
+    # the 8192 x 131072 chunk with its keys in a paged cache (pages of `ps` keys
+    # spread over a larger pool in a random order): the indices of every row
+    # equal those of the contiguous cache bit for bit, and sampled rows of the
+    # paged scoring pass match the oracle on the keys in logical order
+    from long_context_sparse_block_b200 import _lib
+    from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
+    from tests.test_gpu_paged import make_paged
+    wl = W.WORKLOADS["chunk_128k"]
+    inp = W.generate(wl)
+    rows = _rows(wl)
+    g = inputs_to_device(inp)
+    pk = make_paged(_lib, g["K"], ps, seed=ps)
+    shape = IndexerShape(wl.n_q, wl.q_pos0, wl.n_k, wl.H, wl.d, wl.B, wl.h, wl.k)
+    ix = MisaIndexer(shape)
+    want = ix.run(g["Q"], g["K"], g["w"]).clone()
+    got = ix.run(g["Q"], pk, g["w"]).clone()
+    assert _lib.misa_last_device_status() == 0
+    assert torch.equal(got, want)
+    dumps = {}
+
+    def grab(c0, c1, lg):
+        for t in rows:
+            if c0 <= t < c1:
+                dumps[t] = lg[t - c0].cpu().numpy()
+
+    ix2 = MisaIndexer(IndexerShape(wl.n_q, wl.q_pos0, wl.n_k, wl.H, wl.d, wl.B, wl.h, wl.k,
+                                   sub_chunk=1024))
+    unf = ix2.run(g["Q"], pk, g["w"], on_subchunk=grab).cpu().numpy()
+    assert np.array_equal(unf, got.cpu().numpy())
+    heads = ix2.heads.cpu().numpy()
+    Kd = oracle.bf16_to_f64(inp["K"])
+    sel = np.array(rows)
+    Qd = oracle.bf16_to_f64(inp["Q"][sel])
+    wd = inp["w"][sel].astype(np.float64)
+    for i, t in enumerate(rows):
+        pos = wl.q_pos0 + t
+        hs = heads[t:t + 1]
+        lg_gpu = dumps[t]
+        assert np.array_equal(unf[t], oracle.topk(lg_gpu[None, :], pos, wl.n_k, wl.k)[0])
+        ref = oracle.score(Qd[i:i + 1], wd[i:i + 1], hs, Kd, pos)[0]
+        mag = (np.abs(wd[i, hs[0]])[:, None] * np.maximum(Qd[i, hs[0]] @ Kd[:pos + 1].T, 0)).sum(0)
+        assert_logits_close(lg_gpu, ref[:pos + 1], mag, what=f"paged row {t}")
