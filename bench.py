@@ -448,6 +448,72 @@ def _recall(sel, ref, n_k):
     return hit / max(tot, 1)
 
 
+class DecodeBatch:
+    """A batched decode step: n_seq sequences of the chunk's n_k keys each in one
+    page pool (every sequence its own copy of the chunk's keys, in its own
+    seeded page order), one new query each (rows of the chunk's queries)."""
+
+    def __init__(self, wl, Q, K, w, n_seq: int = 64, ps: int = 64, k_scale=None):
+        """K: bf16 codes [n_k, d], or e4m3 codes (uint8) with k_scale [n_k]."""
+        import torch
+
+        from long_context_sparse_block_b200 import _lib
+        from long_context_sparse_block_b200 import workloads as Wm
+        self.lib, self.wl, self.n_seq = _lib, wl, n_seq
+        nb = wl.n_k // ps
+        table, n_pages = Wm.page_table(n_seq * wl.n_k, ps, seed=65)
+        self.pages = torch.empty((n_pages, ps, wl.d), dtype=K.dtype, device="cuda")
+        self.bts = torch.from_numpy(table.reshape(n_seq, nb).copy()).cuda()
+        self.ks = None
+        if k_scale is not None:
+            self.ks = torch.ones((n_pages, ps), dtype=torch.float32, device="cuda")
+        Kp = K.view(nb, ps, wl.d)
+        for b in range(n_seq):
+            self.pages[self.bts[b].long()] = Kp
+            if self.ks is not None:
+                self.ks[self.bts[b].long()] = k_scale.view(nb, ps)
+        self.lens = torch.full((n_seq,), wl.n_k, dtype=torch.int32, device="cuda")
+        self.Q = Q[-n_seq:].contiguous()
+        self.w = w[-n_seq:].contiguous()
+        self.M_max = -(-wl.n_k // wl.B)
+        _, self.hl = _lib.misa_decode_pool_keys(self.pages, self.bts, self.lens, wl.B, self.M_max,
+                                                self.M_max, k_scale=self.ks)
+        self.heads = torch.empty((n_seq, wl.h), dtype=torch.int32, device="cuda")
+        self.idx = torch.empty((n_seq, wl.k), dtype=torch.int32, device="cuda")
+        self.lg = torch.empty((n_seq, wl.n_k), dtype=torch.float32, device="cuda")
+        self.key_bytes = n_seq * wl.n_k * wl.d * K.element_size()
+        self.step()
+
+    def score_topk(self):
+        self.lib.misa_decode_score_topk(self.Q, self.w, self.heads, self.pages, self.bts,
+                                        self.lens, self.wl.k, idx=self.idx, logits=self.lg,
+                                        k_scale=self.ks)
+
+    def step(self):
+        wl = self.wl
+        self.lib.misa_decode_pool_keys(self.pages, self.bts, self.lens, wl.B, self.M_max, 1,
+                                       kbar_hl=self.hl, k_scale=self.ks)
+        self.lib.misa_decode_route_heads(self.Q, self.w, self.hl, self.lens, wl.B, wl.h,
+                                         heads=self.heads)
+        self.score_topk()
+
+
+def run_decode_part(args):
+    """--part decode: only the batched decode step, for profiling captures."""
+    import torch
+    wl = W.WORKLOADS["chunk_128k"]
+    inp = W.generate(wl)
+
+    def d16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+    dec = DecodeBatch(wl, d16(inp["Q"]), d16(inp["K"]), torch.from_numpy(inp["w"]).cuda())
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    ms = _time_ms(dec.step, torch.cuda.current_stream(), flush, reps=args.steps, warm=args.warmup)
+    return {"part": "decode", "n_seq": dec.n_seq, "n_k": wl.n_k, "h": wl.h, "k": wl.k,
+            "ms_per_step": round(ms, 4), "key_gbs": round(dec.key_bytes / (ms * 1e-3) / 1e9, 1)}
+
+
 def run_variants(wl, inp, stream, flush):
     """The other measured configurations: on the chunk, h=4, the dense 64-head
     indexer in this library, MISA-dagger (k'=8192, all-head rerank to 2048) with
@@ -492,6 +558,26 @@ def run_variants(wl, inp, stream, flush):
     dense_bf = MisaIndexer(IndexerShape(h=wl.H, dense=True, **base))
     out["dagger_fp8_recall_vs_dense_bf16"] = round(_recall(fin8, dense_bf.run(Q, K, w), wl.n_k), 4)
     del dense_bf, dg8, fin8, ref8, K8, ks     # (K8c, sc stay on the host)
+
+    # end to end from pinned host buffers with three piece schedules (the main
+    # e2e figure uses run_host's default, the ramp)
+    from long_context_sparse_block_b200.indexer import ramp_pieces
+    ixh = MisaIndexer(IndexerShape(h=wl.h, **base))
+    Qh = torch.from_numpy(inp["Q"].view(np.int16)).pin_memory()
+    Kh = torch.from_numpy(inp["K"].view(np.int16)).pin_memory()
+    wh = torch.from_numpy(inp["w"]).pin_memory()
+    idx_h = torch.empty((wl.n_q, wl.k), dtype=torch.int32).pin_memory()
+    for label, pcs in (("p4", 4), ("p8", 8), ("ramp", ramp_pieces(wl.n_q))):
+        out[f"e2e_{label}_ms"] = round(_time_ms(lambda: ixh.run_host(Qh, Kh, wh, out=idx_h, pieces=pcs),
+                                                stream, flush), 4)
+    # where the end-to-end time goes: events on the three streams of one run
+    tl = []
+    flush.zero_()
+    ixh.run_host(Qh, Kh, wh, out=idx_h, timeline=tl)
+    torch.cuda.synchronize()
+    t0 = tl[0][1]
+    out["e2e_ramp_timeline_ms"] = {label: round(t0.elapsed_time(ev), 3) for label, ev in tl[1:]}
+    del ixh, Qh, Kh, wh, idx_h
 
     # the same chunk with its keys in a paged cache (pages of 64 keys in a
     # seeded random order in a larger pool, unused rows filled with +inf codes):
@@ -563,44 +649,22 @@ def run_variants(wl, inp, stream, flush):
 
     out["decode_step_ms"] = round(_time_ms(decode_step, stream, flush), 4)
 
-    # batched decode: 64 sequences of 131072 keys each in one page pool (every
-    # sequence its own copy of the chunk's keys in its own seeded page order),
-    # one new query each (rows of the chunk's queries): re-pool each
-    # sequence's last block, route, score and select, three launches plus the
-    # top-k
-    n_seq, ps = 64, 64
-    nb = wl.n_k // ps
-    table, n_pages = Wm.page_table(n_seq * wl.n_k, ps, seed=65)
-    pages = torch.empty((n_pages, ps, wl.d), dtype=torch.int16, device="cuda")
-    bts = torch.from_numpy(table.reshape(n_seq, nb).copy()).cuda()
-    Kp = K.view(nb, ps, wl.d)
-    for b in range(n_seq):
-        pages[bts[b].long()] = Kp
-    del Kp
-    seq_lens = torch.full((n_seq,), wl.n_k, dtype=torch.int32, device="cuda")
-    Qd = Q[-n_seq:].contiguous()
-    wd = w[-n_seq:].contiguous()
-    M_max = -(-wl.n_k // wl.B)
-    _, hl_d = _lib.misa_decode_pool_keys(pages, bts, seq_lens, wl.B, M_max, M_max)
-    heads_d = torch.empty((n_seq, wl.h), dtype=torch.int32, device="cuda")
-    idx_d = torch.empty((n_seq, wl.k), dtype=torch.int32, device="cuda")
-    lg_d = torch.empty((n_seq, wl.n_k), dtype=torch.float32, device="cuda")
-
-    def decode_batch():
-        _lib.misa_decode_pool_keys(pages, bts, seq_lens, wl.B, M_max, 1, kbar_hl=hl_d)
-        _lib.misa_decode_route_heads(Qd, wd, hl_d, seq_lens, wl.B, wl.h, heads=heads_d)
-        _lib.misa_decode_score_topk(Qd, wd, heads_d, pages, bts, seq_lens, wl.k, idx=idx_d,
-                                    logits=lg_d)
-
-    t_db = _time_ms(decode_batch, stream, flush)
-    t_ds = _time_ms(lambda: _lib.misa_decode_score_topk(Qd, wd, heads_d, pages, bts, seq_lens,
-                                                         wl.k, idx=idx_d, logits=lg_d),
-                    stream, flush)
-    key_bytes = n_seq * wl.n_k * wl.d * 2
+    # batched decode: 64 sequences of 131072 keys each in one page pool, one
+    # new query each (re-pool each sequence's last block, route, score, select)
+    dec = DecodeBatch(wl, Q, K, w)
+    t_db = _time_ms(dec.step, stream, flush)
+    t_ds = _time_ms(dec.score_topk, stream, flush)
     out["decode_batch64_ms"] = round(t_db, 4)
     out["decode_batch64_score_topk_ms"] = round(t_ds, 4)
-    out["decode_batch64_key_gbs"] = round(key_bytes / (t_ds * 1e-3) / 1e9, 1)
-    del pages, bts, seq_lens, Qd, wd, hl_d, heads_d, idx_d, lg_d
+    out["decode_batch64_key_gbs"] = round(dec.key_bytes / (t_ds * 1e-3) / 1e9, 1)
+    del dec
+    # the same with the caches in e4m3 (a scale per key): half the bytes
+    dec8 = DecodeBatch(wl, Q, torch.from_numpy(K8c).cuda(), w, k_scale=torch.from_numpy(sc).cuda())
+    t_8 = _time_ms(dec8.score_topk, stream, flush)
+    out["decode_batch64_fp8_ms"] = round(_time_ms(dec8.step, stream, flush), 4)
+    out["decode_batch64_fp8_score_topk_ms"] = round(t_8, 4)
+    out["decode_batch64_fp8_key_gbs"] = round(dec8.key_bytes / (t_8 * 1e-3) / 1e9, 1)
+    del dec8
     del ixu, lg, Q, K, w
 
     # the prefill configurations (whole-sequence prefill, the fused path per
@@ -690,6 +754,8 @@ def main():
                     help="index only the first N queries of the chunk (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
+    ap.add_argument("--part", default="", choices=["", "decode"],
+                    help="run one part alone for profiling captures (decode: the batched step)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the h=4 / dense / MISA-dagger / FP8 measurements")
     args = ap.parse_args()
@@ -698,6 +764,10 @@ def main():
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.part == "decode":
+        print(json.dumps(run_decode_part(args)), flush=True)
+        return
 
     if args.impl == "reference":
         out = run_reference(args, rank)

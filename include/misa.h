@@ -290,8 +290,9 @@ int misa_decode_route_heads(const uint16_t* Q, const float* w, const uint16_t* k
  * keys of largest logit, ties to the lower index, ascending, -1 padded.  A
  * scoring pass shaped for one query per sequence: 128-key tiles against the
  * query's h head rows padded to 16, 32 or 64 MMA columns, so the keys are read
- * once and the MMA stays small.  bf16 pages only (FP8 pages:
- * MISA_ERR_UNSUPPORTED); h a power of two <= 64.  logits [n_seq, ld] fp32
+ * once and the MMA stays small.  bf16 or e4m3 pages (e4m3: decoded exactly to
+ * bf16 in the kernel, the row's scale multiplying the head-sum, as in
+ * misa_score_tokens); h a power of two <= 64.  logits [n_seq, ld] fp32
  * scratch (ld >= max_blocks * page_size; entries s < seq_lens[b] hold the
  * logits afterwards). */
 int misa_decode_score_topk(const uint16_t* Q, const float* w, const int32_t* heads,

@@ -632,14 +632,14 @@ int misa_decode_score_topk(const uint16_t* Q, const float* w, const int32_t* hea
   const int64_t max_len = static_cast<int64_t>(max_blocks) * page_size;
   if (const int st = check_keys(key, max_len)) return st;
   if (ld < max_len) return MISA_ERR_INVALID_ARG;
-  if (key.fp8() || !good_d(d) || !pow2(h) || h > 64) return MISA_ERR_UNSUPPORTED;
+  if (!good_d(d) || !pow2(h) || h > 64) return MISA_ERR_UNSUPPORTED;
   if (n_seq == 0) return MISA_OK;
   DevCtl ctl;
   if (!make_ctl(ctl)) return MISA_ERR_CUDA;
   const cudaStream_t s = as_stream(stream);
-  cudaError_t e = launch_decode_score(Q, w, heads, pages, block_tables, max_blocks,
-                                      key.kpg.page_shift, n_pages, seq_lens, n_seq, H, d, h, logits,
-                                      ld, ctl, s);
+  cudaError_t e = launch_decode_score(Q, w, heads, pages, k_scale, key.fp8(), block_tables,
+                                      max_blocks, key.kpg.page_shift, n_pages, seq_lens, n_seq, H, d,
+                                      h, logits, ld, ctl, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   if (k == 0) return MISA_OK;
   return cuda_status(launch_topk(logits, ld, n_seq, 0, max_len, k, idx, ctl, s, nullptr, seq_lens));

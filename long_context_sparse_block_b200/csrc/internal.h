@@ -38,12 +38,12 @@ cudaError_t launch_pool_keys_batch(const void* pages, const float* k_scale, bool
                                    int64_t n_pages, const int32_t* lens, int n_seq, int d, int B,
                                    int64_t M_max, int64_t n_last, float* kbar, uint16_t* kbar_hl,
                                    const DevCtl& ctl, cudaStream_t s);
-// logits[b, s] for s < lens[b] (bf16 pages).
+// logits[b, s] for s < lens[b] (bf16 pages, or e4m3 pages with per-row scales).
 cudaError_t launch_decode_score(const uint16_t* Q, const float* w, const int32_t* heads,
-                                const void* pages, const int32_t* block_tables, int max_blocks,
-                                int page_shift, int64_t n_pages, const int32_t* lens, int n_seq,
-                                int H, int d, int h, float* logits, int64_t ld, const DevCtl& ctl,
-                                cudaStream_t s);
+                                const void* pages, const float* k_scale, bool fp8,
+                                const int32_t* block_tables, int max_blocks, int page_shift,
+                                int64_t n_pages, const int32_t* lens, int n_seq, int H, int d, int h,
+                                float* logits, int64_t ld, const DevCtl& ctl, cudaStream_t s);
 
 // Score kernel launch description: store mode writes fused logits (logits,
 // ld); select mode (tau != nullptr) keeps logits >= tau[t] in per-row

@@ -500,10 +500,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
     uint32_t accph = 0, tcount = 0;
     int prev_g = -1;
     float* tau_s = reinterpret_cast<float*>(smem + L::OFF_TAU) + e * 16;  // select: thresholds
-    // the per-tile reads of weights and thresholds: shared-space loads with
-    // 32-bit addresses (broadcasts: every lane reads the same word)
-    const uint32_t w_s32 = smem_u32(w_s), tau_s32 = smem_u32(tau_s);
-    (void)tau_s32;
+    (void)tau_s;
     for (; it.left > 0; it.next(p), ++tcount) {
       if (it.g != prev_g) {
         for (int i = lane; i < EC; i += 32) {
@@ -532,49 +529,68 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
       if (lane == 0) ok = mbar_wait(bar(ACCFULL + acc), accph, abort_flag, p.ctl);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
-      constexpr bool SPLIT = EC == 64 && HT >= 4 && HT <= 32;  // no query spans the halves
-      uint32_t v[EC];
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * kCols + part * EC);
       float sums[HT >= 4 ? QPW : 1];
-      auto qsum = [&](int qq) {
+      // w * ReLU head-sum of query qq (of this warp) from its h columns x[0..HT)
+      auto qsum_of = [&](int qq, const uint32_t* x) {
         float2 a2 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int j = 0; j < HT; j += 4) {
-          const float4 w4 = lds_f32x4(w_s32 + static_cast<uint32_t>((qq * HT + j) * 4));
-          const uint32_t* x = v + qq * HT + j;
+          const float4 w4 = *reinterpret_cast<const float4*>(w_s + qq * HT + j);
           a2 = fma2(make_float2(w4.x, w4.y),
-                    make_float2(relu(__uint_as_float(x[0])), relu(__uint_as_float(x[1]))), a2);
+                    make_float2(relu(__uint_as_float(x[j])), relu(__uint_as_float(x[j + 1]))), a2);
           a2 = fma2(make_float2(w4.z, w4.w),
-                    make_float2(relu(__uint_as_float(x[2])), relu(__uint_as_float(x[3]))), a2);
+                    make_float2(relu(__uint_as_float(x[j + 2])), relu(__uint_as_float(x[j + 3]))),
+                    a2);
         }
         return a2.x + a2.y;
       };
-      if constexpr (SPLIT) {
-        // two 32-column halves: the second lands while the first half's
-        // queries are summed
-        uint32_t (&va)[32] = *reinterpret_cast<uint32_t(*)[32]>(v);
-        uint32_t (&vb)[32] = *reinterpret_cast<uint32_t(*)[32]>(v + 32);
-        tmem_ld32(taddr, va);
-        tmem_wait_ld_regs(va);
-        tmem_ld32(taddr + 32, vb);
+      auto release_acc = [&]() {  // the accumulator is in registers: back to the MMA warp
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
+        if (++acc == 2) {
+          acc = 0;
+          accph ^= 1;
+        }
+      };
+      // h <= 32: the warp's 64 columns are read CW at a time (whole queries),
+      // the next load in flight while the current queries are summed; only two
+      // CW-column buffers are live, which leaves registers for the selection
+      constexpr bool CHUNKED = EC == 64 && HT >= 4 && HT <= 32;
+      if constexpr (CHUNKED) {
+        constexpr int CW = HT <= 16 ? 16 : 32;  // columns per TMEM load
+        constexpr int NCH = EC / CW;            // loads per tile
+        constexpr int QPC = CW / HT;            // queries per load
+        uint32_t vb[2][CW];
+        auto ld_cols = [&](uint32_t addr, uint32_t (&r)[CW]) {
+          if constexpr (CW == 16)
+            tmem_ld16(addr, r);
+          else
+            tmem_ld32(addr, r);
+        };
+        ld_cols(taddr, vb[0]);
+        tmem_wait_ld_regs(vb[0]);
 #pragma unroll
-        for (int qq = 0; qq < QPW / 2; ++qq) sums[qq] = qsum(qq);
-        tmem_wait_ld_regs(vb);
-      } else {
+        for (int c = 0; c < NCH; ++c) {
+          if (c + 1 < NCH)
+            ld_cols(taddr + static_cast<uint32_t>((c + 1) * CW), vb[(c + 1) & 1]);
+          else
+            release_acc();
+#pragma unroll
+          for (int q = 0; q < QPC; ++q) sums[c * QPC + q] = qsum_of(c * QPC + q, vb[c & 1] + q * HT);
+          if (c + 1 < NCH) tmem_wait_ld_regs(vb[(c + 1) & 1]);
+        }
+      }
+      uint32_t v[CHUNKED ? 1 : EC];
+      if constexpr (!CHUNKED) {
         if constexpr (EC == 64)
           tmem_ld64(taddr, v);
         else
           tmem_ld128(taddr, v);
         tmem_wait_ld();
-      }
-      // the accumulator is in registers: hand it back to the MMA warp now
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(ACCEMPTY + acc));
-      if (++acc == 2) {
-        acc = 0;
-        accph ^= 1;
+        release_acc();
       }
       const int64_t s = it.kt * kTileKeys + quad * 32 + lane;
       const bool s_ok = s < p.n_k;
@@ -582,8 +598,10 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
       float* dst = p.logits + tq0 * p.ld + s;
       (void)dst;
       if constexpr (HT >= 4) {
+        if constexpr (!CHUNKED) {
 #pragma unroll
-        for (int qq = SPLIT ? QPW / 2 : 0; qq < QPW; ++qq) sums[qq] = qsum(qq);
+          for (int qq = 0; qq < QPW; ++qq) sums[qq] = qsum_of(qq, v + qq * HT);
+        }
         if constexpr (KSC) {
           // per-token scale > 0: w * ReLU(scale * dot) = scale * w * ReLU(dot)
           const float ks = s_ok ? __ldg(p.k_scale + p.kpg.row(s, p.ctl)) : 0.0f;
@@ -604,7 +622,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           if (full) {
 #pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
-              const bool pass = sums[qq] >= lds_f32(tau_s32 + qq * 4);
+              const bool pass = sums[qq] >= tau_s[qq];
               m[qq] = __ballot_sync(0xffffffffu, pass);
               if (pass) *dst = sums[qq];
               dst += p.ld;
@@ -615,7 +633,7 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
             const uint32_t valid = s_ok ? (((1u << q_end) - 1u) & ~((1u << cut) - 1u)) : 0u;
 #pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
-              const bool pass = ((valid >> qq) & 1u) && sums[qq] >= lds_f32(tau_s32 + qq * 4);
+              const bool pass = ((valid >> qq) & 1u) && sums[qq] >= tau_s[qq];
               m[qq] = __ballot_sync(0xffffffffu, pass);
               if (pass) *dst = sums[qq];
               dst += p.ld;

@@ -52,6 +52,35 @@ def _piece_bounds(n: int, pieces: int):
     return [(a, b) for a, b in zip(cuts, cuts[1:]) if b > a]
 
 
+def ramp_pieces(n: int):
+    """A piece schedule that starts and ends small: n/16, n/8, then pieces of
+    n/4 for the middle, and a last piece of n/16, so the first copy-in that
+    nothing overlaps is short, each later piece arrives while the one before it
+    is indexed (indexing a query takes longer than copying it), and the last
+    piece's indexing and copy-out are short."""
+    a, b = max(1, n // 16), max(1, n // 8)
+    if n < 4 * (a + b):
+        return [n]
+    mid = n - 2 * a - b
+    q = max(1, n // 4)
+    sizes = [a, b] + [q] * (mid // q) + ([mid % q] if mid % q else []) + [a]
+    return sizes
+
+
+def _bounds_of(n: int, pieces):
+    """Query ranges of run_host for a piece count or for explicit piece sizes."""
+    if isinstance(pieces, int):
+        return _piece_bounds(n, pieces)
+    out, c0 = [], 0
+    for size in pieces:
+        if size > 0 and c0 < n:
+            out.append((c0, min(n, c0 + size)))
+            c0 += size
+    if c0 < n:
+        out.append((c0, n))
+    return out
+
+
 class MisaIndexer:
     def __init__(self, shape: IndexerShape, device="cuda"):
         s = self.shape = shape
@@ -110,14 +139,17 @@ class MisaIndexer:
                                  k_scale=k_scale, idx=self.final[c0:c1], ws=self.ws)
         return self.final
 
-    def run_host(self, Qh, Kh, wh, out=None, k_scale_h=None, pieces: int = 4):
+    def run_host(self, Qh, Kh, wh, out=None, k_scale_h=None, pieces=None, timeline=None):
         """End to end from host buffers (pin them for asynchronous copies): Q, K, w
         (and FP8 key scales) as in run(); returns the selected indices in `out`, a
         pinned host int32 [n_q, k] tensor (allocated when None), complete when the
-        current stream reaches this point.  The queries go in `pieces` pieces on
-        three streams (copy in, index, copy out) so that the copies of one piece
-        overlap the indexing of another; the keys go first, and the first and
-        last pieces are small."""
+        current stream reaches this point.  The queries go in pieces on three
+        streams (copy in, index, copy out) so that the copies of one piece
+        overlap the indexing of another; the keys go first.  `pieces`: a list of
+        piece sizes (default ramp_pieces(n_q)) or a piece count (the first and
+        last pieces small, see _piece_bounds).  `timeline` (a list, diagnostic):
+        receives (label, timing event) pairs recorded at the start, after each
+        copy in, after each piece is indexed and after each copy out."""
         s = self.shape
         dev = self.heads.device
         if getattr(self, "_dev", None) is None:
@@ -132,9 +164,17 @@ class MisaIndexer:
         if out is None:
             out = torch.empty(tuple(self.final.shape), dtype=torch.int32, pin_memory=True)
         compute = torch.cuda.current_stream(dev)
+
+        def mark(label, stream):
+            if timeline is not None:
+                ev = torch.cuda.Event(enable_timing=True)
+                ev.record(stream)
+                timeline.append((label, ev))
+
+        mark("start", compute)
         cin.wait_stream(compute)   # the device buffers are free again
         cout.wait_stream(compute)
-        bounds = _piece_bounds(s.n_q, pieces)
+        bounds = _bounds_of(s.n_q, ramp_pieces(s.n_q) if pieces is None else pieces)
         ev_in = []
         with torch.cuda.stream(cin):
             K.copy_(Kh, non_blocking=True)
@@ -142,16 +182,18 @@ class MisaIndexer:
                 ks.copy_(k_scale_h, non_blocking=True)
             ev_k = torch.cuda.Event()
             ev_k.record(cin)
-            for c0, c1 in bounds:
+            mark("keys in", cin)
+            for i, (c0, c1) in enumerate(bounds):
                 Q[c0:c1].copy_(Qh[c0:c1], non_blocking=True)
                 w[c0:c1].copy_(wh[c0:c1], non_blocking=True)
                 e = torch.cuda.Event()
                 e.record(cin)
                 ev_in.append(e)
+                mark(f"piece {i} in", cin)
         compute.wait_event(ev_k)
         if not s.dense:
             _lib.misa_pool_keys(K, s.B, k_scale=ks, kbar_hl=self.kbar_hl, want_kbar=False)
-        for (c0, c1), e in zip(bounds, ev_in):
+        for i, ((c0, c1), e) in enumerate(zip(bounds, ev_in)):
             compute.wait_event(e)
             if not s.dense:
                 _lib.misa_route_heads(Q[c0:c1], w[c0:c1], self.kbar_hl, s.q_pos0 + c0, s.n_k,
@@ -160,8 +202,10 @@ class MisaIndexer:
                 self._select(a0, min(c1, a0 + self.sub), Q, K, w, ks)
             done = torch.cuda.Event()
             done.record(compute)
+            mark(f"piece {i} indexed", compute)
             cout.wait_event(done)
             with torch.cuda.stream(cout):
                 out[c0:c1].copy_(self.final[c0:c1], non_blocking=True)
+            mark(f"piece {i} out", cout)
         compute.wait_stream(cout)
         return out

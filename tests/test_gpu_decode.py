@@ -84,52 +84,65 @@ def test_decode_step_matches_oracle(lib):
 
 # ------------------------------------------------------------------ batched decode
 
-def _decode_batch(lens, H, d, B, h, k, ps, seed):
+def _decode_batch(lens, H, d, B, h, k, ps, seed, fp8=False):
     """One new query per sequence at the end of its own keys; all keys in one
-    page pool (pages of ps keys in a seeded random order, unused rows +inf)."""
+    page pool (pages of ps keys in a seeded random order, unused rows +inf, or
+    NaN codes and scales for e4m3 pages).  Returns (seqs, Q, w, pages, bts,
+    scales)."""
     seqs = []
     for b, n in enumerate(lens):
         wl = W.small_workload(f"dec{seed}_{b}", n_q=1, q_pos0=n - 1, n_k=n, H=H, d=d, B=B, h=h,
                               k=k, seed=seed + b, generator="clustered")
-        seqs.append(W.generate(wl))
+        seqs.append(W.generate(wl, fp8_keys=fp8))
     nb = [-(-n // ps) for n in lens]
     max_blocks = max(nb)
     table, n_pages = W.page_table(sum(nb) * ps, ps, seed=seed)
-    pages = np.full((n_pages, ps, d), 0x7F80, dtype=np.uint16)
+    code, fill = (np.uint8, 0x7F) if fp8 else (np.uint16, 0x7F80)
+    pages = np.full((n_pages, ps, d), fill, dtype=code)
+    scales = np.full((n_pages, ps), np.nan, dtype=np.float32) if fp8 else None
     bts = np.full((len(lens), max_blocks), -1, dtype=np.int32)
     o = 0
     for b, n in enumerate(lens):
-        flat = np.full((nb[b] * ps, d), 0x7F80, dtype=np.uint16)
-        flat[:n] = seqs[b]["K"]
+        flat = np.full((nb[b] * ps, d), fill, dtype=code)
+        flat[:n] = seqs[b]["K8" if fp8 else "K"]
         bts[b, :nb[b]] = table[o:o + nb[b]]
         pages[table[o:o + nb[b]]] = flat.reshape(nb[b], ps, d)
+        if fp8:
+            sflat = np.full(nb[b] * ps, np.nan, dtype=np.float32)
+            sflat[:n] = seqs[b]["k_scale"]
+            scales[table[o:o + nb[b]]] = sflat.reshape(nb[b], ps)
         o += nb[b]
     Q = np.concatenate([s["Q"] for s in seqs])
     w = np.concatenate([s["w"] for s in seqs])
-    return seqs, Q, w, pages, bts
+    return seqs, Q, w, pages, bts, scales
 
 
-@pytest.mark.parametrize("H,d,h,ps", [(64, 128, 8, 64), (64, 128, 64, 32), (32, 64, 4, 128)])
-def test_batched_decode_matches_oracle(lib, H, d, h, ps):
+@pytest.mark.parametrize("H,d,h,ps,fp8", [(64, 128, 8, 64, False), (64, 128, 64, 32, False),
+                                          (32, 64, 4, 128, False), (64, 128, 8, 64, True),
+                                          (16, 32, 16, 16, True)])
+def test_batched_decode_matches_oracle(lib, H, d, h, ps, fp8):
     lens = [1, 100, 128, 3000, 7777, 20000]
     B, k = 128, 256
-    seqs, Qn, wn, pages_n, bts_n = _decode_batch(lens, H, d, B, h, k, ps, seed=500 + h)
+    seqs, Qn, wn, pages_n, bts_n, sc_n = _decode_batch(lens, H, d, B, h, k, ps, seed=500 + h,
+                                                       fp8=fp8)
     Q, w, pages, bts = dev(Qn), dev(wn), dev(pages_n), dev(bts_n)
+    ks = dev(sc_n) if fp8 else None
     seq_lens = dev(np.array(lens, dtype=np.int32))
     M_max = -(-bts_n.shape[1] * ps // B)
-    _, hl = lib.misa_decode_pool_keys(pages, bts, seq_lens, B, M_max, M_max)
+    _, hl = lib.misa_decode_pool_keys(pages, bts, seq_lens, B, M_max, M_max, k_scale=ks)
     dense = h == H
     heads, r = lib.misa_decode_route_heads(Q, w, hl, seq_lens, B, h, want_r=True)
     idx, logits = lib.misa_decode_score_topk(Q, w, None if dense else heads, pages, bts, seq_lens,
-                                             k, h=h)
+                                             k, h=h, k_scale=ks)
     assert lib.misa_last_device_status() == lib.MISA_OK
     hl_np, heads_np, r_np = hl.cpu().numpy(), heads.cpu().numpy(), r.cpu().numpy()
     idx_np, lg_np = idx.cpu().numpy(), logits.cpu().numpy()
     for b, n in enumerate(lens):
-        g = inputs_to_device(seqs[b])
+        g = inputs_to_device(seqs[b], fp8=fp8)
+        Kb, ksb = (g["K8"], g["k_scale"]) if fp8 else (g["K"], None)
         M = -(-n // B)
         # pooling and routing equal the single-sequence calls bit for bit
-        _, hl1 = lib.misa_pool_keys(g["K"], B)
+        _, hl1 = lib.misa_pool_keys(Kb, B, k_scale=ksb)
         hl1 = hl1.cpu().numpy()
         assert np.array_equal(hl_np[b, 0, :M], hl1[0]) and np.array_equal(hl_np[b, 1, :M], hl1[1])
         heads1, r1 = lib.misa_route_heads(g["Q"], g["w"], dev(hl1.view(np.int16)), n - 1, n, B, h,
@@ -137,7 +150,7 @@ def test_batched_decode_matches_oracle(lib, H, d, h, ps):
         assert np.array_equal(r_np[b], r1.cpu().numpy()[0])
         assert np.array_equal(heads_np[b], heads1.cpu().numpy()[0])
         # against the oracle
-        Qd, Kd, wd = oracle.decode_inputs(seqs[b])
+        Qd, Kd, wd = oracle.decode_inputs(seqs[b], fp8_keys=fp8)
         kb = oracle.pool_keys(Kd, B)
         r_o, h_o = oracle.route(Qd, wd, kb, n - 1, n, B, h)
         check_heads(heads_np[b:b + 1], r_o, h_o, h, r_gpu=r_np[b:b + 1])
@@ -150,7 +163,7 @@ def test_batched_decode_matches_oracle(lib, H, d, h, ps):
         assert recall(idx_np[b:b + 1], oracle.topk(ref[None, :], n - 1, n, k)) >= 0.999
         # and the prefill scoring kernel on the same query gives the same logits
         lg1 = lib.misa_score_tokens(g["Q"], g["w"], None if dense else dev(heads_np[b:b + 1]),
-                                    g["K"], n - 1, h=h).cpu().numpy()[0, :n]
+                                    Kb, n - 1, k_scale=ksb, h=h).cpu().numpy()[0, :n]
         assert np.array_equal(lg1, row), f"seq {b}: decode and prefill logits differ"
 
 
@@ -161,7 +174,7 @@ def test_batched_decode_appends_keys_incrementally(lib):
     lens0 = [31, 64, 200]
     steps = 40
     full = [n + steps for n in lens0]
-    seqs, Qn, wn, pages_n, bts_n = _decode_batch(full, H, d, B, h, k, ps, seed=600)
+    seqs, Qn, wn, pages_n, bts_n, _ = _decode_batch(full, H, d, B, h, k, ps, seed=600)
     pages, bts = dev(pages_n), dev(bts_n)
     M_max = -(-bts_n.shape[1] * ps // B)
     lens = np.array(lens0, dtype=np.int32)

@@ -177,7 +177,7 @@ def test_indexer_host_pipeline_equals_device_run(lib, kp):
     Qh = torch.from_numpy(np.ascontiguousarray(inp["Q"]).view(np.int16)).pin_memory()
     Kh = torch.from_numpy(np.ascontiguousarray(inp["K"]).view(np.int16)).pin_memory()
     wh = torch.from_numpy(inp["w"]).pin_memory()
-    for pieces in (1, 3, 4):
+    for pieces in (None, 1, 3, 4):
         out = ix.run_host(Qh, Kh, wh, pieces=pieces)
         torch.cuda.current_stream().synchronize()
         assert np.array_equal(out.numpy(), want)

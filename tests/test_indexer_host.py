@@ -118,3 +118,15 @@ def test_unfused_sequence_hands_each_subchunk_to_the_callback(fake):
         assert b[1] == s.q_pos0 + c0 and b[2] == s.n_k and b[3] == s.k
         assert _rows(kw2["idx"], ix.sel) == (c0, c1)
     assert not fake.named("misa_score_topk")
+
+
+def test_piece_schedules_cover_the_queries_once():
+    from long_context_sparse_block_b200.indexer import _bounds_of, ramp_pieces
+    for n in (1, 7, 100, 1000, 8192, 12345):
+        for pieces in (1, 3, 4, 8, ramp_pieces(n), [n // 2, n], [5, 0, 3]):
+            b = _bounds_of(n, pieces)
+            assert b[0][0] == 0 and b[-1][1] == n
+            assert all(c1 > c0 for c0, c1 in b)
+            assert all(b[i][1] == b[i + 1][0] for i in range(len(b) - 1))
+    r = ramp_pieces(8192)
+    assert sum(r) == 8192 and r[0] == 512 and r[-1] == 512 and max(r) == 2048
