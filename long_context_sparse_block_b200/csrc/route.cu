@@ -16,13 +16,16 @@
 // own row's causal columns, then the 4 epilogue warps exchange r through shared
 // memory and one warp per query runs the top-h as h rounds of a warp argmax.
 //
-// Warp roles (256 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
-// issuer, warps 2-5 epilogue (one per TMEM lane quadrant: one tcgen05.ld of
-// the 128 block columns per tile, the accumulator handed back right after it
-// lands), warps 6-7 top-h selection.  The epilogue hands each row tile's
+// Work unit: NA consecutive 128-row tiles contracted against the same stream
+// of pooled-key tiles (prefill: NA = 2, so each hi/lo tile pair read from L2
+// feeds 256 rows; decode: NA = 1, each query has pooled keys of its own).
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer, then
+// 4 * NA epilogue warps (one per TMEM lane quadrant and row tile: one
+// tcgen05.ld of the 128 block columns per tile, the accumulator handed back
+// right after it lands), then 2 top-h warps.  The epilogue hands each unit's
 // partial sums to the top-h warps through a double-buffered shared array, so
-// the (latency-bound) selection of one row tile overlaps the contraction of
-// the next.  Pooled-key tiles stream through a 3-stage ring.  Row tiles are
+// the (latency-bound) selection of one unit overlaps the contraction of the
+// next.  Pooled-key tiles stream through a 2- or 3-stage ring.  Units are
 // distributed round-robin over a persistent grid.
 #include "internal.h"
 
@@ -31,13 +34,20 @@ namespace {
 
 constexpr int kRows = 128;    // MMA M: (query, head) rows per tile
 constexpr int kBlkN = 128;    // MMA N: pooled blocks per tile
-constexpr int kRouteEpiWarps = 4;
 constexpr int kRouteTopWarps = 2;
-constexpr int kRouteThreads = 64 + 32 * (kRouteEpiWarps + kRouteTopWarps);
-constexpr int kRouteStages = 3;
 constexpr uint64_t kDrainNs = 2000000;
+constexpr int kMaxDynSmem = 232448;  // per block (227 KB)
 
-template <int D>
+// NA = row tiles a CTA contracts against each pooled-key tile (prefill: 2, so
+// each pooled-key tile read from L2 serves 256 (query, head) rows; decode: 1,
+// every query has pooled keys of its own).  Four epilogue warps per row tile.
+template <int NA>
+struct RouteRoles {
+  static constexpr int EPI = 4 * NA;
+  static constexpr int THREADS = 64 + 32 * (EPI + kRouteTopWarps);
+};
+
+template <int D, int NA>
 struct RouteLayout {
   static constexpr int ROWB = D >= 64 ? 128 : 64;
   static constexpr int KCH = D * 2 / ROWB;
@@ -45,14 +55,19 @@ struct RouteLayout {
   static constexpr int A_BYTES = kRows * D * 2;
   static constexpr int B_CHUNK = kBlkN * ROWB;
   static constexpr int B_HALF = kBlkN * D * 2;           // hi or lo tile
+  static constexpr int R_BYTES = 2 * NA * kRows * 4;     // [2 buf][NA * kRows] block sums
+  static constexpr int STAGES_FIT = (kMaxDynSmem - 1024 - 512 - R_BYTES - NA * A_BYTES) / (2 * B_HALF);
+  static constexpr int STAGES = STAGES_FIT < 3 ? STAGES_FIT : 3;
+  static_assert(STAGES >= 2, "pooled-key ring needs two stages");
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + A_BYTES;
-  static constexpr int OFF_R = OFF_B + kRouteStages * 2 * B_HALF;  // [2 buf][kRows] block sums
-  static constexpr int OFF_BAR = OFF_R + 2 * kRows * 4;
-  static constexpr int NBAR = 2 * kRouteStages + 10;
+  static constexpr int OFF_B = OFF_A + NA * A_BYTES;
+  static constexpr int OFF_R = OFF_B + STAGES * 2 * B_HALF;
+  static constexpr int OFF_BAR = OFF_R + R_BYTES;
+  static constexpr int NBAR = 2 * STAGES + 10;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
+  static_assert(ALLOC <= kMaxDynSmem, "shared memory");
 };
 
 struct RouteParams {
@@ -108,11 +123,16 @@ __device__ __forceinline__ void better(float& br, int& bj, float r, int j) {
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(kRouteThreads, 1)
+template <int D, int NA>
+__global__ void __launch_bounds__(RouteRoles<NA>::THREADS, 1)
 route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
                    const __grid_constant__ CUtensorMap kbmap, const RouteParams p, int64_t M) {
-  using L = RouteLayout<D>;
+  using L = RouteLayout<D, NA>;
+  constexpr int EPI = RouteRoles<NA>::EPI;
+  constexpr int kRouteStages = L::STAGES;
+  constexpr int TM_COLS = 2 * NA * kBlkN;  // two accumulators per row tile
+  // work unit: NA consecutive row tiles (the last unit may hold fewer)
+  const int units = (p.row_tiles + NA - 1) / NA;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const uint32_t sA = smem_u32(smem + L::OFF_A);
@@ -135,10 +155,10 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
     mbar_init(bar(AEMPTY), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(ACCFULL + i), 1);
-      mbar_init(bar(ACCEMPTY + i), kRouteEpiWarps);
+      mbar_init(bar(ACCEMPTY + i), EPI);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(RFULL + i), kRouteEpiWarps);
+      mbar_init(bar(RFULL + i), EPI);
       mbar_init(bar(REMPTY + i), kRouteTopWarps);
     }
     *abort_flag = 0;
@@ -147,7 +167,7 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
     tma_prefetch_desc(&kbmap);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_alloc(smem_u32(tmem_slot), TM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -160,8 +180,9 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
     int stage = 0;
     uint32_t phase = 0, tcount = 0;
     bool ok = true;
-    for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x) {
-      const int nN = ntiles_of(p, rt, M);
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const int rt = u * NA, na = min(NA, p.row_tiles - rt);
+      const int nN = ntiles_of(p, rt + na - 1, M);  // the unit's last row tile sees the most
       if (nN == 0) continue;
       // decode: the tile's rows start at query rt's first head row, and its
       // pooled keys are slices 2rt (hi) and 2rt+1 (lo)
@@ -170,9 +191,11 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
       if (lane == 0) {
         ok = mbar_wait(bar(AEMPTY), (tcount & 1) ^ 1, abort_flag, p.ctl);
         if (ok) {
-          mbar_arrive_expect_tx(bar(AFULL), L::A_BYTES);
-          for (int c = 0; c < L::KCH; ++c)
-            tma_load_2d(sA + c * L::A_CHUNK, &qmap, bar(AFULL), c * (L::ROWB / 2), row0);
+          mbar_arrive_expect_tx(bar(AFULL), na * L::A_BYTES);
+          for (int a = 0; a < na; ++a)
+            for (int c = 0; c < L::KCH; ++c)
+              tma_load_2d(sA + a * L::A_BYTES + c * L::A_CHUNK, &qmap, bar(AFULL), c * (L::ROWB / 2),
+                          row0 + a * kRows);
         }
         for (int nb = 0; nb < nN && ok; ++nb) {
           ok = mbar_wait(bar(EMPTY + stage), phase ^ 1, abort_flag, p.ctl);
@@ -200,8 +223,9 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
     uint32_t phase = 0, accph = 0, tcount = 0;
     bool ok = true;
     constexpr uint32_t idesc = umma_idesc_bf16_f32(kRows, kBlkN);
-    for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x) {
-      const int nN = ntiles_of(p, rt, M);
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const int rt = u * NA, na = min(NA, p.row_tiles - rt);
+      const int nN = ntiles_of(p, rt + na - 1, M);
       if (nN == 0) continue;
       if (lane == 0) {
         ok = mbar_wait(bar(AFULL), tcount & 1, abort_flag, p.ctl);
@@ -210,16 +234,19 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
                mbar_wait(bar(ACCEMPTY + acc), accph ^ 1, abort_flag, p.ctl);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBlkN);
           const uint32_t bstage = sB + stage * 2 * L::B_HALF;
-          for (int half = 0; half < 2; ++half) {
+          for (int a = 0; a < na; ++a) {
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((acc * NA + a) * kBlkN);
+            for (int half = 0; half < 2; ++half) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const int c = (kk * 32) / L::ROWB, within = (kk * 32) % L::ROWB;
-              const uint64_t ad = umma_desc_kmajor(sA + c * L::A_CHUNK + within, L::ROWB);
-              const uint64_t bd =
-                  umma_desc_kmajor(bstage + half * L::B_HALF + c * L::B_CHUNK + within, L::ROWB);
-              tc_mma_bf16(d_tmem, ad, bd, idesc, (half > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const int c = (kk * 32) / L::ROWB, within = (kk * 32) % L::ROWB;
+                const uint64_t ad =
+                    umma_desc_kmajor(sA + a * L::A_BYTES + c * L::A_CHUNK + within, L::ROWB);
+                const uint64_t bd =
+                    umma_desc_kmajor(bstage + half * L::B_HALF + c * L::B_CHUNK + within, L::ROWB);
+                tc_mma_bf16(d_tmem, ad, bd, idesc, (half > 0 || kk > 0) ? 1u : 0u);
+              }
             }
           }
           tc_commit(bar(EMPTY + stage));
@@ -244,19 +271,22 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
     }
   } else {
     // ------------------------------------------------------------ epilogue / top-h
-    const bool top_role = warp >= 2 + kRouteEpiWarps;
+    const bool top_role = warp >= 2 + EPI;
     const int QT = queries_per_tile(p);
-    uint32_t rcount = 0;  // row tiles handed over so far (buffer = rcount & 1)
+    uint32_t rcount = 0;  // units handed over so far (buffer = rcount & 1)
     bool ok = true;
     if (!top_role) {
       const int quad = warp & 3;
+      const int a = (warp - 2) / 4;       // row tile of the unit
       const int row = quad * 32 + lane;   // TMEM lane of this thread
       int acc = 0;
       uint32_t accph = 0;
-      for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x, ++rcount) {
-        const int nN = ntiles_of(p, rt, M);
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++rcount) {
+        const int rt0 = u * NA, na = min(NA, p.row_tiles - rt0);
+        const int nN = ntiles_of(p, rt0 + na - 1, M);
+        const int rt = rt0 + a;
         const int t = rt * QT + row / p.H;
-        const bool valid = t < p.n_q && row / p.H < QT;
+        const bool valid = a < na && t < p.n_q && row / p.H < QT;
         const int64_t nc = valid ? query_blocks(p, t, M) : 0;
         float sum = 0.0f;
         for (int nb = 0; nb < nN; ++nb) {
@@ -266,7 +296,7 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
           tc_fence_after();
           uint32_t v[kBlkN];
           tmem_ld128(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                         static_cast<uint32_t>(acc * kBlkN),
+                         static_cast<uint32_t>((acc * NA + a) * kBlkN),
                      v);
           tmem_wait_ld();
           tc_fence_before();
@@ -299,21 +329,22 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
         if (lane == 0) ok = mbar_wait(bar(REMPTY + buf), ((rcount >> 1) & 1) ^ 1, abort_flag, p.ctl);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        r_s[buf * kRows + row] = sum;
+        r_s[buf * NA * kRows + a * kRows + row] = sum;
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(RFULL + buf));
       }
     } else {
       // top-h: one warp per query, h rounds of a warp argmax by (r desc, head asc)
-      const int tw = warp - 2 - kRouteEpiWarps;
-      for (int rt = blockIdx.x; rt < p.row_tiles && ok; rt += gridDim.x, ++rcount) {
+      const int tw = warp - 2 - EPI;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++rcount) {
         const uint32_t buf = rcount & 1;
         if (lane == 0) ok = mbar_wait(bar(RFULL + buf), (rcount >> 1) & 1, abort_flag, p.ctl);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        const float* rb = r_s + buf * kRows;
-        for (int qq = tw; qq < QT; qq += kRouteTopWarps) {
-          const int tq = rt * QT + qq;
+        const float* rb = r_s + buf * NA * kRows;
+        const int rt0 = u * NA, na = min(NA, p.row_tiles - rt0);
+        for (int qq = tw; qq < na * QT; qq += kRouteTopWarps) {
+          const int tq = rt0 * QT + qq;
           if (tq >= p.n_q) break;
           constexpr int SL = 4;  // slots per lane: H <= 128
           float rv[SL];
@@ -365,21 +396,30 @@ route_heads_kernel(const __grid_constant__ CUtensorMap qmap,
   if (*abort_flag) drain_pause(kDrainNs);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 256);
+    tmem_dealloc(tmem_base, TM_COLS);
   }
 }
 
+template <int D, int NA>
+cudaError_t launch_dn(const RouteParams& p, const CUtensorMap& qm, const CUtensorMap& km,
+                      int64_t M, cudaStream_t s) {
+  using L = RouteLayout<D, NA>;
+  auto kern = route_heads_kernel<D, NA>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(sm_count(), (p.row_tiles + NA - 1) / NA);
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, RouteRoles<NA>::THREADS, L::ALLOC, s>>>(qm, km, p, M);
+  return cudaGetLastError();
+}
+
+// Prefill: two row tiles per pooled-key tile once there are enough of them to
+// keep every SM busy; decode: one (each query has its own pooled keys).
 template <int D>
 cudaError_t launch_d(const RouteParams& p, const CUtensorMap& qm, const CUtensorMap& km, int64_t M,
                      cudaStream_t s) {
-  using L = RouteLayout<D>;
-  auto kern = route_heads_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
-  if (e != cudaSuccess) return e;
-  const int grid = std::min(sm_count(), p.row_tiles);
-  if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kRouteThreads, L::ALLOC, s>>>(qm, km, p, M);
-  return cudaGetLastError();
+  if (!p.lens && p.row_tiles >= 2 * sm_count()) return launch_dn<D, 2>(p, qm, km, M, s);
+  return launch_dn<D, 1>(p, qm, km, M, s);
 }
 
 // Tensor maps and launch: Q as [n_q * H, d] rows; the pooled keys as [slices,
