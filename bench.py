@@ -10,8 +10,9 @@ heads and select the top-2048 tokens per query (one fused call: sampled per-row
 thresholds, tensor-core scoring with the ReLU * w head-sum and threshold test in
 the epilogue, exact selection among the kept logits).  Inputs are seeded synthetic arrays
 of the chunk's shape (clustered keys, head-specific query mixtures), resident in
-HBM when the timed region starts.  L2 is flushed (a 256 MiB write) before every
-timed step; all times are CUDA events on the launching stream.
+HBM when the timed region starts.  L2 is flushed before every timed step (a
+256 MiB write, then a 256 MiB read of another buffer, so no input and no dirty
+line is left in it); all times are CUDA events on the launching stream.
 
 N > 1 (torchrun, one process per GPU): every rank indexes its own chunk
 (independent problems, no data-path collective), timing is the max over ranks
@@ -55,6 +56,21 @@ def _peaks():
 
 
 # ------------------------------------------------------------------ clocks
+
+class L2Flush:
+    """Empties L2 between timed steps: a 256 MiB write (evicts every input line),
+    then a 256 MiB read of a second buffer, which writes the first one's dirty
+    lines back before the timed region instead of inside it."""
+
+    def __init__(self):
+        import torch
+        self.w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        self.r = torch.zeros(32 * 1024 * 1024, dtype=torch.int64, device="cuda")
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.max()
+
 
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
@@ -253,7 +269,7 @@ def run_ours(args, rank, world, local_rank, inp):
                          sub_chunk=args.sub_chunk)
     ix = MisaIndexer(shape)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
 
     # per-stage events: pool and route from torch events around their calls;
     # the stages inside the fused score + top-k call from the library's own
@@ -287,7 +303,7 @@ def run_ours(args, rank, world, local_rank, inp):
     fused = _lib.misa_workspace_size("score_topk", ix.sub, wl.n_k, wl.k, 0) > 0
     launches_per_step = 2 + (7 if fused else 2) * math.ceil(wl.n_q / ix.sub)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step(False)
     clocks = ClockSampler(local_rank)
     if rank == 0:
@@ -301,7 +317,7 @@ def run_ours(args, rank, world, local_rank, inp):
     _lib.misa_profile_start()
     spans = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush()
         spans.append(step(True))
     torch.cuda.synchronize()
     if world > 1:
@@ -336,7 +352,7 @@ def run_ours(args, rank, world, local_rank, inp):
     idx_h = torch.empty(ix.final.shape, dtype=torch.int32).pin_memory()
     e2e_ms = []
     for i in range(0 if args.no_e2e else args.warmup + args.steps):
-        flush.zero_()
+        flush()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -382,7 +398,7 @@ def run_ours(args, rank, world, local_rank, inp):
             "query_sub_chunk": ix.sub,
             "fused_score_topk": fused,
             "rows_repaired_last_subchunk": repaired,
-            "l2": "flushed by a 256 MiB write before every timed step",
+            "l2": "flushed before every timed step: a 256 MiB write, then a 256 MiB read of another buffer (no input and no dirty line left in L2)",
             "parallelism": f"independent chunks per rank x{world}",
         },
         "roofline": {
@@ -422,7 +438,7 @@ def _time_ms(fn, stream, flush, reps=5, warm=2):
     import torch
     ts = []
     for i in range(warm + reps):
-        flush.zero_()
+        flush()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -508,10 +524,36 @@ def run_decode_part(args):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
 
     dec = DecodeBatch(wl, d16(inp["Q"]), d16(inp["K"]), torch.from_numpy(inp["w"]).cuda())
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     ms = _time_ms(dec.step, torch.cuda.current_stream(), flush, reps=args.steps, warm=args.warmup)
     return {"part": "decode", "n_seq": dec.n_seq, "n_k": wl.n_k, "h": wl.h, "k": wl.k,
             "ms_per_step": round(ms, 4), "key_gbs": round(dec.key_bytes / (ms * 1e-3) / 1e9, 1)}
+
+
+def run_topk_part(args):
+    """--part topk: only the standalone top-k over the chunk's fused logits (the
+    unfused path's selection), for profiling captures; --queries cuts the rows."""
+    import torch
+    from long_context_sparse_block_b200 import _lib
+    wl = _workload(args)
+    inp = W.generate(wl)
+
+    def d16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+    Q, K, w = d16(inp["Q"]), d16(inp["K"]), torch.from_numpy(inp["w"]).cuda()
+    _, hl = _lib.misa_pool_keys(K, wl.B)
+    heads, _ = _lib.misa_route_heads(Q, w, hl, wl.q_pos0, wl.n_k, wl.B, wl.h)
+    lg = _lib.misa_score_tokens(Q, w, heads, K, wl.q_pos0)
+    del Q
+    idx = torch.empty((wl.n_q, wl.k), dtype=torch.int32, device="cuda")
+    ms = _time_ms(lambda: _lib.misa_topk(lg, wl.q_pos0, wl.n_k, wl.k, idx=idx),
+                  torch.cuda.current_stream(), L2Flush(), reps=args.steps, warm=args.warmup)
+    # bytes: every visible logit of every row, read once
+    n_vis = sum(min(wl.q_pos0 + t + 1, wl.n_k) for t in range(wl.n_q))
+    gbs = n_vis * 4 / (ms * 1e-3) / 1e9
+    return {"part": "topk", "n_q": wl.n_q, "n_k": wl.n_k, "k": wl.k, "ms_per_step": round(ms, 4),
+            "logit_gbs": round(gbs, 1), "hbm_frac": round(gbs / _peaks()["hbm_gbs"], 3)}
 
 
 def run_variants(wl, inp, stream, flush):
@@ -572,7 +614,7 @@ def run_variants(wl, inp, stream, flush):
                                                 stream, flush), 4)
     # where the end-to-end time goes: events on the three streams of one run
     tl = []
-    flush.zero_()
+    flush()
     ixh.run_host(Qh, Kh, wh, out=idx_h, timeline=tl)
     torch.cuda.synchronize()
     t0 = tl[0][1]
@@ -754,7 +796,7 @@ def main():
                     help="index only the first N queries of the chunk (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
-    ap.add_argument("--part", default="", choices=["", "decode"],
+    ap.add_argument("--part", default="", choices=["", "decode", "topk"],
                     help="run one part alone for profiling captures (decode: the batched step)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the h=4 / dense / MISA-dagger / FP8 measurements")
@@ -765,6 +807,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
 
+    if args.part == "topk":
+        print(json.dumps(run_topk_part(args)), flush=True)
+        return
     if args.part == "decode":
         print(json.dumps(run_decode_part(args)), flush=True)
         return

@@ -143,19 +143,6 @@ pool_keys_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_scal
 }
 
 template <int D, bool FP8>
-cudaError_t launch(const void* K, const float* k_scale, const KeyPages& kpg, int64_t n_k, int B,
-                   int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl, const DevCtl& ctl,
-                   cudaStream_t s) {
-  const int64_t M = (n_k + B - 1) / B;
-  if (m1 > M) m1 = M;
-  if (m1 <= m0) return cudaSuccess;
-  pool_keys_kernel<D, FP8><<<static_cast<unsigned>(m1 - m0), kPoolThreads, 0, s>>>(
-      static_cast<const uint8_t*>(K), k_scale, kpg, n_k, B, M, m0, kbar, kbar_hl, ctl,
-      PoolBatch{nullptr, 0, nullptr, 0, 0});
-  return cudaGetLastError();
-}
-
-template <int D, bool FP8>
 cudaError_t launch_batch(const void* K, const float* k_scale, const KeyPages& kpg, int B,
                          const PoolBatch& batch, int n_seq, float* kbar, uint16_t* kbar_hl,
                          const DevCtl& ctl, cudaStream_t s) {
@@ -163,6 +150,136 @@ cudaError_t launch_batch(const void* K, const float* k_scale, const KeyPages& kp
   pool_keys_kernel<D, FP8><<<grid, kPoolThreads, 0, s>>>(static_cast<const uint8_t*>(K), k_scale,
                                                         kpg, 0, B, batch.M_max, 0, kbar, kbar_hl,
                                                         ctl, batch);
+  return cudaGetLastError();
+}
+
+// Large ranges of bf16 keys: one persistent CTA per SM takes a contiguous share
+// of the blocks and streams them through a ring of shared-memory stages that
+// bulk copies (the TMA engine: a block's rows, or its runs inside pages) fill
+// `stages` blocks ahead, so every SM keeps ~200 KB in flight.  Each block is
+// summed with the per-block kernel's thread-to-row mapping and order (rows
+// ph, ph + PHASES, ... per thread, then the phases in order), so both kernels
+// give the same bits.
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads, 1)
+pool_stream_kernel(const uint8_t* __restrict__ K, KeyPages kpg, int64_t n_k, int B, int64_t M,
+                   int64_t m0, int64_t m1, float* __restrict__ kbar, uint16_t* __restrict__ kbar_hl,
+                   int stages, DevCtl ctl) {
+  constexpr int EPU = 8;
+  constexpr int UPR = D / EPU;
+  constexpr int PHASES = kPoolThreads / UPR;
+  constexpr int ROW_BYTES = D * 2;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  float(*part)[D] = reinterpret_cast<float(*)[D]>(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + PHASES * D * 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + stages);
+  uint8_t* ring = smem_raw + ((PHASES * D * 4 + 8 * stages + 16 + 127) / 128) * 128;
+  const int64_t stage_bytes = static_cast<int64_t>(B) * ROW_BYTES;
+  const int64_t nblk = m1 - m0;
+  const int64_t b0 = m0 + nblk * blockIdx.x / gridDim.x;
+  const int nb = static_cast<int>(m0 + nblk * (blockIdx.x + 1) / gridDim.x - b0);
+  const int tid = threadIdx.x, u = tid % UPR, ph = tid / UPR;
+  if (tid == 0) {
+    for (int i = 0; i < stages; ++i) mbar_init(smem_u32(full + i), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // (thread 0) block b0 + j into stage j % stages
+  auto issue = [&](int j) {
+    const int64_t first = (b0 + j) * B;
+    const int n_m = static_cast<int>(n_k - first < B ? n_k - first : static_cast<int64_t>(B));
+    const uint32_t bar = smem_u32(full + j % stages);
+    const uint32_t dst = smem_u32(ring + (j % stages) * stage_bytes);
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n_m) * ROW_BYTES);
+    if (!kpg.paged()) {
+      bulk_load(dst, K + first * ROW_BYTES, static_cast<uint32_t>(n_m) * ROW_BYTES, bar);
+      return;
+    }
+    const int ps = 1 << kpg.page_shift;
+    for (int r = 0; r < n_m;) {
+      const int64_t s = first + r;
+      const int in_page = ps - static_cast<int>(s & (ps - 1));
+      const int run = in_page < n_m - r ? in_page : n_m - r;
+      bulk_load(dst + r * ROW_BYTES, K + kpg.row(s, ctl) * ROW_BYTES,
+                static_cast<uint32_t>(run) * ROW_BYTES, bar);
+      r += run;
+    }
+  };
+  if (tid == 0)
+    for (int j = 0; j < nb && j < stages; ++j) issue(j);
+  for (int j = 0; j < nb; ++j) {
+    const int64_t m = b0 + j;
+    const int64_t first = m * B;
+    const int n_m = static_cast<int>(n_k - first < B ? n_k - first : static_cast<int64_t>(B));
+    const bool ok = mbar_wait(smem_u32(full + j % stages), (j / stages) & 1, abort_flag, ctl);
+    float acc[EPU];
+#pragma unroll
+    for (int e = 0; e < EPU; ++e) acc[e] = 0.0f;
+    const uint8_t* blk = ring + (j % stages) * stage_bytes + u * 16;
+    for (int r = ph; ok && r < n_m; r += PHASES) {
+      const uint4 a = *reinterpret_cast<const uint4*>(blk + r * ROW_BYTES);
+      const uint32_t* wv = reinterpret_cast<const uint32_t*>(&a);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[i]));
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < EPU; ++e) part[ph][u * EPU + e] = acc[e];
+    if (!__syncthreads_and(ok)) break;
+    // the stage is read: refill it
+    if (tid == 0 && j + stages < nb) issue(j + stages);
+    for (int c = tid; c < D; c += kPoolThreads) {
+      float sum = 0.0f;
+#pragma unroll 8
+      for (int p = 0; p < PHASES; ++p) sum += part[p][c];
+      const float mean = sum / static_cast<float>(n_m);
+      if (kbar) kbar[m * D + c] = mean;
+      if (kbar_hl) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(mean - __bfloat162float(hi));
+        kbar_hl[m * D + c] = __bfloat16_as_ushort(hi);
+        kbar_hl[(M + m) * D + c] = __bfloat16_as_ushort(lo);
+      }
+    }
+    __syncthreads();  // part is rewritten by the next block
+  }
+  if (*abort_flag) drain_pause(2000000);  // let issued copies land
+}
+
+template <int D, bool FP8>
+cudaError_t launch(const void* K, const float* k_scale, const KeyPages& kpg, int64_t n_k, int B,
+                   int64_t m0, int64_t m1, float* kbar, uint16_t* kbar_hl, const DevCtl& ctl,
+                   cudaStream_t s) {
+  const int64_t M = (n_k + B - 1) / B;
+  if (m1 > M) m1 = M;
+  if (m1 <= m0) return cudaSuccess;
+  const int sms = sm_count();
+  if constexpr (!FP8) {
+    // the streaming kernel when every SM gets two or more blocks and three
+    // block stages fit
+    constexpr int PHASES = kPoolThreads / (D / 8);
+    const int64_t stage_bytes = static_cast<int64_t>(B) * D * 2;
+    const int64_t fixed = ((PHASES * D * 4 + 8 * 8 + 16 + 127) / 128) * 128 + 128;
+    const int64_t budget = 227 * 1024 - fixed;
+    const int stages = static_cast<int>(std::min<int64_t>(8, budget / stage_bytes));
+    if (m1 - m0 >= 2 * static_cast<int64_t>(sms) && stages >= 3) {
+      const size_t smem = static_cast<size_t>(fixed + stages * stage_bytes);
+      cudaError_t e = cudaFuncSetAttribute(pool_stream_kernel<D>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      pool_stream_kernel<D><<<static_cast<unsigned>(sms), kPoolThreads, smem, s>>>(
+          static_cast<const uint8_t*>(K), kpg, n_k, B, M, m0, m1, kbar, kbar_hl, stages, ctl);
+      return cudaGetLastError();
+    }
+  }
+  pool_keys_kernel<D, FP8><<<static_cast<unsigned>(m1 - m0), kPoolThreads, 0, s>>>(
+      static_cast<const uint8_t*>(K), k_scale, kpg, n_k, B, M, m0, kbar, kbar_hl, ctl,
+      PoolBatch{nullptr, 0, nullptr, 0, 0});
   return cudaGetLastError();
 }
 

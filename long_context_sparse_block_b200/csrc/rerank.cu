@@ -130,20 +130,28 @@ rerank_scores_kernel(const RerankParams p) {
       fence_proxy_async_smem();
       mbar_arrive(bar(BFULL));
       ++qcount;
-      // each producer thread holds one candidate of every tile, loaded a tile
-      // ahead; all of a tile's copies are in flight at once (bf16: asynchronous
-      // 16-byte copies, whole rows per warp instruction, arriving on the stage
-      // barrier when they land; FP8: each thread loads its own row's codes for
-      // the next tile while decoding this tile's)
+      // each producer thread holds one candidate of every tile: its index is
+      // loaded kAhead tiles ahead and checked (and mapped to a physical row) one
+      // tile ahead, so no index load stalls the copies; all of a tile's copies
+      // are in flight at once (bf16: asynchronous 16-byte copies, whole rows per
+      // warp instruction, arriving on the stage barrier when they land; FP8:
+      // each thread loads its own row's codes for the next tile while decoding
+      // this tile's)
       const int32_t* crow = p.cand + static_cast<int64_t>(t) * p.kp;
-      // physical key row of this thread's candidate of a tile (-1: ignored)
-      auto cand_of = [&](int tile) -> int64_t {
+      auto raw_of = [&](int tile) -> int32_t {
         const int i = tile * kCand + tid;
-        int64_t c = i < p.kp ? static_cast<int64_t>(__ldg(crow + i)) : -1;
+        return (tile < tiles && i < p.kp) ? __ldg(crow + i) : -1;
+      };
+      // physical key row of a candidate (-1: ignored)
+      auto row_of = [&](int32_t c) -> int64_t {
         return (c >= 0 && c <= pos && c < p.n_k) ? p.kpg.row(c, p.ctl) : -1;
       };
+      constexpr int kAhead = 4;
+      int32_t rq[kAhead];
+#pragma unroll
+      for (int i = 0; i < kAhead; ++i) rq[i] = raw_of(i);
       constexpr int U8 = D / 16;  // 16-byte units of an e4m3 row
-      int64_t c_next = tiles > 0 ? cand_of(0) : -1;
+      int64_t c_next = tiles > 0 ? row_of(rq[0]) : -1;
       uint4 raw_next[FP8 ? U8 : 1];
       if constexpr (FP8) {
 #pragma unroll
@@ -158,7 +166,10 @@ rerank_scores_kernel(const RerankParams p) {
 #pragma unroll
           for (int u = 0; u < U8; ++u) raw[u] = raw_next[u];
         }
-        if (tile + 1 < tiles) c_next = cand_of(tile + 1);
+#pragma unroll
+        for (int i = 0; i + 1 < kAhead; ++i) rq[i] = rq[i + 1];
+        rq[kAhead - 1] = raw_of(tile + kAhead);
+        if (tile + 1 < tiles) c_next = row_of(rq[0]);
         if constexpr (FP8) {
 #pragma unroll
           for (int u = 0; u < U8; ++u)
@@ -267,20 +278,22 @@ rerank_scores_kernel(const RerankParams p) {
       for (int i = lane; i < NB; i += 32)
         w_s[i] = i < p.H ? __ldg(p.w + static_cast<int64_t>(t) * p.H + i) : 0.0f;
       __syncwarp();
-      // this lane's candidate of each of the group's tiles, loaded two tiles
-      // ahead (and, for FP8 keys, its scale one tile ahead)
+      // this lane's candidate of each of the group's tiles: its index loaded
+      // two of the group's tiles ahead and checked one ahead (and, for FP8
+      // keys, its scale loaded one ahead)
       const int first = static_cast<int>((grp - gtile % 2 + 2) % 2);
       const int32_t* crow = p.cand + static_cast<int64_t>(t) * p.kp;
-      // this lane's candidate of a tile: its physical key row (for the FP8
-      // scale), -1 when ignored
-      auto cand_of = [&](int tile) -> int64_t {
+      auto raw_of = [&](int tile) -> int32_t {
         const int i = tile * kCand + quad * 32 + lane;
-        if (tile >= tiles || i >= p.kp) return -1;
-        const int64_t c = __ldg(crow + i);
+        return (tile < tiles && i < p.kp) ? __ldg(crow + i) : -1;
+      };
+      // a candidate's physical key row (for the FP8 scale), -1 when ignored
+      auto row_of = [&](int32_t c) -> int64_t {
         if (c < 0 || c > pos || c >= p.n_k) return -1;
         return FP8 ? p.kpg.row(c, p.ctl) : c;
       };
-      int64_t c_cur = cand_of(first), c_nxt = cand_of(first + 2);
+      int32_t r_nxt = raw_of(first + 2), r_far = raw_of(first + 4);
+      int64_t c_cur = row_of(raw_of(first));
       float ks_cur = (FP8 && c_cur >= 0) ? __ldg(p.k_scale + c_cur) : 1.0f;
       for (int tile = first; tile < tiles; tile += 2) {
         if (lane == 0) ok = mbar_wait(bar(ACCFULL + grp), accph, abort_flag, p.ctl);
@@ -327,8 +340,9 @@ rerank_scores_kernel(const RerankParams p) {
         if (i < p.kp)
           p.full[static_cast<int64_t>(t) * p.ldf + i] =
               c_cur >= 0 ? (FP8 ? sum * ks_cur : sum) : -INFINITY;
-        c_cur = c_nxt;
-        c_nxt = cand_of(tile + 4);
+        c_cur = row_of(r_nxt);
+        r_nxt = r_far;
+        r_far = raw_of(tile + 6);
         ks_cur = (FP8 && c_cur >= 0) ? __ldg(p.k_scale + c_cur) : 1.0f;
       }
       gtile += tiles;
