@@ -44,6 +44,40 @@ def test_pool_matches_oracle(lib, n_k, d, B, fp8):
     assert np.all(np.abs(hi + lo - kbar) <= 2.0 ** -16 * np.abs(kbar) + 1e-30)
 
 
+@pytest.mark.parametrize("d,B,page_size", [(128, 128, 0), (64, 64, 16), (32, 128, 128),
+                                           (128, 128, 16)])
+def test_pool_stream_equals_per_block_and_oracle(lib, d, B, page_size):
+    # 301+ blocks (the last one partial): the full pooling takes the streaming
+    # kernel (bulk-copy stages, one CTA per SM), ranges of 100 blocks the per-block
+    # kernel; both sum in the same order, so they agree bit for bit, and both
+    # match the oracle; through pages (runs inside pages) the same bits again
+    n_k = 300 * B + 57
+    inp = W.generate(_wl(1, n_k - 1, n_k, 4, d, B, 1, 1, seed=n_k + d))
+    Kdev = dev(inp["K"])
+    kbar, hl = lib.misa_pool_keys(Kdev, B)
+    M = kbar.shape[0]
+    kb2 = torch.empty_like(kbar)
+    hl2 = torch.empty_like(hl)
+    for m0 in range(0, M, 100):
+        lib.misa_pool_keys_range(Kdev, B, m0, min(M, m0 + 100), kbar=kb2, kbar_hl=hl2)
+    assert torch.equal(kbar, kb2) and torch.equal(hl, hl2)
+    Kd = oracle.bf16_to_f64(inp["K"])
+    ref = oracle.pool_keys(Kd, B)
+    assert np.max(np.abs(kbar.cpu().numpy().astype(np.float64) - ref)) <= 1e-6 * np.abs(Kd).max() + 1e-9
+    if page_size:
+        n_blocks = -(-n_k // page_size)
+        table = torch.from_numpy(np.random.default_rng(d + B).permutation(n_blocks + 2)[:n_blocks]
+                                 .astype(np.int32)).cuda()
+        pages = torch.zeros(((n_blocks + 2) * page_size, d), dtype=Kdev.dtype, device="cuda")
+        flat = torch.zeros((n_blocks * page_size, d), dtype=Kdev.dtype, device="cuda")
+        flat[:n_k] = Kdev
+        pages.view(n_blocks + 2, page_size, d)[table.long()] = flat.view(n_blocks, page_size, d)
+        pk = lib.PagedKeys(pages.view(n_blocks + 2, page_size, d), table, n_k)
+        kb3, hl3 = lib.misa_pool_keys(pk, B)
+        assert torch.equal(kbar, kb3) and torch.equal(hl, hl3)
+    assert lib.misa_last_device_status() == lib.MISA_OK
+
+
 # ------------------------------------------------------------------ router
 
 @pytest.mark.parametrize("n_q,q_pos0,n_k,H,d,B,h,gen", [
@@ -68,6 +102,36 @@ def test_route_matches_oracle(lib, n_q, q_pos0, n_k, H, d, B, h, gen):
     no_block = sum(1 for t in range(n_q) if (q_pos0 + t + 1) // B == 0)
     print(f"near-tie rows: {exempt} of {n_q} ({no_block} see no complete block)")
     assert np.all(np.diff(heads, axis=1) > 0)                           # ascending, distinct
+
+
+def test_route_two_tile_units_equal_single_tiles(lib):
+    # 309 row tiles of 128 (query, head) rows: the whole call contracts two row
+    # tiles per pooled-key tile (the last unit holds one); slices of at most 100
+    # row tiles take one tile per unit.  Each row's arithmetic is the same, so r
+    # and the heads agree bit for bit, and they match the oracle.
+    n_q, H, d, B, h = 618, 64, 128, 128, 8
+    n_k = 9000
+    q_pos0 = n_k - n_q
+    wl = _wl(n_q, q_pos0, n_k, H, d, B, h, 8, seed=4242)
+    inp = W.generate(wl)
+    g = inputs_to_device(inp)
+    _, hl = lib.misa_pool_keys(g["K"], B)
+    heads, r = lib.misa_route_heads(g["Q"], g["w"], hl, q_pos0, n_k, B, h, want_r=True)
+    heads2 = torch.empty_like(heads)
+    r2 = torch.empty_like(r)
+    step = 100 * 128 // H  # queries in 100 row tiles
+    for c0 in range(0, n_q, step):
+        c1 = min(n_q, c0 + step)
+        hh, rr = lib.misa_route_heads(g["Q"][c0:c1], g["w"][c0:c1], hl, q_pos0 + c0, n_k, B, h,
+                                      want_r=True)
+        heads2[c0:c1] = hh
+        r2[c0:c1] = rr
+    assert torch.equal(r, r2) and torch.equal(heads, heads2)
+    Qd, Kd, wd = oracle.decode_inputs(inp)
+    r_ora, heads_ora = oracle.route(Qd, wd, oracle.pool_keys(Kd, B), q_pos0, n_k, B, h)
+    r = r.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(r - r_ora) <= 2e-3 * np.abs(r_ora) + 1e-5)
+    check_heads(heads.cpu().numpy(), r_ora, heads_ora, h, r_gpu=r.astype(np.float32))
 
 
 # ------------------------------------------------------------------ scoring
