@@ -656,7 +656,7 @@ topk_kernel(const TopkParams p) {
 // a threshold tau; the kernels below choose tau from a scored sample of the
 // row's visible keys and then take the exact top-k among the kept candidates.
 
-constexpr double kFusedMargin = 1.3;  // ~1.3 k candidates expected above tau
+constexpr double kFusedMargin = 1.4;  // ~1.4 k candidates expected above tau
 constexpr int kSampleBlock = 128;     // keys per contiguous sample block
 
 // Copies the keys of n_blocks contiguous 128-key blocks, evenly spaced over
@@ -682,7 +682,7 @@ gather_sample_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_
 }
 
 // Per row: tau[t] = lower edge of the 22-bit key bin holding the m-th largest
-// sampled logit, m ~ 1.3 k * n_s / visible(t) (or -inf: keep every visible key).
+// sampled logit, m ~ 1.4 k * n_s / visible(t) (or -inf: keep every visible key).
 // Also zeroes the row's repair flag gate[1 + t] and (block 0) the any-row flag
 // gate[0].
 __global__ void __launch_bounds__(kTopkThreads)
