@@ -576,10 +576,8 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   return true;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, kCtasPerSm)
-topk_kernel(const TopkParams p) {
-  if (p.gate && p.gate[1 + blockIdx.x] == 0) return;  // row needs no repair
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+// Row t of a top-k launch (all of the block's threads).
+__device__ void topk_row(const TopkParams& p, int t, uint8_t* smem_raw) {
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
   SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
   uint32_t* lkeys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
@@ -587,7 +585,6 @@ topk_kernel(const TopkParams p) {
   uint32_t* sel = lposs + p.cap;             // fast path only: ties at the k-th key
   uint32_t* counts = sel + kEqMax;           // fast path only
 
-  const int t = blockIdx.x;
   const uint32_t k = static_cast<uint32_t>(p.k);
   const int64_t n = p.row_len ? max(int64_t(0), min(static_cast<int64_t>(__ldg(p.row_len + t)), p.n_k))
                               : min(p.q_pos0 + t + 1, p.n_k);
@@ -649,6 +646,25 @@ topk_kernel(const TopkParams p) {
     }
   }
   for (uint32_t i = min(kept, k) + threadIdx.x; i < k; i += kTopkThreads) out.out[i] = -1;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, kCtasPerSm)
+topk_kernel(const TopkParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  topk_row(p, blockIdx.x, smem_raw);
+}
+
+// The repair launch: only rows with gate[1 + t] != 0, a persistent grid that
+// walks the row flags (nothing but the flag reads when no row is flagged).
+__global__ void __launch_bounds__(kTopkThreads, kCtasPerSm)
+topk_gated_kernel(const TopkParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  if (p.gate[0] == 0) return;  // no row flagged
+  for (int t = blockIdx.x; t < p.n_q; t += gridDim.x) {
+    if (p.gate[1 + t] == 0) continue;
+    topk_row(p, t, smem_raw);
+    __syncthreads();  // shared memory is reused by the next flagged row
+  }
 }
 
 // ---------------------------------------------------------------- fused top-k
@@ -917,10 +933,19 @@ cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, 
   int cap = k <= 4096 ? kFastCap : std::min(24576, ((2 * k + 4096) + 1023) / 1024 * 1024);
   const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * 8 +
                       (k <= kFastMaxK ? (kEqMax + kWarps) * 4 : 0);
+  TopkParams p{vals, ld, n_q, q_pos0, n_k, k, idx, cap, ctl, gate, row_len};
+  if (gate) {
+    cudaError_t e = cudaFuncSetAttribute(topk_gated_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = std::min(n_q, kCtasPerSm * sm_count());
+    topk_gated_kernel<<<grid, kTopkThreads, smem, s>>>(p);
+    return cudaGetLastError();
+  }
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  TopkParams p{vals, ld, n_q, q_pos0, n_k, k, idx, cap, ctl, gate, row_len};
   topk_kernel<<<n_q, kTopkThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
