@@ -555,12 +555,12 @@ score_tokens_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           accph ^= 1;
         }
       };
-      // h <= 32: the warp's 64 columns are read CW at a time (whole queries),
+      // h <= 32: the warp's 64 columns are read 32 at a time (whole queries),
       // the next load in flight while the current queries are summed; only two
       // CW-column buffers are live, which leaves registers for the selection
       constexpr bool CHUNKED = EC == 64 && HT >= 4 && HT <= 32;
       if constexpr (CHUNKED) {
-        constexpr int CW = HT <= 16 ? 16 : 32;  // columns per TMEM load
+        constexpr int CW = HT <= 64 ? 32 : 16;  // columns per TMEM load (16: 2% slower)
         constexpr int NCH = EC / CW;            // loads per tile
         constexpr int QPC = CW / HT;            // queries per load
         uint32_t vb[2][CW];
