@@ -839,17 +839,15 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
 //   any other row: the tokens tied at T are sorted and the lowest kept, then
 //   the kept tokens are sorted and written.  Two kept entries with the same
 //   token break the contract (distinct candidates) and are reported.
-__global__ void __launch_bounds__(kTopkThreads)
-select_candidates_kernel(const float* __restrict__ vals, int64_t ldv,
-                         const int32_t* __restrict__ cand, int kp, int64_t q_pos0, int64_t n_k,
-                         int k, int32_t* __restrict__ idx, int tmp_cap, DevCtl ctl) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+__device__ void select_candidates_row(const float* __restrict__ vals, int64_t ldv,
+                                      const int32_t* __restrict__ cand, int kp, int64_t q_pos0,
+                                      int64_t n_k, int k, int32_t* __restrict__ idx, int tmp_cap,
+                                      const DevCtl& ctl, int t, uint8_t* smem_raw) {
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
   SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
   uint32_t* toks = keys + kp;
   uint32_t* tmp = toks + kp;  // tmp_cap entries: the next power of two >= kp
-  const int t = blockIdx.x;
   const int64_t pos = q_pos0 + t;
   const float* vrow = vals + static_cast<int64_t>(t) * ldv;
   const int32_t* crow = cand + static_cast<int64_t>(t) * kp;
@@ -921,6 +919,92 @@ select_candidates_kernel(const float* __restrict__ vals, int64_t ldv,
     out[i] = i < n_win ? static_cast<int32_t>(tmp[i]) : -1;
 }
 
+// The rows the ordered kernel below marked (idx row starting with kUnorderedRow)
+// — candidates in any order — over a persistent grid.
+constexpr int32_t kUnorderedRow = -2;
+
+__global__ void __launch_bounds__(kTopkThreads)
+select_candidates_kernel(const float* __restrict__ vals, int64_t ldv,
+                         const int32_t* __restrict__ cand, int kp, int n_q, int64_t q_pos0,
+                         int64_t n_k, int k, int32_t* __restrict__ idx, int tmp_cap, DevCtl ctl) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  for (int t = blockIdx.x; t < n_q; t += gridDim.x) {
+    if (idx[static_cast<int64_t>(t) * k] != kUnorderedRow) continue;
+    __syncthreads();  // every thread has read the marker before the row is rewritten
+    select_candidates_row(vals, ldv, cand, kp, q_pos0, n_k, k, idx, tmp_cap, ctl, t, smem_raw);
+    __syncthreads();  // shared memory is reused by the next marked row
+  }
+}
+
+// Candidate entries: keys staged in shared memory, tokens read where they are.
+struct CandSrc {
+  const uint32_t* keys;
+  const int32_t* toks;
+  int64_t n;
+  __device__ __forceinline__ void load4(int64_t i0, uint32_t (&key)[4], uint32_t (&pos)[4]) const {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool in = i0 + e < n;
+      key[e] = in ? keys[i0 + e] : 0u;
+      pos[e] = in ? static_cast<uint32_t>(__ldg(toks + i0 + e)) : 0u;
+    }
+  }
+};
+
+// Rows whose valid candidates ascend, with only absent entries after them (what
+// the coarse selection emits): only the keys are staged (48 KB of shared
+// memory, four CTAs per SM), the tokens are read from the candidate row, and
+// one ordered pass writes the selection.  Any other row gets kUnorderedRow in
+// its first output slot and is left to select_candidates_kernel.
+__global__ void __launch_bounds__(kTopkThreads)
+select_candidates_ordered_kernel(const float* __restrict__ vals, int64_t ldv,
+                                 const int32_t* __restrict__ cand, int kp, int64_t q_pos0,
+                                 int64_t n_k, int k, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
+  const int t = blockIdx.x;
+  const int64_t pos = q_pos0 + t;
+  const float* vrow = vals + static_cast<int64_t>(t) * ldv;
+  const int32_t* crow = cand + static_cast<int64_t>(t) * kp;
+  int32_t* out = idx + static_cast<int64_t>(t) * k;
+  const uint32_t kk = static_cast<uint32_t>(k);
+  auto stage = [&](int i, float v, int32_t tok) {
+    const bool valid = tok >= 0 && tok <= pos && tok < n_k;
+    const uint32_t key = valid ? f2key(v) : 0u;
+    keys[i] = key;
+    return key != 0u ? 1u : 0u;
+  };
+  uint32_t c = 0;
+  bool unordered = false;
+  const bool vec = (kp & 3) == 0 && (reinterpret_cast<uintptr_t>(vrow) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(crow) & 15u) == 0;
+  if (vec) {
+    for (int i = threadIdx.x * 4; i < kp; i += kTopkThreads * 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(vrow + i));
+      const int4 tk = __ldg(reinterpret_cast<const int4*>(crow + i));
+      c += stage(i, v.x, tk.x) + stage(i + 1, v.y, tk.y) + stage(i + 2, v.z, tk.z) +
+           stage(i + 3, v.w, tk.w);
+    }
+  } else {
+    for (int i = threadIdx.x; i < kp; i += kTopkThreads) c += stage(i, __ldg(vrow + i), __ldg(crow + i));
+  }
+  uint32_t present;
+  block_excl_scan(c, sc, present);  // (also orders the key writes before the reads below)
+  for (int i = threadIdx.x; i + 1 < kp; i += kTopkThreads)
+    if (keys[i + 1] != 0u && (keys[i] == 0u || __ldg(crow + i) >= __ldg(crow + i + 1))) unordered = true;
+  if (__syncthreads_or(unordered)) {
+    if (threadIdx.x == 0) out[0] = kUnorderedRow;
+    return;
+  }
+  const CandSrc src{keys, crow, static_cast<int64_t>(kp)};
+  uint32_t T = 0u, need = 0u;  // present <= k: every present entry (key > 0)
+  if (present > kk) T = kth_largest_spread(src, kk, hist, sc, need);
+  const uint32_t kept = ordered_select(src, T, need, kk, OutEmit{out, kk}, sc);
+  for (uint32_t i = min(kept, kk) + threadIdx.x; i < kk; i += kTopkThreads) out[i] = -1;
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, int64_t n_k,
@@ -974,15 +1058,23 @@ cudaError_t launch_select_candidates(const float* vals, int64_t ldv, const int32
                                      int n_q, int64_t q_pos0, int64_t n_k, int k, int32_t* idx,
                                      const DevCtl& ctl, cudaStream_t s) {
   if (n_q <= 0 || k <= 0 || kp <= 0) return cudaSuccess;
+  // every row through the ordered kernel; rows it marks through the general one
+  const size_t smem1 = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(kp) * 4;
+  cudaError_t e = cudaFuncSetAttribute(select_candidates_ordered_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem1));
+  if (e != cudaSuccess) return e;
+  select_candidates_ordered_kernel<<<n_q, kTopkThreads, smem1, s>>>(vals, ldv, cand, kp, q_pos0,
+                                                                    n_k, k, idx);
   int cap = 1;
   while (cap < kp) cap <<= 1;
   const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + (2 * static_cast<size_t>(kp) + cap) * 4;
-  cudaError_t e = cudaFuncSetAttribute(select_candidates_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  e = cudaFuncSetAttribute(select_candidates_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  select_candidates_kernel<<<n_q, kTopkThreads, smem, s>>>(vals, ldv, cand, kp, q_pos0, n_k, k,
-                                                           idx, cap, ctl);
+  const int grid = std::min(n_q, 2 * sm_count());
+  select_candidates_kernel<<<grid, kTopkThreads, smem, s>>>(vals, ldv, cand, kp, n_q, q_pos0, n_k,
+                                                            k, idx, cap, ctl);
   return cudaGetLastError();
 }
 
