@@ -1011,10 +1011,13 @@ cudaError_t launch_topk(const float* vals, int64_t ld, int n_q, int64_t q_pos0, 
                         int k, int32_t* idx, const DevCtl& ctl, cudaStream_t s, const int* gate,
                         const int32_t* row_len) {
   if (n_q <= 0 || k <= 0) return cudaSuccess;
-  // list capacity: kFastCap for k <= 4096 (three CTAs per SM); larger k need
-  // room for ~1.4 k sampled-threshold entries (fast path) or for the entries in
-  // or above the k-th histogram bin (fallback)
-  int cap = k <= 4096 ? kFastCap : std::min(24576, ((2 * k + 4096) + 1023) / 1024 * 1024);
+  // list capacity: kFastCap for k <= 2048 (three CTAs per SM); larger k need
+  // room for ~1.4 k sampled-threshold entries (fast path; the list is split into
+  // equal per-warp regions, so with headroom for the warps' uneven shares) or
+  // for the entries in or above the k-th histogram bin (fallback)
+  int cap = k <= 2048 ? kFastCap
+                      : (k <= 4096 ? (2 * k + 1023) / 1024 * 1024
+                                   : std::min(24576, ((2 * k + 4096) + 1023) / 1024 * 1024));
   const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * 8 +
                       (k <= kFastMaxK ? (kEqMax + kWarps) * 4 : 0);
   TopkParams p{vals, ld, n_q, q_pos0, n_k, k, idx, cap, ctl, gate, row_len};
