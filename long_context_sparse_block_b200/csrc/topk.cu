@@ -36,6 +36,8 @@
 // a sample gather of 32 x 128 keys, a per-row threshold from the scored sample,
 // and the exact selection over the logits the select pass kept (pass-mask bits,
 // values in place), which flags rows it cannot finish for the exact repair.
+#include <type_traits>
+
 #include "internal.h"
 
 namespace misa {
@@ -744,20 +746,47 @@ fused_tau_kernel(const float* __restrict__ sample, int64_t lds, int n_s, int64_t
   if (threadIdx.x == 0) tau[t] = tf;
 }
 
+// List entries whose positions are kept as their low 16 bits: the list is in
+// position order, so the high bits of entry i's position count the 65536-key
+// boundaries at or below it (cross[j] = entries below position 65536 (j + 1)).
+struct ListSrc16 {
+  const uint32_t* keys;
+  const uint16_t* poss;
+  int64_t n;
+  uint32_t cross[3];
+  __device__ __forceinline__ uint32_t pos(int64_t i) const {
+    const uint32_t hi = (i >= cross[0] ? 1u : 0u) + (i >= cross[1] ? 1u : 0u) + (i >= cross[2] ? 1u : 0u);
+    return static_cast<uint32_t>(poss[i]) | (hi << 16);
+  }
+  __device__ __forceinline__ void load4(int64_t i0, uint32_t (&key)[4], uint32_t (&pos4)[4]) const {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int64_t i = i0 + e;
+      const bool in = i < n;
+      key[e] = in ? keys[i] : 0u;
+      pos4[e] = in ? pos(i) : 0u;
+    }
+  }
+};
+
 // Per row: the exact top-k among the logits the select-mode scoring kept (the
 // bits of the row's pass mask; their values stored in place).  They hold the
 // whole top-k whenever at least min(k, visible) of them passed.  Rows short of
 // that, or with more than list_cap kept, raise their repair flag (and the
-// any-row flag gate[0]) and write nothing.
+// any-row flag gate[0]) and write nothing.  P16 (large k): positions are
+// staged as 16-bit halves (6 bytes per list entry instead of 8), so the long
+// lists of large k still fit two CTAs per SM.
+template <bool P16>
 __global__ void __launch_bounds__(kTopkThreads)
 fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t* __restrict__ mask,
                     int64_t mask_ld, int64_t q_pos0, int64_t n_k, int k, int32_t* __restrict__ idx,
                     int* __restrict__ gate, int list_cap) {
+  using Pos = typename std::conditional<P16, uint16_t, uint32_t>::type;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
   SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
-  uint32_t* poss = keys + list_cap;
+  Pos* poss = reinterpret_cast<Pos*>(keys + list_cap);
   const int t = blockIdx.x;
   const int64_t visible = min(q_pos0 + t + 1, n_k);
   // every thread owns a run of 4-word units (the scoring pass wrote whole
@@ -767,13 +796,29 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
   const uint32_t per = (units + kTopkThreads - 1) / kTopkThreads;
   const uint32_t u0 = min(threadIdx.x * per, units), u1 = min(u0 + per, units);
   const uint4* mrow = reinterpret_cast<const uint4*>(mask + static_cast<int64_t>(t) * mask_ld);
-  uint32_t c = 0;
+  if (P16) {
+    // res[1 + j]: entries below position 65536 (j + 1), i.e. in units below 512 (j + 1)
+    if (threadIdx.x < 3) sc.res[1 + threadIdx.x] = 0u;
+    __syncthreads();
+  }
+  uint32_t c = 0, c_lo[3] = {0u, 0u, 0u};
   for (uint32_t u = u0; u < u1; ++u) {
     const uint4 m = __ldg(mrow + u);
-    c += __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
+    const uint32_t cu = __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
+    c += cu;
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+      if (u < 512u * (j + 1)) c_lo[j] += cu;
+  }
+  if (P16) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+      if (c_lo[j]) atomicAdd(&sc.res[1 + j], c_lo[j]);
   }
   uint32_t total;
-  uint32_t slot = block_excl_scan(c, sc, total);
+  uint32_t slot = block_excl_scan(c, sc, total);  // (also publishes res[1..3])
+  const uint32_t cross[3] = {P16 ? sc.res[1] : 0u, P16 ? sc.res[2] : 0u, P16 ? sc.res[3] : 0u};
+  __syncthreads();  // every thread has read res before the selection reuses it
   const uint32_t need_total = static_cast<uint32_t>(visible < k ? visible : k);
   if (total < need_total || total > static_cast<uint32_t>(list_cap)) {
     if (threadIdx.x == 0) {
@@ -791,20 +836,23 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
     for (int q = 0; q < 4; ++q) {
       uint32_t m = mw[q];
       while (m) {
-        poss[slot++] = (u * 4u + q) * 32u + static_cast<uint32_t>(__ffs(m) - 1);
+        poss[slot++] = static_cast<Pos>((u * 4u + q) * 32u + static_cast<uint32_t>(__ffs(m) - 1));
         m &= m - 1u;
       }
     }
   }
   __syncthreads();
   const float* row = logits + static_cast<int64_t>(t) * ld;
+  const ListSrc16 ls16{keys, reinterpret_cast<const uint16_t*>(poss), static_cast<int64_t>(total),
+                       {cross[0], cross[1], cross[2]}};
+  auto pos_of = [&](uint32_t i) { return P16 ? ls16.pos(i) : static_cast<uint32_t>(poss[i]); };
   constexpr int kBatch = 16;
   for (uint32_t b0 = 0; b0 < total; b0 += kBatch * kTopkThreads) {
     float v[kBatch];
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       const uint32_t i = b0 + j * kTopkThreads + threadIdx.x;
-      v[j] = i < total ? __ldg(row + poss[i]) : 0.0f;
+      v[j] = i < total ? __ldg(row + pos_of(i)) : 0.0f;
     }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
@@ -813,12 +861,18 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
     }
   }
   __syncthreads();
-  const ListSrc ls{keys, poss, static_cast<int64_t>(total)};
   const OutEmit out{idx + static_cast<int64_t>(t) * k, static_cast<uint32_t>(k)};
-  uint32_t T = 0u, need = 0u;
-  if (total > static_cast<uint32_t>(k))
-    T = kth_largest_spread(ls, static_cast<uint32_t>(k), hist, sc, need);
-  const uint32_t kept = ordered_select(ls, T, need, static_cast<uint32_t>(k), out, sc);
+  uint32_t T = 0u, need = 0u, kept;
+  if constexpr (P16) {
+    if (total > static_cast<uint32_t>(k))
+      T = kth_largest_spread(ls16, static_cast<uint32_t>(k), hist, sc, need);
+    kept = ordered_select(ls16, T, need, static_cast<uint32_t>(k), out, sc);
+  } else {
+    const ListSrc ls{keys, reinterpret_cast<const uint32_t*>(poss), static_cast<int64_t>(total)};
+    if (total > static_cast<uint32_t>(k))
+      T = kth_largest_spread(ls, static_cast<uint32_t>(k), hist, sc, need);
+    kept = ordered_select(ls, T, need, static_cast<uint32_t>(k), out, sc);
+  }
   for (uint32_t i = min(kept, static_cast<uint32_t>(k)) + threadIdx.x; i < static_cast<uint32_t>(k);
        i += kTopkThreads)
     out.out[i] = -1;
@@ -1081,20 +1135,25 @@ cudaError_t launch_select_candidates(const float* vals, int64_t ldv, const int32
   return cudaGetLastError();
 }
 
-int fused_list_cap(int k) { return std::max(6144, (3 * k + 1023) / 1024 * 1024); }
+// k <= 4096: 8-byte entries, max(6144, 3k) of them (three CTAs per SM at k =
+// 2048); larger k: 6-byte entries, 2k of them (two CTAs per SM at k = 8192, whose
+// kept lists run ~1.5 k on the chunk with threshold margin 1.4).
+int fused_list_cap(int k) {
+  return k <= 4096 ? std::max(6144, (3 * k + 1023) / 1024 * 1024) : (2 * k + 1023) / 1024 * 1024;
+}
 
 cudaError_t launch_fused_finish(const float* logits, int64_t ld, const uint32_t* mask,
                                 int64_t mask_ld, int n_q, int64_t q_pos0, int64_t n_k, int k,
                                 int32_t* idx, int* gate, cudaStream_t s) {
   if (n_q <= 0 || k <= 0) return cudaSuccess;
   const int cap = fused_list_cap(k);
-  const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * 8;
-  cudaError_t e = cudaFuncSetAttribute(fused_finish_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const bool p16 = k > 4096;
+  const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(cap) * (p16 ? 6 : 8);
+  auto kern = p16 ? fused_finish_kernel<true> : fused_finish_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  fused_finish_kernel<<<n_q, kTopkThreads, smem, s>>>(logits, ld, mask, mask_ld, q_pos0, n_k, k,
-                                                       idx, gate, cap);
+  kern<<<n_q, kTopkThreads, smem, s>>>(logits, ld, mask, mask_ld, q_pos0, n_k, k, idx, gate, cap);
   return cudaGetLastError();
 }
 
