@@ -129,4 +129,5 @@ def test_piece_schedules_cover_the_queries_once():
             assert all(c1 > c0 for c0, c1 in b)
             assert all(b[i][1] == b[i + 1][0] for i in range(len(b) - 1))
     r = ramp_pieces(8192)
-    assert sum(r) == 8192 and r[0] == 512 and r[-1] == 512 and max(r) == 2048
+    assert r == [384, 896, 1536, 2304, 2560, 512]
+    assert ramp_pieces(10) == [10]
