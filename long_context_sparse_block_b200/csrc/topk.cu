@@ -718,9 +718,35 @@ fused_tau_kernel(const float* __restrict__ sample, int64_t lds, int n_s, int64_t
   const int64_t visible = min(q_pos0 + t + 1, n_k);
   const float* row = sample + static_cast<int64_t>(t) * lds;
   uint32_t c = 0;
-  for (int i = threadIdx.x; i < n_s; i += kTopkThreads) {
-    keys[i] = f2key(__ldg(row + i));
-    c += keys[i] != 0u;
+  if ((n_s & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+    // 16-byte loads, four in flight per thread before the first is used
+    const float4* row4 = reinterpret_cast<const float4*>(row);
+    const int n4 = n_s >> 2;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += 4 * kTopkThreads) {
+      float4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * kTopkThreads;
+        if (i < n4) v[j] = __ldg(row4 + i);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * kTopkThreads;
+        if (i < n4) {
+          const uint32_t k4[4] = {f2key(v[j].x), f2key(v[j].y), f2key(v[j].z), f2key(v[j].w)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            keys[4 * i + e] = k4[e];
+            c += k4[e] != 0u;
+          }
+        }
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < n_s; i += kTopkThreads) {
+      keys[i] = f2key(__ldg(row + i));
+      c += keys[i] != 0u;
+    }
   }
   uint32_t present;
   block_excl_scan(c, sc, present);  // (also orders the key writes before the reads below)
@@ -801,15 +827,24 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
     if (threadIdx.x < 3) sc.res[1 + threadIdx.x] = 0u;
     __syncthreads();
   }
+  // the first kHold units of the run are loaded at once and stay in registers
+  // for the second pass (all of it while n_k <= 131072)
+  constexpr uint32_t kHold = 4;
+  uint4 mh[kHold];
+#pragma unroll
+  for (uint32_t j = 0; j < kHold; ++j)
+    mh[j] = u0 + j < u1 ? __ldg(mrow + u0 + j) : make_uint4(0u, 0u, 0u, 0u);
   uint32_t c = 0, c_lo[3] = {0u, 0u, 0u};
-  for (uint32_t u = u0; u < u1; ++u) {
-    const uint4 m = __ldg(mrow + u);
+  auto count_unit = [&](uint32_t u, const uint4& m) {
     const uint32_t cu = __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
     c += cu;
 #pragma unroll
     for (int j = 0; j < 3; ++j)
       if (u < 512u * (j + 1)) c_lo[j] += cu;
-  }
+  };
+#pragma unroll
+  for (uint32_t j = 0; j < kHold; ++j) count_unit(u0 + j, mh[j]);  // (zero past u1)
+  for (uint32_t u = u0 + kHold; u < u1; ++u) count_unit(u, __ldg(mrow + u));
   if (P16) {
 #pragma unroll
     for (int j = 0; j < 3; ++j)
@@ -829,8 +864,7 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
   }
   // kept positions in ascending order, then their logits (batches of
   // independent loads)
-  for (uint32_t u = u0; u < u1; ++u) {
-    const uint4 m4 = __ldg(mrow + u);
+  auto emit_unit = [&](uint32_t u, const uint4& m4) {
     const uint32_t mw[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -840,7 +874,10 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
         m &= m - 1u;
       }
     }
-  }
+  };
+#pragma unroll
+  for (uint32_t j = 0; j < kHold; ++j) emit_unit(u0 + j, mh[j]);
+  for (uint32_t u = u0 + kHold; u < u1; ++u) emit_unit(u, __ldg(mrow + u));
   __syncthreads();
   const float* row = logits + static_cast<int64_t>(t) * ld;
   const ListSrc16 ls16{keys, reinterpret_cast<const uint16_t*>(poss), static_cast<int64_t>(total),

@@ -62,6 +62,10 @@ FUSED_CASES = [
     (129, 20000, 24000, 64, 128, 128, 32, 1024, False),
     (100, 6000, 7000, 64, 128, 128, 8, 8192, False),     # k above most rows' prefix
     (64, 4095, 4200, 16, 32, 32, 4, 1, False),            # smallest fused prefix, k = 1
+    # 2^17 < n_k < 2^18: more than four mask units per finish thread, and the
+    # 16-bit list positions of large k cross three 65536-key boundaries
+    (24, 200000, 200100, 64, 128, 128, 8, 2048, False),
+    (24, 200000, 200100, 64, 128, 128, 8, 6000, False),
 ]
 
 
