@@ -293,7 +293,11 @@ struct RegionSrc {
 // band of values (the kept top few percent of a row), which a fixed top-bits
 // digit piles onto a few bins (and their shared-memory atomics onto a few
 // addresses); here they spread over up to 4096 bins.
-template <class Src>
+// kWholeBin: when the bin of the m-th key holds exactly the entries still
+// needed, stop there and return T = bin floor - 1 with need = 0 (every entry
+// above T is taken, none equal to it) -- for callers that take the entries by
+// "key > T, then `need` of key == T" and nothing else.
+template <class Src, bool kWholeBin = false>
 __device__ uint32_t kth_largest_spread(const Src& src, uint32_t m, uint32_t* hist, SmemCtl& sc,
                                        uint32_t& need) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -349,7 +353,12 @@ __device__ uint32_t kth_largest_spread(const Src& src, uint32_t m, uint32_t* his
     find_bin<kBins1>(hist, m, sc);
     T |= sc.res[0] << lob;
     m -= sc.res[1];
+    const bool whole = kWholeBin && lob > 0 && T > 0u && hist[sc.res[0]] == m;
     __syncthreads();
+    if (whole) {  // T is the bin floor
+      need = 0u;
+      return T - 1u;
+    }
     if (lob == 0) break;
     hib = lob - 1;
   }
@@ -902,12 +911,12 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
   uint32_t T = 0u, need = 0u, kept;
   if constexpr (P16) {
     if (total > static_cast<uint32_t>(k))
-      T = kth_largest_spread(ls16, static_cast<uint32_t>(k), hist, sc, need);
+      T = kth_largest_spread<ListSrc16, true>(ls16, static_cast<uint32_t>(k), hist, sc, need);
     kept = ordered_select(ls16, T, need, static_cast<uint32_t>(k), out, sc);
   } else {
     const ListSrc ls{keys, reinterpret_cast<const uint32_t*>(poss), static_cast<int64_t>(total)};
     if (total > static_cast<uint32_t>(k))
-      T = kth_largest_spread(ls, static_cast<uint32_t>(k), hist, sc, need);
+      T = kth_largest_spread<ListSrc, true>(ls, static_cast<uint32_t>(k), hist, sc, need);
     kept = ordered_select(ls, T, need, static_cast<uint32_t>(k), out, sc);
   }
   for (uint32_t i = min(kept, static_cast<uint32_t>(k)) + threadIdx.x; i < static_cast<uint32_t>(k);
