@@ -555,7 +555,7 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
   const RegionSrc rs{lkeys, lposs, counts, static_cast<int64_t>(kWarps) * region, region, inv};
   // ---- exact k-th key within the list
   uint32_t T = 0u, need = 0u;
-  if (total > k) T = kth_largest_spread(rs, k, hist, sc, need);
+  if (total > k) T = kth_largest_spread<RegionSrc, true>(rs, k, hist, sc, need);
   // ---- kept positions: key > T, and the `need` lowest positions with key == T,
   // marked in a bitmap of the row (ascending output without a sort)
   uint32_t* bitmap = hist;                       // kBins1 words = 131072 positions
@@ -571,7 +571,7 @@ __device__ bool topk_fast(const TopkParams& p, const RowSrc& src, const OutEmit&
     const uint32_t pos = lposs[x];
     if (key > T) {
       atomicOr(&bitmap[pos >> 5], 1u << (pos & 31u));
-    } else if (key == T && key != 0u) {
+    } else if (need > 0u && key == T && key != 0u) {  // (need = 0: no tie is taken)
       const uint32_t e = atomicAdd(neq, 1u);
       if (e < static_cast<uint32_t>(kEqMax)) sel[e] = pos;
     }
@@ -983,7 +983,9 @@ __device__ void select_candidates_row(const float* __restrict__ vals, int64_t ld
 
   const ListSrc ls{keys, toks, static_cast<int64_t>(kp)};
   uint32_t T = 0u, need = 0u;  // present <= k: every present entry (key > 0)
-  if (present > kk) T = kth_largest_spread(ls, kk, hist, sc, need);
+  if (present > kk)  // (ordered rows take entries only by key > T and `need` of key == T)
+    T = unordered ? kth_largest_spread(ls, kk, hist, sc, need)
+                  : kth_largest_spread<ListSrc, true>(ls, kk, hist, sc, need);
   if (!unordered) {
     const uint32_t kept = ordered_select(ls, T, need, kk, OutEmit{out, kk}, sc);
     for (uint32_t i = min(kept, kk) + threadIdx.x; i < kk; i += kTopkThreads) out[i] = -1;
@@ -1100,7 +1102,7 @@ select_candidates_ordered_kernel(const float* __restrict__ vals, int64_t ldv,
   }
   const CandSrc src{keys, crow, static_cast<int64_t>(kp)};
   uint32_t T = 0u, need = 0u;  // present <= k: every present entry (key > 0)
-  if (present > kk) T = kth_largest_spread(src, kk, hist, sc, need);
+  if (present > kk) T = kth_largest_spread<CandSrc, true>(src, kk, hist, sc, need);
   const uint32_t kept = ordered_select(src, T, need, kk, OutEmit{out, kk}, sc);
   for (uint32_t i = min(kept, kk) + threadIdx.x; i < kk; i += kTopkThreads) out[i] = -1;
 }
