@@ -333,6 +333,10 @@ def _adversarial_rows(n, rng):
     big[::7] = np.float32(1e30)
     rows.append(big)
     rows.append(-np.abs(rng.standard_normal(n)).astype(np.float32) - 1.0)    # all negative
+    # consecutive floats, descending with the position: the k-th key is the floor
+    # of its radix bin whenever 16 | n - k, so the select stops there with the
+    # threshold one ulp below it, a value the row also holds (and must not take)
+    rows.append((np.uint32(0x3FC00000) + (n - 1 - np.arange(n)).astype(np.uint32)).view(np.float32))
     return np.stack(rows)
 
 
