@@ -712,13 +712,14 @@ gather_sample_kernel(const uint8_t* __restrict__ K, const float* __restrict__ k_
 // sampled logit, m ~ 1.4 k * n_s / visible(t) (or -inf: keep every visible key).
 // Also zeroes the row's repair flag gate[1 + t] and (block 0) the any-row flag
 // gate[0].
+constexpr int kTauPer = 16;  // sample keys held per thread: n_s <= kTauPer * kTopkThreads
+
 __global__ void __launch_bounds__(kTopkThreads)
 fused_tau_kernel(const float* __restrict__ sample, int64_t lds, int n_s, int64_t q_pos0,
                  int64_t n_k, int k, float* __restrict__ tau, int* __restrict__ gate) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
   SmemCtl& sc = *reinterpret_cast<SmemCtl*>(smem_raw + kBins1 * 4);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kBins1 * 4 + sizeof(SmemCtl));
   const int t = blockIdx.x;
   if (threadIdx.x == 0) {
     gate[1 + t] = 0;
@@ -726,53 +727,59 @@ fused_tau_kernel(const float* __restrict__ sample, int64_t lds, int n_s, int64_t
   }
   const int64_t visible = min(q_pos0 + t + 1, n_k);
   const float* row = sample + static_cast<int64_t>(t) * lds;
-  uint32_t c = 0;
+  // the row's sampled logits as keys in registers (0 = absent or past n_s),
+  // every load issued before the first is used
+  uint32_t key[kTauPer];
   if ((n_s & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
-    // 16-byte loads, four in flight per thread before the first is used
     const float4* row4 = reinterpret_cast<const float4*>(row);
     const int n4 = n_s >> 2;
-    for (int i0 = threadIdx.x; i0 < n4; i0 += 4 * kTopkThreads) {
-      float4 v[4];
+    float4 v[kTauPer / 4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = i0 + j * kTopkThreads;
-        if (i < n4) v[j] = __ldg(row4 + i);
-      }
+    for (int j = 0; j < kTauPer / 4; ++j) {
+      const int i = threadIdx.x + j * kTopkThreads;
+      v[j] = i < n4 ? __ldg(row4 + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = i0 + j * kTopkThreads;
-        if (i < n4) {
-          const uint32_t k4[4] = {f2key(v[j].x), f2key(v[j].y), f2key(v[j].z), f2key(v[j].w)};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            keys[4 * i + e] = k4[e];
-            c += k4[e] != 0u;
-          }
-        }
-      }
+    for (int j = 0; j < kTauPer / 4; ++j) {
+      key[4 * j] = f2key(v[j].x);
+      key[4 * j + 1] = f2key(v[j].y);
+      key[4 * j + 2] = f2key(v[j].z);
+      key[4 * j + 3] = f2key(v[j].w);
     }
   } else {
-    for (int i = threadIdx.x; i < n_s; i += kTopkThreads) {
-      keys[i] = f2key(__ldg(row + i));
-      c += keys[i] != 0u;
+    float v[kTauPer];
+#pragma unroll
+    for (int j = 0; j < kTauPer; ++j) {
+      const int i = threadIdx.x + j * kTopkThreads;
+      v[j] = i < n_s ? __ldg(row + i) : -INFINITY;
     }
+#pragma unroll
+    for (int j = 0; j < kTauPer; ++j) key[j] = f2key(v[j]);
   }
+  for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) hist[i] = 0u;
+  uint32_t c = 0;
+#pragma unroll
+  for (int j = 0; j < kTauPer; ++j) c += key[j] != 0u;
   uint32_t present;
-  block_excl_scan(c, sc, present);  // (also orders the key writes before the reads below)
+  block_excl_scan(c, sc, present);  // (also orders the zeroing before the counts below)
   const uint32_t m = static_cast<uint32_t>(kFusedMargin * k * static_cast<double>(n_s) /
                                            static_cast<double>(visible)) + 16u;
   float tf = -INFINITY;
   if (m <= present) {
-    for (int i = threadIdx.x; i < kBins1; i += kTopkThreads) hist[i] = 0u;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n_s; i += kTopkThreads)
-      if (keys[i] != 0u) atomicAdd(&hist[keys[i] >> 20], 1u);
+    // the m-th largest key's 12-bit top digit, then its next 10 bits
+#pragma unroll
+    for (int j = 0; j < kTauPer; ++j)
+      if (key[j] != 0u) atomicAdd(&hist[key[j] >> 20], 1u);
     __syncthreads();
     find_bin<kBins1>(hist, m, sc);
     const uint32_t b1 = sc.res[0], above1 = sc.res[1];
     __syncthreads();
-    const ListSrc ls{keys, keys, static_cast<int64_t>(n_s)};
-    digit_hist(ls, 20, b1, 10, hist);
+    for (int i = threadIdx.x; i < 1024; i += kTopkThreads) hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kTauPer; ++j)
+      if (key[j] != 0u && (key[j] >> 20) == b1) atomicAdd(&hist[(key[j] >> 10) & 1023u], 1u);
+    __syncthreads();
     find_bin<1024>(hist, m - above1, sc);
     const uint32_t tk = (b1 << 20) | (sc.res[0] << 10);  // >= every real key's bin floor
     const uint32_t bits = (tk & 0x80000000u) ? (tk & 0x7FFFFFFFu) : ~tk;  // key -> float bits
@@ -1151,7 +1158,8 @@ cudaError_t launch_gather_sample(const void* K, const float* k_scale, const KeyP
 cudaError_t launch_fused_tau(const float* sample, int64_t lds, int n_s, int n_q, int64_t q_pos0,
                              int64_t n_k, int k, float* tau, int* gate, cudaStream_t s) {
   if (n_q <= 0) return cudaSuccess;
-  const size_t smem = kBins1 * 4 + sizeof(SmemCtl) + static_cast<size_t>(n_s) * 4;
+  if (n_s > kTauPer * kTopkThreads) return cudaErrorInvalidValue;
+  const size_t smem = kBins1 * 4 + sizeof(SmemCtl);
   cudaError_t e = cudaFuncSetAttribute(fused_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
