@@ -586,7 +586,8 @@ def run_variants(wl, inp, stream, flush):
     out["dagger_ms"] = round(_time_ms(lambda: dg.run(Q, K, w), stream, flush), 4)
     out["dagger_recall_vs_dense"] = round(_recall(dg.run(Q, K, w), ref, wl.n_k), 4)
     del dense, ref, dg
-    # FP8 keys (e4m3 + per-token scale), every stage decoding in-kernel
+    # FP8 keys (e4m3 + per-token scale): pooling and the rerank read the codes,
+    # the fused scoring their bf16 decode (made once per chunk by the indexer)
     K8c, sc = Wm.e4m3_quantize_keys(Wm.bf16_values(inp["K"]).astype(np.float64))
     K8 = torch.from_numpy(K8c).cuda()
     ks = torch.from_numpy(sc).cuda()

@@ -55,7 +55,12 @@ typedef enum misa_status {
 
 typedef enum misa_kdtype {
     MISA_K_BF16 = 0,
-    MISA_K_FP8E4M3 = 1
+    MISA_K_FP8E4M3 = 1,
+    /* bf16 codes with a per-token fp32 scale k_scale[n_k] > 0 that multiplies
+     * the dot product like the e4m3 scale: e4m3 keys decoded once by
+     * misa_keys_e4m3_to_bf16 and kept with their scales.  Accepted only by
+     * misa_score_topk with contiguous keys; the other calls refuse it. */
+    MISA_K_BF16_SCALED = 2
 } misa_kdtype;
 
 /*
@@ -205,12 +210,30 @@ int misa_rerank_noalloc(const uint16_t* Q, const float* w, const void* K, const 
  *     sequence also needs q_pos0 >= 4095 and h in {4, 8, 16, 32, 64}, else the
  *     call is unfused.  After a fused call, ws holds n_q + 1 int32 repair flags
  *     at offset 0: [0] != 0 iff any row took the fallback, [1 + t] for row t.
+ * kdtype may also be MISA_K_BF16_SCALED (contiguous keys): the fused sequence
+ * then reads the given bf16 codes and their scales directly, where e4m3 keys
+ * are decoded into the workspace on every call, so a caller that scores the
+ * same FP8 keys in several query pieces decodes them once.  The logits equal
+ * those of the e4m3 keys the codes were decoded from.
  * Shapes and other limits as misa_score_tokens; 0 <= k <= 16384.
  */
 int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, const void* K,
                     const float* k_scale, int kdtype, int n_q, int64_t q_pos0, int64_t n_k, int H,
                     int d, int h, int k, int32_t* idx, float* logits, int64_t ld, void* ws,
                     size_t ws_bytes, void* stream);
+
+/*
+ * FP8 index keys (the FP8 indexer of the integration issue "Clarification on
+ * the Figure 3 baseline...": e4m3 codes with a per-token scale) decoded to bf16
+ * codes: Kbf[s, i] = bf16(e4m3(K8[s, i])), exact (every e4m3 value is a bf16
+ * value; NaN codes give a bf16 NaN); the scales are not applied (pass them with
+ * the codes as MISA_K_BF16_SCALED).
+ *   K8 [n_k, d] e4m3 codes, Kbf [n_k, d] bf16 codes: caller-owned device
+ *   memory, 16-byte aligned, not overlapping; d in {32, 64, 128}.
+ * Asynchronous on `stream`.  Returns MISA_ERR_INVALID_ARG for bad pointers or
+ * sizes, MISA_ERR_UNSUPPORTED for other d.
+ */
+int misa_keys_e4m3_to_bf16(const uint8_t* K8, int64_t n_k, int d, uint16_t* Kbf, void* stream);
 
 /*
  * Paged key caches.  The integration issue ("Clarification on the Figure 3

@@ -24,6 +24,7 @@ MISA_ERR_WORKSPACE = -5
 MISA_ERR_DEVICE = -6
 MISA_K_BF16 = 0
 MISA_K_FP8E4M3 = 1
+MISA_K_BF16_SCALED = 2
 
 
 class MisaError(RuntimeError):
@@ -49,6 +50,7 @@ _SIGS = {
                                    _int, _int, _vp, _vp]),
     "misa_score_topk": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _int, _int, _int,
                                _int, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "misa_keys_e4m3_to_bf16": (_int, [_vp, _i64, _int, _vp, _vp]),
     "misa_pool_keys_paged": (_int, [_vp, _vp, _int, _vp, _int, _i64, _i64, _int, _int, _i64, _i64,
                                     _vp, _vp, _vp]),
     "misa_score_tokens_paged": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _vp, _int, _i64, _int, _i64,
@@ -337,14 +339,31 @@ def misa_score_topk(Q, w, heads, K, q_pos0: int, k: int, k_scale=None, h: int | 
         _check("misa_score_topk_paged", st)
         return idx
     _need(k_scale, n_k, "k_scale")
+    # bf16 codes that come with scales are decoded e4m3 keys (misa_keys_e4m3_to_bf16)
+    kd = _kdtype(K)
+    if kd == MISA_K_BF16 and k_scale is not None:
+        kd = MISA_K_BF16_SCALED
     st = _lib.misa_score_topk(_ptr(Q, _BF16_CODES, "Q"), _ptr(w, (torch.float32,), "w"),
                               _ptr(heads, (torch.int32,), "heads"), _ptr(K, name="K"),
-                              _ptr(k_scale, (torch.float32,), "k_scale"), _kdtype(K), n_q, q_pos0,
+                              _ptr(k_scale, (torch.float32,), "k_scale"), kd, n_q, q_pos0,
                               n_k, H, d, h, k, _ptr(idx, (torch.int32,), "idx"),
                               ctypes.c_void_p(logits.data_ptr()), logits.stride(0),
                               _ptr(ws, name="ws") if ws_bytes else None, ws_bytes, _stream())
     _check("misa_score_topk", st)
     return idx
+
+
+def misa_keys_e4m3_to_bf16(K8, out=None):
+    """e4m3 key codes [n_k, d] -> bf16 codes [n_k, d] (int16 view), exact; the
+    per-token scales are not applied (score the codes with them as scaled keys)."""
+    n_k, d = K8.shape
+    if out is None:
+        out = torch.empty((n_k, d), dtype=torch.int16, device=K8.device)
+    _need(out, n_k * d, "out")
+    st = _lib.misa_keys_e4m3_to_bf16(_ptr(K8, _E4M3_CODES, "K8"), n_k, d,
+                                     _ptr(out, _BF16_CODES, "out"), _stream())
+    _check("misa_keys_e4m3_to_bf16", st)
+    return out
 
 
 def misa_workspace_size(op: str, n_q: int, n_k: int, k: int, kp: int) -> int:

@@ -95,10 +95,12 @@ KeyArg paged_keys(const void* pages, const float* k_scale, int kdtype, const int
   return KeyArg{pages, k_scale, kdtype, KeyPages{block_table, shift, n_pages}};
 }
 
-int check_keys(const KeyArg& k, int64_t n_k) {
+// scaled_bf16_ok: the call takes MISA_K_BF16_SCALED (contiguous keys only).
+int check_keys(const KeyArg& k, int64_t n_k, bool scaled_bf16_ok = false) {
   if (!k.K || !aligned16(k.K)) return MISA_ERR_INVALID_ARG;
-  if (k.kdtype != MISA_K_BF16 && k.kdtype != MISA_K_FP8E4M3) return MISA_ERR_INVALID_ARG;
-  if (k.fp8() && (!k.k_scale || !aligned4(k.k_scale))) return MISA_ERR_INVALID_ARG;
+  const bool scaled = k.kdtype == MISA_K_BF16_SCALED && scaled_bf16_ok && !k.kpg.bt;
+  if (k.kdtype != MISA_K_BF16 && k.kdtype != MISA_K_FP8E4M3 && !scaled) return MISA_ERR_INVALID_ARG;
+  if ((k.fp8() || scaled) && (!k.k_scale || !aligned4(k.k_scale))) return MISA_ERR_INVALID_ARG;
   if (n_k > 0x7fffffffLL) return MISA_ERR_INVALID_ARG;
   if (k.kpg.bt) {
     if (!aligned4(k.kpg.bt)) return MISA_ERR_INVALID_ARG;
@@ -320,7 +322,7 @@ int score_topk_impl(const uint16_t* Q, const float* w, const int32_t* heads, con
       ld < n_k || ld % 4 != 0 || k < 0 || k > 16384)
     return MISA_ERR_INVALID_ARG;
   if (!heads && h != H) return MISA_ERR_INVALID_ARG;
-  if (const int st = check_keys(key, n_k)) return st;
+  if (const int st = check_keys(key, n_k, true)) return st;
   if (!good_d(d) || !pow2(h) || h > 128) return MISA_ERR_UNSUPPORTED;
   if (n_q == 0 || k == 0) return MISA_OK;
   const size_t need = misa_workspace_size("score_topk", n_q, n_k, k, 0);
@@ -328,14 +330,16 @@ int score_topk_impl(const uint16_t* Q, const float* w, const int32_t* heads, con
   DevCtl ctl;
   if (!make_ctl(ctl)) return MISA_ERR_CUDA;
   const cudaStream_t s = as_stream(stream);
-  const bool fp8 = key.fp8();
+  const bool fp8 = key.fp8();                               // e4m3 codes
+  const bool decoded = key.kdtype == MISA_K_BF16_SCALED;     // bf16 codes + scales
   ScoreLaunch a{};
   a.Q = Q;
   a.w = w;
   a.heads = heads;
   a.K = key.K;
   a.k_scale = key.k_scale;
-  a.fp8 = fp8;
+  a.fp8 = fp8 || decoded;  // a per-key scale in the epilogue
+  a.k_bf16 = decoded;
   a.kpg = key.kpg;
   a.n_q = n_q;
   a.q_pos0 = q_pos0;
@@ -376,13 +380,13 @@ int score_topk_impl(const uint16_t* Q, const float* w, const int32_t* heads, con
       if (kbf_scale) a.k_scale = kbf_scale;
       a.kpg = KeyPages{nullptr, 0, 0};
     }
-    e = launch_gather_sample(a.K, fp8 ? a.k_scale : nullptr, a.kpg, 2 * d, q_pos0 + 1,
-                             kSampleBlocks, Ks, fp8 ? ks_scale : nullptr, ctl, s);
+    e = launch_gather_sample(a.K, a.fp8 ? a.k_scale : nullptr, a.kpg, 2 * d, q_pos0 + 1,
+                             kSampleBlocks, Ks, a.fp8 ? ks_scale : nullptr, ctl, s);
   }
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   ScoreLaunch sa = a;  // the sample: every sampled key is visible to every query
   sa.K = Ks;
-  sa.k_scale = fp8 ? ks_scale : nullptr;
+  sa.k_scale = a.fp8 ? ks_scale : nullptr;
   sa.kpg = KeyPages{nullptr, 0, 0};
   sa.q_pos0 = kSampleKeys - 1;
   sa.n_k = kSampleKeys;
@@ -561,6 +565,17 @@ int misa_score_topk(const uint16_t* Q, const float* w, const int32_t* heads, con
                     size_t ws_bytes, void* stream) {
   return score_topk_impl(Q, w, heads, contiguous_keys(K, k_scale, kdtype), n_q, q_pos0, n_k, H, d,
                          h, k, idx, logits, ld, ws, ws_bytes, stream);
+}
+
+int misa_keys_e4m3_to_bf16(const uint8_t* K8, int64_t n_k, int d, uint16_t* Kbf, void* stream) {
+  if (!K8 || !aligned16(K8) || !Kbf || !aligned16(Kbf) || n_k < 0 || n_k > 0x7fffffffLL)
+    return MISA_ERR_INVALID_ARG;
+  if (!good_d(d)) return MISA_ERR_UNSUPPORTED;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(K8), a1 = a0 + static_cast<uintptr_t>(n_k) * d;
+  const uintptr_t b0 = reinterpret_cast<uintptr_t>(Kbf), b1 = b0 + static_cast<uintptr_t>(n_k) * d * 2;
+  if (n_k > 0 && a0 < b1 && b0 < a1) return MISA_ERR_INVALID_ARG;  // overlapping buffers
+  // n_k * d is a multiple of 16 (d is): whole 16-code units
+  return cuda_status(launch_e4m3_to_bf16(K8, Kbf, n_k * d, as_stream(stream)));
 }
 
 int misa_score_topk_paged(const uint16_t* Q, const float* w, const int32_t* heads,

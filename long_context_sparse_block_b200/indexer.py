@@ -101,13 +101,25 @@ class MisaIndexer:
         else:
             self.final = self.sel
 
-    def _select(self, c0, c1, Q, K, w, k_scale):
+    def _scoring_keys(self, K, k_scale):
+        """The keys the fused scoring reads: e4m3 keys decoded to bf16 codes once
+        per chunk (scored with their scales), so that every query sub-chunk or
+        piece does not decode them again; bf16 keys as they are."""
+        if k_scale is None or K.dtype not in (torch.uint8, torch.float8_e4m3fn):
+            return K
+        kd = getattr(self, "_kdec", None)
+        if kd is None or kd.shape != K.shape or kd.device != K.device:
+            kd = self._kdec = torch.empty(K.shape, dtype=torch.int16, device=K.device)
+        return _lib.misa_keys_e4m3_to_bf16(K, out=kd)
+
+    def _select(self, c0, c1, Q, K, w, k_scale, Ks=None):
         """Scoring, top-k (and the MISA-dagger rerank) of queries c0..c1-1 whose
-        heads are routed; Q and w hold the whole chunk's rows."""
+        heads are routed; Q and w hold the whole chunk's rows.  Ks: the keys the
+        scoring reads (K decoded, from _scoring_keys); the rerank reads K."""
         s = self.shape
         heads = None if s.dense else self.heads[c0:c1]
-        _lib.misa_score_topk(Q[c0:c1], w[c0:c1], heads, K, s.q_pos0 + c0, self.sel.shape[1],
-                             k_scale=k_scale, h=s.h, idx=self.sel[c0:c1],
+        _lib.misa_score_topk(Q[c0:c1], w[c0:c1], heads, K if Ks is None else Ks, s.q_pos0 + c0,
+                             self.sel.shape[1], k_scale=k_scale, h=s.h, idx=self.sel[c0:c1],
                              logits=self.logits[:c1 - c0], ws=self.ws_sel)
         if s.kp:
             _lib.misa_rerank(Q[c0:c1], w[c0:c1], K, self.sel[c0:c1], s.q_pos0 + c0, s.k,
@@ -123,10 +135,11 @@ class MisaIndexer:
         if not s.dense:
             _lib.misa_pool_keys(K, s.B, k_scale=k_scale, kbar_hl=self.kbar_hl, want_kbar=False)
             _lib.misa_route_heads(Q, w, self.kbar_hl, s.q_pos0, s.n_k, s.B, s.h, heads=self.heads)
+        Ks = self._scoring_keys(K, k_scale) if on_subchunk is None else K
         for c0 in range(0, s.n_q, self.sub):
             c1 = min(s.n_q, c0 + self.sub)
             if on_subchunk is None:
-                self._select(c0, c1, Q, K, w, k_scale)
+                self._select(c0, c1, Q, K, w, k_scale, Ks)
                 continue
             lg = self.logits[:c1 - c0]
             heads = None if s.dense else self.heads[c0:c1]
@@ -193,13 +206,14 @@ class MisaIndexer:
         compute.wait_event(ev_k)
         if not s.dense:
             _lib.misa_pool_keys(K, s.B, k_scale=ks, kbar_hl=self.kbar_hl, want_kbar=False)
+        Ks = self._scoring_keys(K, ks)
         for i, ((c0, c1), e) in enumerate(zip(bounds, ev_in)):
             compute.wait_event(e)
             if not s.dense:
                 _lib.misa_route_heads(Q[c0:c1], w[c0:c1], self.kbar_hl, s.q_pos0 + c0, s.n_k,
                                       s.B, s.h, heads=self.heads[c0:c1])
             for a0 in range(c0, c1, self.sub):
-                self._select(a0, min(c1, a0 + self.sub), Q, K, w, ks)
+                self._select(a0, min(c1, a0 + self.sub), Q, K, w, ks, Ks)
             done = torch.cuda.Event()
             done.record(compute)
             mark(f"piece {i} indexed", compute)

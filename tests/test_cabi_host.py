@@ -160,6 +160,41 @@ def test_paged_arguments_rejected_before_launch(lib):
     assert rr(p, p, *good, p, 16, 4, 0, 100, 64, 128, 32, p, p, None, 0, None) == INV
 
 
+def test_scaled_bf16_keys_and_their_decode_rejected_before_launch(lib):
+    so = _so(lib)
+    p = ctypes.c_void_p(16 * 1024)
+    q = ctypes.c_void_p(64 * 1024 * 1024)    # far from p: no overlap
+    odd = ctypes.c_void_p(16 * 1024 + 2)
+    INV, UNS = lib.MISA_ERR_INVALID_ARG, lib.MISA_ERR_UNSUPPORTED
+    SC = lib.MISA_K_BF16_SCALED
+    # decode: null or misaligned buffers, overlapping buffers, d unsupported, n_k < 0
+    dec = so.misa_keys_e4m3_to_bf16
+    assert dec(None, 100, 128, q, None) == INV
+    assert dec(p, 100, 128, None, None) == INV
+    assert dec(odd, 100, 128, q, None) == INV
+    assert dec(p, 100, 128, odd, None) == INV
+    assert dec(p, 100, 128, ctypes.c_void_p(16 * 1024 + 4096), None) == INV
+    assert dec(p, 100, 96, q, None) == UNS
+    assert dec(p, -1, 128, q, None) == INV
+    assert dec(p, 0, 128, q, None) == 0
+    # scaled bf16 keys: the fused call needs their scales; paged caches and the
+    # other calls refuse the key type
+    assert so.misa_score_topk(p, p, p, p, None, SC, 10, 8000, 9000, 64, 128, 8, 64, p, p, 9000,
+                              p, 1 << 30, None) == INV
+    assert so.misa_score_topk(p, p, p, p, odd, SC, 10, 8000, 9000, 64, 128, 8, 64, p, p, 9000,
+                              p, 1 << 30, None) == INV
+    assert so.misa_score_topk(p, p, p, p, p, SC, 10, 8000, 9000, 64, 128, 8, 64, p, p, 9000,
+                              None, 0, None) == lib.MISA_ERR_WORKSPACE
+    assert so.misa_score_topk(p, p, p, p, p, SC, 0, 8000, 9000, 64, 128, 8, 64, p, p, 9000,
+                              None, 0, None) == 0
+    assert so.misa_score_topk_paged(p, p, p, p, p, SC, p, 64, 100, 10, 8000, 9000, 64, 128, 8, 64,
+                                    p, p, 9000, p, 1 << 30, None) == INV
+    assert so.misa_score_tokens(p, p, p, p, p, SC, 10, 0, 100, 64, 128, 8, p, 100, None) == INV
+    assert so.misa_pool_keys(p, p, SC, 128, 128, 64, p, p, None) == INV
+    assert so.misa_rerank(p, p, p, p, SC, p, 16, 4, 0, 100, 64, 128, 8, p, None, p, 1 << 20,
+                          None) == INV
+
+
 def test_empty_work_is_a_no_op(lib):
     so = _so(lib)
     p = ctypes.c_void_p(16 * 1024)

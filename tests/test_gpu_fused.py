@@ -208,3 +208,50 @@ def test_score_topk_long_kept_lists(lib):
     want, _ = _unfused(lib, Qg, wg, heads, Kg, q_pos0, k)
     assert np.array_equal(got, want)
     assert flags[0] == 0 and not flags[1:].any()    # no repair: the list held them
+
+
+def test_e4m3_key_decode_is_exact(lib):
+    # every e4m3 code (the NaN codes included) decodes to the bf16 code of its value
+    codes = np.tile(np.arange(256, dtype=np.uint8), 3).reshape(6, 128)
+    got = lib.misa_keys_e4m3_to_bf16(dev(codes)).cpu().numpy().view(np.uint16)
+    want = oracle.e4m3_keys_to_f64(codes, np.ones(6, dtype=np.float32))
+    assert np.array_equal(oracle.bf16_to_f64(got), want, equal_nan=True)
+
+
+@pytest.mark.parametrize("n_q,q_pos0,n_k,k", [(200, 12000, 14000, 256),   # fused
+                                              (129, 20000, 24000, 2048),  # fused
+                                              (64, 1000, 1100, 64)])      # unfused shape
+def test_score_topk_decoded_fp8_keys_equal_e4m3_keys(lib, n_q, q_pos0, n_k, k):
+    # e4m3 keys decoded once and scored as scaled bf16 keys (what the indexer does
+    # for every query piece) select what the e4m3 keys themselves select
+    wl, inp, g = _inputs(n_q, q_pos0, n_k, 64, 128, 128, 8, k, seed=n_k + k, fp8=True)
+    heads = _heads(lib, g, wl, True)
+    Kd = lib.misa_keys_e4m3_to_bf16(g["K8"])
+    got, flags = _fused(lib, g["Q"], g["w"], heads, Kd, q_pos0, k, k_scale=g["k_scale"])
+    want, _ = _fused(lib, g["Q"], g["w"], heads, g["K8"], q_pos0, k, k_scale=g["k_scale"])
+    assert np.array_equal(got, want)
+    lg = lib.misa_score_tokens(g["Q"], g["w"], heads, g["K8"], q_pos0, k_scale=g["k_scale"])
+    lg_np = lg.cpu().numpy()
+    for t in (0, n_q // 2, n_q - 1):
+        assert np.array_equal(got[t], oracle.topk(lg_np[t:t + 1], q_pos0 + t, n_k, k)[0])
+
+
+def test_indexer_fp8_pieces_equal_whole_chunk(lib):
+    # the indexer decodes the e4m3 keys once per chunk; every piece schedule of the
+    # host pipeline and sub-chunking gives the whole-chunk result
+    from long_context_sparse_block_b200.indexer import IndexerShape, MisaIndexer
+    n_q, q_pos0, n_k, H, d, B, h, k = 300, 9000, 9300, 64, 128, 128, 8, 512
+    wl, inp, g = _inputs(n_q, q_pos0, n_k, H, d, B, h, k, seed=61, fp8=True)
+    shape = IndexerShape(n_q, q_pos0, n_k, H, d, B, h, k)
+    want = MisaIndexer(shape).run(g["Q"], g["K8"], g["w"], k_scale=g["k_scale"]).cpu().numpy()
+    lg = lib.misa_score_tokens(g["Q"], g["w"], _heads(lib, g, wl, True), g["K8"], q_pos0,
+                               k_scale=g["k_scale"]).cpu().numpy()
+    assert np.array_equal(want[7], oracle.topk(lg[7:8], q_pos0 + 7, n_k, k)[0])
+    sub = MisaIndexer(IndexerShape(n_q, q_pos0, n_k, H, d, B, h, k, sub_chunk=128))
+    assert np.array_equal(sub.run(g["Q"], g["K8"], g["w"], k_scale=g["k_scale"]).cpu().numpy(),
+                          want)
+    Qh, K8h, wh, ksh = (t.cpu().pin_memory() for t in (g["Q"], g["K8"], g["w"], g["k_scale"]))
+    for pieces in (None, 3, [100, 50, 150]):
+        out = MisaIndexer(shape).run_host(Qh, K8h, wh, k_scale_h=ksh, pieces=pieces)
+        torch.cuda.current_stream().synchronize()
+        assert np.array_equal(out.numpy(), want)
