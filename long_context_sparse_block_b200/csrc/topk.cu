@@ -811,6 +811,40 @@ struct ListSrc16 {
   }
 };
 
+__device__ __forceinline__ uint32_t entry_pos(const ListSrc& s, uint32_t i) { return s.poss[i]; }
+__device__ __forceinline__ uint32_t entry_pos(const ListSrc16& s, uint32_t i) { return s.pos(i); }
+
+// ordered_select over a list of at most 65535 entries with a single block
+// scan: each thread takes a contiguous run of entries, so the runs' counts in
+// thread order give every kept entry its slot in list order.
+template <class Src, class Emit>
+__device__ uint32_t ordered_select_runs(const Src& src, uint32_t T, uint32_t need, const Emit& emit,
+                                        SmemCtl& sc) {
+  const uint32_t n = static_cast<uint32_t>(src.n);
+  const uint32_t per = (n + kTopkThreads - 1) / kTopkThreads;
+  const uint32_t i0 = min(threadIdx.x * per, n), i1 = min(i0 + per, n);
+  uint32_t gt = 0, eq = 0;
+  for (uint32_t i = i0; i < i1; ++i) {
+    const uint32_t key = src.keys[i];
+    gt += key > T;
+    eq += key == T && key != 0u;
+  }
+  uint32_t total;
+  const uint32_t excl = block_excl_scan(gt | (eq << 16), sc, total);
+  uint32_t eq_rank = excl >> 16;
+  uint32_t slot = (excl & 0xFFFFu) + min(eq_rank, need);
+  for (uint32_t i = i0; i < i1; ++i) {
+    const uint32_t key = src.keys[i];
+    if (key > T) {
+      emit(slot++, key, entry_pos(src, i));
+    } else if (key == T && key != 0u) {
+      if (eq_rank < need) emit(slot++, key, entry_pos(src, i));
+      ++eq_rank;
+    }
+  }
+  return (total & 0xFFFFu) + min(total >> 16, need);
+}
+
 // Per row: the exact top-k among the logits the select-mode scoring kept (the
 // bits of the row's pass mask; their values stored in place).  They hold the
 // whole top-k whenever at least min(k, visible) of them passed.  Rows short of
@@ -919,12 +953,12 @@ fused_finish_kernel(const float* __restrict__ logits, int64_t ld, const uint32_t
   if constexpr (P16) {
     if (total > static_cast<uint32_t>(k))
       T = kth_largest_spread<ListSrc16, true>(ls16, static_cast<uint32_t>(k), hist, sc, need);
-    kept = ordered_select(ls16, T, need, static_cast<uint32_t>(k), out, sc);
+    kept = ordered_select_runs(ls16, T, need, out, sc);
   } else {
     const ListSrc ls{keys, reinterpret_cast<const uint32_t*>(poss), static_cast<int64_t>(total)};
     if (total > static_cast<uint32_t>(k))
       T = kth_largest_spread<ListSrc, true>(ls, static_cast<uint32_t>(k), hist, sc, need);
-    kept = ordered_select(ls, T, need, static_cast<uint32_t>(k), out, sc);
+    kept = ordered_select_runs(ls, T, need, out, sc);
   }
   for (uint32_t i = min(kept, static_cast<uint32_t>(k)) + threadIdx.x; i < static_cast<uint32_t>(k);
        i += kTopkThreads)
