@@ -255,6 +255,13 @@ def test_binding_refuses_undersized_buffers(lib):
     size_error(lib.misa_rerank, Q, w, K, torch.zeros((n_q - 1, 32), dtype=torch.int32), 0, k)
     size_error(lib.misa_score_topk, Q, w, heads, K, 0, k, h=h,
                idx=torch.zeros((n_q, k - 1), dtype=torch.int32), logits=lg)
+    # decoded FP8 keys: bf16 codes that come with scales need one per key
+    size_error(lib.misa_score_topk, Q, w, heads, K, 0, k, h=h, k_scale=torch.ones(n_k - 1),
+               logits=lg)
+    size_error(lib.misa_keys_e4m3_to_bf16, K.to(torch.uint8), out=torch.zeros((n_k - 1, d),
+                                                                             dtype=torch.int16))
+    device_error(lib.misa_keys_e4m3_to_bf16, K.to(torch.uint8),
+                 out=torch.zeros((n_k, d), dtype=torch.int16))
 
 
 def test_binding_checks_pass_for_well_sized_buffers(lib):
