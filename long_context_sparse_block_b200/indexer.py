@@ -105,8 +105,9 @@ class MisaIndexer:
         """The keys the fused scoring reads: e4m3 keys decoded to bf16 codes once
         per chunk (scored with their scales), so that every query sub-chunk or
         piece does not decode them again; bf16 keys as they are."""
-        if k_scale is None or K.dtype not in (torch.uint8, torch.float8_e4m3fn):
-            return K
+        if (k_scale is None or not isinstance(K, torch.Tensor)
+                or K.dtype not in (torch.uint8, torch.float8_e4m3fn)):
+            return K  # bf16 keys, or a paged cache (decoded inside the fused call)
         kd = getattr(self, "_kdec", None)
         if kd is None or kd.shape != K.shape or kd.device != K.device:
             kd = self._kdec = torch.empty(K.shape, dtype=torch.int16, device=K.device)
