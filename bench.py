@@ -821,7 +821,7 @@ def main():
             print(json.dumps(out), flush=True)
         return
 
-    # the oracle's process pool is spawned before any CUDA work
+    # the oracle's process pool is forked before any CUDA work (a fork after it would hang)
     wl = _workload(args)
     inp = W.generate(W.WORKLOADS[args.workload])  # each rank indexes its own chunk (same shape)
     if wl.n_q < inp["Q"].shape[0]:
