@@ -199,8 +199,9 @@ int misa_rerank_noalloc(const uint16_t* Q, const float* w, const void* K, const 
  * per-row threshold from it, stores only the logits at or above the threshold
  * (a few k per row, flagged in a per-row bit mask) while scoring, and selects
  * exactly among them.  Rows whose threshold kept fewer than min(k, visible)
- * logits, or more than max(6144, 3k), are recomputed by the unfused sequence,
- * so the result is exact for every input.
+ * logits, or more than the finish's list holds (max(6144, 3k) entries up to
+ * k = 4096, 2k above, rounded up to a multiple of 1024), are recomputed by the
+ * unfused sequence, so the result is exact for every input.
  *   logits [n_q, ld]: scratch for the kept logits and the fallback (contents
  *     unspecified afterwards; ld >= n_k, a multiple of 4, 16-byte aligned).
  *   ws/ws_bytes: misa_workspace_size("score_topk", n_q, n_k, k, 0) bytes,
