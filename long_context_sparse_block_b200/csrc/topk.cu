@@ -816,12 +816,13 @@ __device__ __forceinline__ uint32_t entry_pos(const ListSrc16& s, uint32_t i) { 
 
 // ordered_select over a list of at most 65535 entries with a single block
 // scan: each thread takes a contiguous run of entries, so the runs' counts in
-// thread order give every kept entry its slot in list order.
+// thread order give every kept entry its slot in list order.  The run length
+// is odd, so a warp's lanes read 32 different shared-memory banks.
 template <class Src, class Emit>
 __device__ uint32_t ordered_select_runs(const Src& src, uint32_t T, uint32_t need, const Emit& emit,
                                         SmemCtl& sc) {
   const uint32_t n = static_cast<uint32_t>(src.n);
-  const uint32_t per = (n + kTopkThreads - 1) / kTopkThreads;
+  const uint32_t per = ((n + kTopkThreads - 1) / kTopkThreads) | 1u;
   const uint32_t i0 = min(threadIdx.x * per, n), i1 = min(i0 + per, n);
   uint32_t gt = 0, eq = 0;
   for (uint32_t i = i0; i < i1; ++i) {
